@@ -1,0 +1,12 @@
+"""Gated delta-rule decode step on B200 (sm_100a): eager and DeltaLog-deferred.
+
+The compute path is libdeltalog.so (CUDA kernels behind the C ABI in
+include/deltalog.h); this package is its Python binding plus the host-side
+schedule driver. PyTorch provides device memory and streams only.
+"""
+from ._binding import (  # noqa: F401
+    DL_BF16, DL_DECAY_CHANNEL, DL_DECAY_HEAD, DL_F32, DL_MAX_LOG, EXPORTS, DeltaLogError, Log,
+    dl_gdn_decode_step, dl_kda_decode_step, dl_log_append_read, dl_log_merge, dl_log_merge_read,
+    dl_status_string, load,
+)
+from .schedule import DeferredDecoder  # noqa: F401

@@ -1,0 +1,223 @@
+"""ctypes binding of libdeltalog.so (include/deltalog.h).
+
+Argument marshalling only: every function here checks that the tensors are
+CUDA, contiguous and of a supported dtype, reads their shapes, and passes raw
+device pointers, sizes and the stream to the C ABI. All arithmetic runs in the
+library's CUDA kernels. There is no fallback: a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdeltalog.so")
+
+DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = range(5)
+DL_F32, DL_BF16 = 0, 1
+DL_DECAY_HEAD, DL_DECAY_CHANNEL = 0, 1
+DL_MAX_LOG = 64
+ABI_VERSION = 1
+
+EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
+           "dl_log_merge_read", "dl_status_string", "dl_last_error", "dl_abi_version")
+
+
+class DeltaLogError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn}: status {status} ({_status_name(status)}): {message}")
+        self.status = status
+
+
+class dl_log(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("a", ctypes.c_void_p), ("dtype", ctypes.c_int), ("L", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libdeltalog.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libdeltalog.so not found at {p}: build it with "
+                           "`python -m gated_delta_rule_104_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(p)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    step = [vp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    lib.dl_gdn_decode_step.argtypes = step
+    lib.dl_kda_decode_step.argtypes = step
+    lp = ctypes.POINTER(dl_log)
+    lib.dl_log_append_read.argtypes = [vp, i, i, lp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    lib.dl_log_merge_read.argtypes = [vp, i, i, lp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    lib.dl_log_merge.argtypes = [vp, i, i, lp, i, i, i, i, i, vp]
+    for name in ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
+                 "dl_log_merge_read"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.dl_status_string.argtypes = [ctypes.c_int]
+    lib.dl_status_string.restype = ctypes.c_char_p
+    lib.dl_last_error.argtypes = []
+    lib.dl_last_error.restype = ctypes.c_char_p
+    lib.dl_abi_version.argtypes = []
+    lib.dl_abi_version.restype = ctypes.c_int
+    if lib.dl_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"libdeltalog.so ABI {lib.dl_abi_version()} != binding ABI {ABI_VERSION}: rebuild")
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _status_name(s: int) -> str:
+    return {0: "DL_OK", 1: "DL_ERR_INVALID_ARG", 2: "DL_ERR_UNSUPPORTED", 3: "DL_ERR_LOG_FULL",
+            4: "DL_ERR_CUDA"}.get(s, "?")
+
+
+def check(fn: str, status: int) -> None:
+    if status != DL_OK:
+        msg = load().dl_last_error().decode(errors="replace")
+        raise DeltaLogError(fn, status, msg)
+
+
+# ------------------------------------------------------------------ tensors
+
+def _torch():
+    import torch  # device memory and streams only
+
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return DL_F32
+    if t.dtype == torch.bfloat16:
+        return DL_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t, name: str) -> int:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return _torch().cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dims(S):
+    if S.dim() != 4:
+        raise ValueError("state must be [B, H, d_v, d_k]")
+    B, H, dv, dk = S.shape
+    return int(B), int(H), int(dk), int(dv)
+
+
+def _in_dtype(*ts) -> int:
+    codes = {_dtype_code(t) for t in ts}
+    if len(codes) != 1:
+        raise TypeError("q, k, v, beta and a must share one dtype")
+    return codes.pop()
+
+
+def _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, chan):
+    exp = {"q": (q, B * H * dk), "k": (k, B * H * dk), "v": (v, B * H * dv), "beta": (beta, B * H),
+           "a": (a, B * H * (dk if chan else 1)), "o": (o, B * H * dv)}
+    for name, (t, n) in exp.items():
+        if t.numel() != n:
+            raise ValueError(f"{name} has {t.numel()} elements, expected {n}")
+    if o.dtype != _torch().float32:
+        raise TypeError("o must be float32")
+
+
+def dl_gdn_decode_step(S, q, k, v, beta, a, o, stream=None) -> None:
+    """Eager GDN step in place on S [B,H,d_v,d_k]; o [B,H,d_v] float32."""
+    _eager("dl_gdn_decode_step", S, q, k, v, beta, a, o, stream, chan=False)
+
+
+def dl_kda_decode_step(S, q, k, v, beta, a, o, stream=None) -> None:
+    """Eager KDA step (a [B,H,d_k]) in place on S; o [B,H,d_v] float32."""
+    _eager("dl_kda_decode_step", S, q, k, v, beta, a, o, stream, chan=True)
+
+
+def _eager(fn, S, q, k, v, beta, a, o, stream, chan):
+    B, H, dk, dv = _dims(S)
+    _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, chan)
+    st = _stream(stream)
+    status = getattr(load(), fn)(_ptr(S, "S"), _dtype_code(S), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                 _ptr(beta, "beta"), _ptr(a, "a"), _in_dtype(q, k, v, beta, a),
+                                 _ptr(o, "o"), B, H, dk, dv, st)
+    check(fn, status)
+
+
+class Log:
+    """Caller-owned bounded log buffers of a deferred state (device tensors):
+    k [B,H,L,d_k], v [B,H,L,d_v], beta [B,H,L], a [B,H,L] or [B,H,L,d_k]."""
+
+    def __init__(self, k, v, beta, a, L: int, channel_decay: bool):
+        self.k, self.v, self.beta, self.a = k, v, beta, a
+        self.L = int(L)
+        self.channel_decay = bool(channel_decay)
+        self.dtype = _in_dtype(k, v, beta, a)
+
+    @classmethod
+    def allocate(cls, B, H, d_k, d_v, L, dtype, channel_decay, device="cuda"):
+        torch = _torch()
+        z = lambda *s: torch.zeros(*s, dtype=dtype, device=device)  # noqa: E731
+        a = z(B, H, L, d_k) if channel_decay else z(B, H, L)
+        return cls(z(B, H, L, d_k), z(B, H, L, d_v), z(B, H, L), a, L, channel_decay)
+
+    def struct(self) -> dl_log:
+        return dl_log(_ptr(self.k, "log.k"), _ptr(self.v, "log.v"), _ptr(self.beta, "log.beta"),
+                      _ptr(self.a, "log.a"), self.dtype, self.L)
+
+    @property
+    def kind(self) -> int:
+        return DL_DECAY_CHANNEL if self.channel_decay else DL_DECAY_HEAD
+
+
+def dl_log_append_read(S_base, log: Log, n: int, q, k, v, beta, a, o, stream=None) -> None:
+    """Append entry n and read o from base + log (base not written)."""
+    _log_step("dl_log_append_read", S_base, log, n, q, k, v, beta, a, o, stream)
+
+
+def dl_log_merge_read(S_base, log: Log, n: int, q, k, v, beta, a, o, stream=None) -> None:
+    """Merge log entries 0..n-1 plus this step into the base; o = new base q."""
+    _log_step("dl_log_merge_read", S_base, log, n, q, k, v, beta, a, o, stream)
+
+
+def _log_step(fn, S, log, n, q, k, v, beta, a, o, stream):
+    B, H, dk, dv = _dims(S)
+    _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, log.channel_decay)
+    st = _stream(stream)
+    ls = log.struct()
+    status = getattr(load(), fn)(_ptr(S, "S_base"), _dtype_code(S), log.kind, ctypes.byref(ls), int(n),
+                                 _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(beta, "beta"), _ptr(a, "a"),
+                                 _in_dtype(q, k, v, beta, a), _ptr(o, "o"), B, H, dk, dv, st)
+    check(fn, status)
+
+
+def dl_log_merge(S_base, log: Log, n: int, stream=None) -> None:
+    """Merge log entries 0..n-1 into the base in place."""
+    B, H, dk, dv = _dims(S_base)
+    st = _stream(stream)
+    ls = log.struct()
+    status = load().dl_log_merge(_ptr(S_base, "S_base"), _dtype_code(S_base), log.kind, ctypes.byref(ls),
+                                 int(n), B, H, dk, dv, st)
+    check("dl_log_merge", status)
+
+
+def dl_status_string(status: int) -> str:
+    return load().dl_status_string(int(status)).decode()

@@ -1,0 +1,220 @@
+// C-ABI layer of libdeltalog: host-side argument checks (before any CUDA
+// call), then dispatch to the kernels. Declarations and the contract of each
+// entry point are in include/deltalog.h.
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "launch.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+dl_status fail(dl_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+dl_status ok() {
+    g_err[0] = '\0';
+    return DL_OK;
+}
+
+size_t elem_size(dl_dtype t) { return t == DL_BF16 ? 2 : 4; }
+bool valid_dtype(int t) { return t == DL_F32 || t == DL_BF16; }
+bool valid_decay(int t) { return t == DL_DECAY_HEAD || t == DL_DECAY_CHANNEL; }
+
+struct Buf {
+    const char *name;
+    const void *p;
+    size_t bytes;
+    size_t align;
+};
+
+bool overlaps(const Buf &a, const Buf &b) {
+    if (!a.p || !b.p || !a.bytes || !b.bytes) return false;
+    const uintptr_t a0 = (uintptr_t)a.p, b0 = (uintptr_t)b.p;
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+dl_status check_bufs(const Buf *bufs, int nb) {
+    for (int i = 0; i < nb; ++i) {
+        if (!bufs[i].p) return fail(DL_ERR_INVALID_ARG, "%s is a null pointer", bufs[i].name);
+        if ((uintptr_t)bufs[i].p % bufs[i].align)
+            return fail(DL_ERR_INVALID_ARG, "%s is not %zu-byte aligned", bufs[i].name, bufs[i].align);
+    }
+    return DL_OK;
+}
+
+// Writers must not overlap anything else in the call.
+dl_status check_overlap(const Buf *writers, int nw, const Buf *all, int na) {
+    for (int i = 0; i < nw; ++i)
+        for (int j = 0; j < na; ++j) {
+            if (writers[i].p == all[j].p && writers[i].name == all[j].name) continue;
+            if (overlaps(writers[i], all[j]))
+                return fail(DL_ERR_INVALID_ARG, "%s overlaps %s", writers[i].name, all[j].name);
+        }
+    return DL_OK;
+}
+
+dl_status check_dims(int B, int H, int dk, int dv, int s_dt, int in_dt) {
+    if (B < 1 || H < 1) return fail(DL_ERR_INVALID_ARG, "B and H must be >= 1 (got B=%d, H=%d)", B, H);
+    if ((long long)B * H > (1LL << 26)) return fail(DL_ERR_UNSUPPORTED, "B*H=%lld exceeds 2^26", (long long)B * H);
+    if (!valid_dtype(s_dt)) return fail(DL_ERR_INVALID_ARG, "unknown state dtype %d", s_dt);
+    if (!valid_dtype(in_dt)) return fail(DL_ERR_INVALID_ARG, "unknown input dtype %d", in_dt);
+    if (dk != 64 && dk != 128) return fail(DL_ERR_UNSUPPORTED, "d_k=%d not in {64, 128}", dk);
+    if (dv != 64 && dv != 128 && dv != 256) return fail(DL_ERR_UNSUPPORTED, "d_v=%d not in {64, 128, 256}", dv);
+    return DL_OK;
+}
+
+// Step operands: S, q, k, v, beta, a, o (indices fixed for the callers).
+int step_bufs(Buf *out, const void *S, const char *sname, dl_dtype s_dt, const void *q, const void *k,
+              const void *v, const void *beta, const void *a, dl_dtype in_dt, const float *o, int B,
+              int H, int dk, int dv, bool chan) {
+    const size_t bh = (size_t)B * H, is = elem_size(in_dt);
+    out[0] = {sname, S, bh * dv * dk * elem_size(s_dt), 16};
+    out[1] = {"q", q, bh * dk * is, 16};
+    out[2] = {"k", k, bh * dk * is, 16};
+    out[3] = {"v", v, bh * dv * is, 16};
+    out[4] = {"beta", beta, bh * is, is};
+    out[5] = chan ? Buf{"a", a, bh * dk * is, 16} : Buf{"a", a, bh * is, is};
+    out[6] = {"o", o, bh * dv * sizeof(float), 16};
+    return 7;
+}
+
+dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, int dk, int dv, bool chan) {
+    if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
+    if (!valid_dtype(log->dtype)) return fail(DL_ERR_INVALID_ARG, "unknown log dtype %d", (int)log->dtype);
+    if (log->L < 1 || log->L > DL_MAX_LOG)
+        return fail(DL_ERR_UNSUPPORTED, "log capacity L=%d not in 1..%d", log->L, DL_MAX_LOG);
+    if (log->dtype != in_dt) return fail(DL_ERR_UNSUPPORTED, "log dtype differs from the input dtype");
+    const size_t bhl = (size_t)B * H * log->L, is = elem_size(in_dt);
+    out[0] = {"log.k", log->k, bhl * dk * is, 16};
+    out[1] = {"log.v", log->v, bhl * dv * is, 16};
+    out[2] = {"log.beta", log->beta, bhl * is, is};
+    out[3] = chan ? Buf{"log.a", log->a, bhl * dk * is, 16} : Buf{"log.a", log->a, bhl * is, is};
+    return DL_OK;
+}
+
+dl_status cuda_status(cudaError_t e, const char *what) {
+    if (e != cudaSuccess) return fail(DL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+dl_status eager_step(void *S, dl_dtype s_dt, const void *q, const void *k, const void *v, const void *beta,
+                     const void *a, dl_dtype in_dt, float *o, int B, int H, int dk, int dv,
+                     cudaStream_t stream, bool chan) {
+    dl_status s = check_dims(B, H, dk, dv, s_dt, in_dt);
+    if (s != DL_OK) return s;
+    Buf b[7];
+    int nb = step_bufs(b, S, "S", s_dt, q, k, v, beta, a, in_dt, o, B, H, dk, dv, chan);
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    const Buf writers[2] = {b[0], b[6]};  // S and o are written
+    if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
+    dl::StepParams p{S, q, k, v, beta, a, o, B, H, dk, dv, chan, s_dt, in_dt};
+    return cuda_status(dl::launch_eager(p, stream), "eager step launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+dl_status dl_gdn_decode_step(void *S, dl_dtype s_dtype, const void *q, const void *k, const void *v,
+                             const void *beta, const void *a, dl_dtype in_dtype, float *o, int B, int H,
+                             int d_k, int d_v, cudaStream_t stream) {
+    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, false);
+}
+
+dl_status dl_kda_decode_step(void *S, dl_dtype s_dtype, const void *q, const void *k, const void *v,
+                             const void *beta, const void *a, dl_dtype in_dtype, float *o, int B, int H,
+                             int d_k, int d_v, cudaStream_t stream) {
+    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, true);
+}
+
+dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log, int n,
+                             const void *q, const void *k, const void *v, const void *beta, const void *a,
+                             dl_dtype in_dtype, float *o, int B, int H, int d_k, int d_v,
+                             cudaStream_t stream) {
+    dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
+    if (s != DL_OK) return s;
+    if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
+    const bool chan = kind == DL_DECAY_CHANNEL;
+    Buf b[11];
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    nb += 4;
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
+    // written: o and the log (slot n); the base is only read.
+    const Buf writers[5] = {b[6], b[7], b[8], b[9], b[10]};
+    if ((s = check_overlap(writers, 5, b, nb)) != DL_OK) return s;
+    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    return cuda_status(dl::launch_append_read(p, lg, n, stream), "append-read launch");
+}
+
+dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log, int n, int B, int H,
+                       int d_k, int d_v, cudaStream_t stream) {
+    dl_status s = check_dims(B, H, d_k, d_v, s_dtype, log ? (int)log->dtype : (int)DL_F32);
+    if (s != DL_OK) return s;
+    if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
+    const bool chan = kind == DL_DECAY_CHANNEL;
+    if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
+    Buf b[5];
+    b[0] = {"S_base", S_base, (size_t)B * H * d_v * d_k * elem_size(s_dtype), 16};
+    if ((s = check_log(log, b + 1, log->dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    if ((s = check_bufs(b, 5)) != DL_OK) return s;
+    if (n < 1 || n > log->L) return fail(DL_ERR_INVALID_ARG, "merge needs 1 <= n <= L (n=%d, L=%d)", n, log->L);
+    const Buf writers[1] = {b[0]};
+    if ((s = check_overlap(writers, 1, b, 5)) != DL_OK) return s;
+    const Buf logw[4] = {b[1], b[2], b[3], b[4]};
+    if ((s = check_overlap(logw, 4, b + 1, 4)) != DL_OK) return s;
+    dl::StepParams p{S_base, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, chan,
+                     s_dtype, log->dtype};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    return cuda_status(dl::launch_merge(p, lg, n, false, stream), "merge launch");
+}
+
+dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log, int n,
+                            const void *q, const void *k, const void *v, const void *beta, const void *a,
+                            dl_dtype in_dtype, float *o, int B, int H, int d_k, int d_v,
+                            cudaStream_t stream) {
+    dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
+    if (s != DL_OK) return s;
+    if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
+    const bool chan = kind == DL_DECAY_CHANNEL;
+    Buf b[11];
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    nb += 4;
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
+    const Buf writers[2] = {b[0], b[6]};  // the base and o
+    if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
+    dl::StepParams p{S_base, q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    return cuda_status(dl::launch_merge(p, lg, n, true, stream), "merge-read launch");
+}
+
+const char *dl_status_string(dl_status s) {
+    switch (s) {
+        case DL_OK: return "ok";
+        case DL_ERR_INVALID_ARG: return "invalid argument";
+        case DL_ERR_UNSUPPORTED: return "unsupported size or dtype";
+        case DL_ERR_LOG_FULL: return "log full";
+        case DL_ERR_CUDA: return "CUDA launch error";
+    }
+    return "unknown status";
+}
+
+const char *dl_last_error(void) { return g_err; }
+
+int dl_abi_version(void) { return DL_ABI_VERSION; }
+
+}  // extern "C"

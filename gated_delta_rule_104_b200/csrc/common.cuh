@@ -1,0 +1,143 @@
+// Shared device helpers for the decode-step kernels: element types, widening
+// vector loads, bf16 packing and group reductions. sm_100a only.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dl {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------- scalars
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+
+// bf16 bit pattern (low / high half of a 32-bit word) widened exactly.
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two floats rounded to nearest-even bf16, packed (first in the low half).
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// ---------------------------------------------------------------- loads
+
+// N consecutive elements of T at p (aligned to N * sizeof(T) bytes, at most
+// 16) widened to float. Plain cached loads (small, reused operands).
+template <int N>
+__device__ __forceinline__ void load_vec(const float *p, float (&x)[N]) {
+    static_assert(N % 2 == 0, "even");
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            float4 v = *reinterpret_cast<const float4 *>(p + i);
+            x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 2) {
+            float2 v = *reinterpret_cast<const float2 *>(p + i);
+            x[i] = v.x; x[i + 1] = v.y;
+        }
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void load_vec(const bf16 *p, float (&x)[N]) {
+    static_assert(N % 2 == 0, "even");
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 8) {
+            uint4 v = *reinterpret_cast<const uint4 *>(p + i);
+            x[i] = bf_lo(v.x); x[i + 1] = bf_hi(v.x);
+            x[i + 2] = bf_lo(v.y); x[i + 3] = bf_hi(v.y);
+            x[i + 4] = bf_lo(v.z); x[i + 5] = bf_hi(v.z);
+            x[i + 6] = bf_lo(v.w); x[i + 7] = bf_hi(v.w);
+        }
+    } else if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            uint2 v = *reinterpret_cast<const uint2 *>(p + i);
+            x[i] = bf_lo(v.x); x[i + 1] = bf_hi(v.x);
+            x[i + 2] = bf_lo(v.y); x[i + 3] = bf_hi(v.y);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 2) {
+            uint32_t v = *reinterpret_cast<const uint32_t *>(p + i);
+            x[i] = bf_lo(v); x[i + 1] = bf_hi(v);
+        }
+    }
+}
+
+// 16-byte state vectors: 4 floats or 8 bf16 held in a uint4.
+template <class ST> struct StateVec;
+template <> struct StateVec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void unpack(const uint4 &r, float (&x)[4]) {
+        x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
+        x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&x)[4]) {
+        return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]),
+                          __float_as_uint(x[2]), __float_as_uint(x[3]));
+    }
+};
+template <> struct StateVec<bf16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &r, float (&x)[8]) {
+        x[0] = bf_lo(r.x); x[1] = bf_hi(r.x); x[2] = bf_lo(r.y); x[3] = bf_hi(r.y);
+        x[4] = bf_lo(r.z); x[5] = bf_hi(r.z); x[6] = bf_lo(r.w); x[7] = bf_hi(r.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&x)[8]) {
+        return make_uint4(pack_bf2(x[0], x[1]), pack_bf2(x[2], x[3]),
+                          pack_bf2(x[4], x[5]), pack_bf2(x[6], x[7]));
+    }
+};
+
+// Streaming 16-byte state accesses: the state is touched once per step, so
+// it is read and written with the evict-first (".cs") cache hint and kept out
+// of L1, leaving L2 to the small per-step operands.
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void st_stream(void *p, const uint4 &v) {
+    __stcs(reinterpret_cast<uint4 *>(p), v);
+}
+// Read-only state (the deferred base between merges): non-coherent path,
+// no L1 allocation.
+__device__ __forceinline__ uint4 ld_ro_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// ---------------------------------------------------------------- reductions
+
+// Sum over aligned groups of G consecutive lanes (G a power of two <= 32);
+// every lane of the group receives the group's sum.
+template <int G>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+    for (int off = G / 2; off > 0; off >>= 1)
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// ---------------------------------------------------------------- async copy
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+    uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+}  // namespace dl

@@ -1,0 +1,166 @@
+/*
+ * deltalog.h -- C ABI of the gated delta-rule decode-step library (sm_100a).
+ *
+ * The operation (DeltaLog: Deferred Materialization of Recurrent States for
+ * Linear Attention Decoding, Technical Summary, "Problem" and "Kernel
+ * Implementation"): for each sequence b < B and head h < H, a recurrent state
+ * S in R^{d_v x d_k} is advanced by one decode step with q, k in R^{d_k},
+ * v in R^{d_v}, a scalar beta and a decay a,
+ *
+ *     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,
+ *
+ * where the decay is one scalar per head for Gated DeltaNet (GDN) and one
+ * value per key channel for Kimi Delta Attention (KDA).
+ *
+ * Two schedules:
+ *   eager     -- dl_gdn_decode_step / dl_kda_decode_step read S, apply the
+ *                step and write S back every token (section "Problem: The
+ *                State-Update Tax").
+ *   deferred  -- the DeltaLog schedule (section "Methodology", "Core
+ *                Mechanism: Base + Log" and "Traffic Model"): a dense base
+ *                S_bar is left unwritten while each step appends its factors
+ *                (k, v, beta, a) to a bounded per-head log and reads o from
+ *                base + log (dl_log_append_read); once the log is full the
+ *                caller merges it into the base (dl_log_merge), or fuses the
+ *                merge with that step's read (dl_log_merge_read).
+ *
+ * Conventions for every entry point
+ *   Pointers   device pointers (cudaMalloc'd or equivalent), row-major and
+ *              contiguous with the layouts given per argument. S, q, k, v, o,
+ *              a channel-wise decay and the log's k, v and channel-wise a must
+ *              be 16-byte aligned; beta and a head-wise decay need only their
+ *              element alignment. Misaligned -> DL_ERR_INVALID_ARG.
+ *   Element    dl_dtype of S (s_dtype) and of q, k, v, beta, a and the log
+ *   types      (in_dtype; the log's dtype must equal in_dtype). o is float.
+ *   Shapes     B, H >= 1; d_k in {64, 128}; d_v in {64, 128, 256}; log
+ *              capacity L in 1..64. Other sizes -> DL_ERR_UNSUPPORTED.
+ *   Ownership  the caller owns every buffer. The library allocates no device
+ *              memory, keeps no state between calls and never synchronises:
+ *              the work is enqueued on `stream` (0 = legacy default stream).
+ *   Aliasing   o must not overlap any input or S; the log must not overlap S.
+ *              Overlap -> DL_ERR_INVALID_ARG.
+ *   Errors     arguments are checked on the host before anything is enqueued;
+ *              a failed check enqueues nothing and returns its status. A
+ *              launch failure returns DL_ERR_CUDA. Faults during execution
+ *              surface at the caller's next synchronisation. After any
+ *              non-OK return, dl_last_error() describes the cause (per thread).
+ */
+#ifndef DELTALOG_H
+#define DELTALOG_H
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DL_ABI_VERSION 1
+#define DL_MAX_LOG 64
+
+typedef enum {
+    DL_OK = 0,
+    DL_ERR_INVALID_ARG = 1, /* null / misaligned / overlapping pointer, bad enum, B or H < 1, bad n */
+    DL_ERR_UNSUPPORTED = 2, /* d_k, d_v or L outside the supported set; log dtype != in_dtype */
+    DL_ERR_LOG_FULL = 3,    /* append with n >= L (merge first) */
+    DL_ERR_CUDA = 4         /* the kernel launch failed (cudaGetLastError) */
+} dl_status;
+
+typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
+
+typedef enum {
+    DL_DECAY_HEAD = 0,    /* a is one scalar per (b, h, step): GDN */
+    DL_DECAY_CHANNEL = 1  /* a is one value per key channel: KDA  */
+} dl_decay;
+
+/* Caller-owned bounded log of a deferred state: per (b, h) up to L entries of
+ * the raw step factors, stored unchanged in `dtype` (lossless).
+ * (The page's log keeps "compact update factors" plus log-decay metadata,
+ * Technical Summary, "Core Mechanism: Base + Log"; here the metadata is
+ * recomputed from the stored decays where it is needed.)
+ *   k     [B, H, L, d_k]
+ *   v     [B, H, L, d_v]
+ *   beta  [B, H, L]
+ *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL)
+ * The number of valid entries n (the same for every head) is tracked by the
+ * caller and passed to each call; entries 0..n-1 are valid. */
+typedef struct {
+    void *k;
+    void *v;
+    void *beta;
+    void *a;
+    dl_dtype dtype;
+    int L;
+} dl_log;
+
+/* Eager GDN step (head-wise decay), in place.
+ *   S     [B, H, d_v, d_k] s_dtype, read and overwritten with S_t
+ *   q, k  [B, H, d_k] in_dtype      v [B, H, d_v] in_dtype
+ *   beta  [B, H] in_dtype           a [B, H] in_dtype (one decay per head)
+ *   o     [B, H, d_v] float, written with S_t q
+ * A bf16 S is updated in fp32 and rounded to nearest-even when stored. */
+dl_status dl_gdn_decode_step(void *S, dl_dtype s_dtype,
+                             const void *q, const void *k, const void *v,
+                             const void *beta, const void *a, dl_dtype in_dtype,
+                             float *o, int B, int H, int d_k, int d_v,
+                             cudaStream_t stream);
+
+/* Eager KDA step (channel-wise decay): as dl_gdn_decode_step, except
+ *   a     [B, H, d_k] in_dtype (one decay per key channel). */
+dl_status dl_kda_decode_step(void *S, dl_dtype s_dtype,
+                             const void *q, const void *k, const void *v,
+                             const void *beta, const void *a, dl_dtype in_dtype,
+                             float *o, int B, int H, int d_k, int d_v,
+                             cudaStream_t stream);
+
+/* Deferred step: append this step's (k, v, beta, a) to the log as entry n and
+ * write o = S_n q, where S_n is the base with log entries 0..n replayed, read
+ * without materialising it (Technical Summary, "Append Phase" and
+ * "Kernel Implementation": key-side coefficients computed once per head, then
+ * value tiles read the base). S_base is only read.
+ *   S_base [B, H, d_v, d_k] s_dtype (read only)
+ *   log    entries 0..n-1 read, entry n written
+ *   n      entries already in the log, 0 <= n < L; n >= L -> DL_ERR_LOG_FULL
+ *   q, k, v, beta, a, o: as the eager step of the same decay kind. */
+dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind,
+                             const dl_log *log, int n,
+                             const void *q, const void *k, const void *v,
+                             const void *beta, const void *a, dl_dtype in_dtype,
+                             float *o, int B, int H, int d_k, int d_v,
+                             cudaStream_t stream);
+
+/* Merge log entries 0..n-1 into the base in place: S_base <- S_n (Technical
+ * Summary, "Merge Phase"). Afterwards the caller treats the log as empty.
+ *   n      1 <= n <= L, else DL_ERR_INVALID_ARG
+ * A bf16 base is merged in fp32 and rounded once when stored. */
+dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind,
+                       const dl_log *log, int n,
+                       int B, int H, int d_k, int d_v, cudaStream_t stream);
+
+/* The merge fused with a step's read: S_base <- the base with log entries
+ * 0..n-1 and then this step's (k, v, beta, a) replayed, and o = (new S_base) q.
+ * Equivalent to dl_log_append_read(n) followed by dl_log_merge(n + 1), with one
+ * pass over the base instead of two; the log slot n is not written.
+ *   n      entries already in the log, 0 <= n < L; n >= L -> DL_ERR_LOG_FULL */
+dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind,
+                            const dl_log *log, int n,
+                            const void *q, const void *k, const void *v,
+                            const void *beta, const void *a, dl_dtype in_dtype,
+                            float *o, int B, int H, int d_k, int d_v,
+                            cudaStream_t stream);
+
+/* Static text for a status code. */
+const char *dl_status_string(dl_status s);
+
+/* Description of the most recent non-OK return on the calling thread ("" if
+ * none). The pointer stays valid until the thread's next dl_* call. */
+const char *dl_last_error(void);
+
+/* DL_ABI_VERSION of the built library. */
+int dl_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTALOG_H */

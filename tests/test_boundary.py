@@ -1,0 +1,138 @@
+"""Host-only tests of the C ABI (no GPU needed): the library loads, exports
+every entry point include/deltalog.h declares, and rejects bad arguments with
+the documented status before any CUDA call. Only argument checks that fail are
+exercised here, so no kernel is ever launched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_104_b200._binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "deltalog.h")
+
+A = 0x7f0000000000  # fake, 256-byte aligned "device" addresses: never dereferenced
+MB = 1 << 20
+
+
+def addr(i):
+    return A + i * 64 * MB
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return b.load()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(dl_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = header_functions()
+    assert set(declared) == set(b.EXPORTS), declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert lib.dl_abi_version() == b.ABI_VERSION
+
+
+def test_status_strings(lib):
+    assert b.dl_status_string(0) == "ok"
+    assert "log full" in b.dl_status_string(3)
+    assert b.dl_status_string(99) == "unknown status"
+
+
+def step(lib, fn, S=None, s_dt=b.DL_F32, q=None, k=None, v=None, beta=None, a=None, in_dt=b.DL_BF16,
+         o=None, B=2, H=3, dk=128, dv=128):
+    ptrs = [S or addr(0), q or addr(1), k or addr(2), v or addr(3), beta or addr(4), a or addr(5), o or addr(6)]
+    S, q, k, v, beta, a, o = [None if p == -1 else p for p in ptrs]
+    return getattr(lib, fn)(S, s_dt, q, k, v, beta, a, in_dt, o, B, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("fn", ["dl_gdn_decode_step", "dl_kda_decode_step"])
+def test_eager_argument_checks(lib, fn):
+    assert step(lib, fn, S=-1) == b.DL_ERR_INVALID_ARG
+    assert "S is a null pointer" in lib.dl_last_error().decode()
+    assert step(lib, fn, o=-1) == b.DL_ERR_INVALID_ARG
+    assert step(lib, fn, q=addr(1) + 8) == b.DL_ERR_INVALID_ARG          # misaligned vector operand
+    assert "not 16-byte aligned" in lib.dl_last_error().decode()
+    assert step(lib, fn, B=0) == b.DL_ERR_INVALID_ARG
+    assert step(lib, fn, H=-1) == b.DL_ERR_INVALID_ARG
+    assert step(lib, fn, dk=96) == b.DL_ERR_UNSUPPORTED
+    assert step(lib, fn, dv=512) == b.DL_ERR_UNSUPPORTED
+    assert step(lib, fn, s_dt=7) == b.DL_ERR_INVALID_ARG
+    assert step(lib, fn, in_dt=-1) == b.DL_ERR_INVALID_ARG
+    assert step(lib, fn, o=addr(0) + 4096) == b.DL_ERR_INVALID_ARG      # o inside S
+    assert "overlaps" in lib.dl_last_error().decode()
+    assert step(lib, fn, q=addr(0) + 1024) == b.DL_ERR_INVALID_ARG      # S written over an input
+
+
+def test_scalar_operands_need_only_element_alignment(lib):
+    # beta (and a head-wise a) may sit at any element boundary; the check that
+    # fails here is a deliberate misaligned q, reached only after beta passed.
+    rc = step(lib, "dl_gdn_decode_step", beta=addr(4) + 2, a=addr(5) + 6, q=addr(1) + 2)
+    assert rc == b.DL_ERR_INVALID_ARG and "q is not" in lib.dl_last_error().decode()
+    rc = step(lib, "dl_kda_decode_step", a=addr(5) + 2)  # channel-wise a is a vector operand
+    assert rc == b.DL_ERR_INVALID_ARG and "a is not" in lib.dl_last_error().decode()
+
+
+def make_log(L=8, dtype=b.DL_BF16, base=10):
+    return b.dl_log(addr(base), addr(base + 1), addr(base + 2), addr(base + 3), dtype, L)
+
+
+def append(lib, fn="dl_log_append_read", log=None, n=0, kind=b.DL_DECAY_CHANNEL, S=None, dk=128, dv=128,
+           in_dt=b.DL_BF16, o=None):
+    log = log if log is not None else make_log()
+    lp = ctypes.byref(log) if log != -1 else None
+    return getattr(lib, fn)(S or addr(0), b.DL_F32, kind, lp, n, addr(1), addr(2), addr(3), addr(4), addr(5),
+                            in_dt, o or addr(6), 2, 3, dk, dv, None)
+
+
+@pytest.mark.parametrize("fn", ["dl_log_append_read", "dl_log_merge_read"])
+def test_log_step_argument_checks(lib, fn):
+    assert append(lib, fn, n=8) == b.DL_ERR_LOG_FULL
+    assert "merge first" in lib.dl_last_error().decode()
+    assert append(lib, fn, n=-1) == b.DL_ERR_INVALID_ARG
+    assert append(lib, fn, log=-1) == b.DL_ERR_INVALID_ARG
+    assert append(lib, fn, log=make_log(L=0)) == b.DL_ERR_UNSUPPORTED
+    assert append(lib, fn, log=make_log(L=65)) == b.DL_ERR_UNSUPPORTED
+    assert append(lib, fn, log=make_log(dtype=b.DL_F32)) == b.DL_ERR_UNSUPPORTED  # log dtype != inputs
+    assert append(lib, fn, kind=5) == b.DL_ERR_INVALID_ARG
+    assert append(lib, fn, dv=32) == b.DL_ERR_UNSUPPORTED
+    bad = make_log()
+    bad.v = addr(11) + 8
+    assert append(lib, fn, log=bad) == b.DL_ERR_INVALID_ARG
+    assert append(lib, fn, o=addr(12)) == b.DL_ERR_INVALID_ARG          # o overlaps log.v
+    lo = make_log()
+    lo.k = addr(0) + 256                                                 # log inside the base
+    assert append(lib, fn, log=lo) == b.DL_ERR_INVALID_ARG
+
+
+def test_merge_argument_checks(lib):
+    def merge(n, log=None, kind=b.DL_DECAY_HEAD, S=None, dk=128):
+        log = log if log is not None else make_log()
+        return lib.dl_log_merge(S or addr(0), b.DL_F32, kind, ctypes.byref(log), n, 2, 3, dk, 128, None)
+
+    assert merge(0) == b.DL_ERR_INVALID_ARG
+    assert merge(9) == b.DL_ERR_INVALID_ARG
+    assert merge(3, kind=2) == b.DL_ERR_INVALID_ARG
+    assert merge(3, dk=32) == b.DL_ERR_UNSUPPORTED
+    assert merge(3, S=addr(0) + 4) == b.DL_ERR_INVALID_ARG
+    assert lib.dl_log_merge(addr(0), b.DL_F32, 0, None, 1, 2, 3, 128, 128, None) == b.DL_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors():
+    torch = pytest.importorskip("torch")
+    S = torch.zeros(1, 1, 64, 64)
+    x = torch.zeros(1, 1, 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        b.dl_gdn_decode_step(S, x, x, x, torch.zeros(1, 1), torch.zeros(1, 1), x, stream=0)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not found"):
+        b.load(str(tmp_path / "libdeltalog.so"))
