@@ -1,0 +1,561 @@
+"""Decode-step benchmark: gated delta-rule state updates on B200.
+
+One bench step = one full decode of the workload's T tokens for all B
+sequences (every head of every layer-slice in the batch), through the C ABI:
+  * deferred (the headline, DeltaLog schedule): dl_log_append_read on the
+    steps that append, dl_log_merge_read on the step that fills the log
+    (merge fused with that step's read), i.e. every row of the path: append,
+    key-side recursion, base read, merge;
+  * eager, timed the same way, reported beside it;
+  * e2e: the deferred decode from pinned host buffers -- initial state and
+    each token's q, k, v, beta, a copied in, each token's o and the final
+    state copied out, all inside the timed region.
+Metric: decode tokens/s = B * T / time (state updates/s = B * H * T / time)
+and achieved HBM GB/s of the dominant kernel against the measured peak.
+
+Timing: W untimed warm-up steps, then K steps between a barrier +
+cuda.synchronize on both sides, CUDA events on the launching stream, max
+over ranks. Inputs (a 512 MiB fp32 state) are larger than L2, so no flush.
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own batch
+(weak scaling; sequences are independent, no collective on the data path).
+
+--impl reference times the fp64 CPU oracle (the only other implementation
+of this path) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402  (seeded inputs; no method arithmetic)
+
+METRIC = "decode tokens/sec (B×H state updates/s) and achieved HBM GB/s vs peak, 1 B200"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "kda_b256_h32_d128_t512"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "append_read_kda_b256_h32_d128_L16.md")
+KERNEL_SOURCES = ["gated_delta_rule_104_b200/csrc/deferred_read.cu", "gated_delta_rule_104_b200/csrc/common.cuh"]
+
+
+# ---------------------------------------------------------------- byte model
+
+def entry_bytes(w: W.Workload) -> int:
+    """Bytes of one log entry / one step's (k, v, beta, a)."""
+    s_in = 2 if w.in_dtype == "bf16" else 4
+    return (w.d_k + w.d_v + 1 + (w.d_k if w.decay == W.CHANNEL else 1)) * s_in
+
+
+def state_bytes_head(w: W.Workload) -> int:
+    return w.d_v * w.d_k * (2 if w.state_dtype == "bf16" else 4)
+
+
+def alg_bytes(w: W.Workload, kind: str, n: int) -> int:
+    """Algorithmic HBM bytes of one launch over all B*H heads.
+
+    eager:        state read + write, this step's inputs, o
+    append_read:  state read (no write), n log entries read, one entry
+                  written, this step's inputs, o
+    merge_read:   state read + write, n log entries, this step's inputs, o
+    merge:        state read + write, n log entries
+    """
+    e, S = entry_bytes(w), state_bytes_head(w)
+    s_in = 2 if w.in_dtype == "bf16" else 4
+    q, o = w.d_k * s_in, 4 * w.d_v
+    per_head = {
+        "eager": 2 * S + e + q + o,
+        "append_read": S + n * e + e + e + q + o,
+        "merge_read": 2 * S + n * e + e + q + o,
+        "merge": 2 * S + n * e,
+    }[kind]
+    return per_head * w.heads
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def reduce_max(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    try:
+        txt = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in txt.splitlines():
+        if ":" in line and line.strip().startswith("- `"):
+            key, _, val = line.strip()[3:].partition("`:")
+            vals[key.strip()] = val.strip()
+    if vals.get("source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms (read only)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(w: W.Workload, L: int, budget_s: float, first_head: int = 0):
+    """Time the fp64 oracle (deferred schedule, log capacity L) on heads of the
+    workload until about ``budget_s`` seconds of CPU work; returns
+    (tokens/s-equivalent, heads, seconds, threads)."""
+    import oracle  # test infrastructure: CPU baseline only
+
+    oracle.build()
+    threads = oracle.omp_threads()
+    chunk = max(1, threads)
+    heads_done, secs, h0 = 0, 0.0, first_head
+    while secs < budget_s and heads_done < w.heads:
+        heads = [(h0 + i) % w.heads for i in range(min(chunk, w.heads - heads_done))]
+        x = W.generate(w, heads=heads)
+        t0 = time.perf_counter()
+        oracle.run_workload_heads(w, x, "deferred", L)
+        secs += time.perf_counter() - t0
+        heads_done += len(heads)
+        h0 += len(heads)
+        chunk = min(chunk * 2, 4096)
+    tokens = heads_done * w.T / w.H  # one token = one sequence step across its H heads
+    return tokens / secs, heads_done, secs, threads
+
+
+def run_reference(args, w, L):
+    rank, _, ws = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.build()
+    budget = args.cpu_seconds_per_step
+    for _ in range(args.warmup):
+        oracle_sample(w, L, min(2.0, budget))
+    vals, secs_all, heads_all = [], 0.0, 0
+    for i in range(args.steps):
+        v, heads, secs, threads = oracle_sample(w, L, budget, first_head=i * 997)
+        vals.append(v)
+        secs_all += secs
+        heads_all += heads
+    value = heads_all * w.T / w.H / secs_all
+    sample = (f"{heads_all} of {w.heads} (b,h) heads x all {w.T} steps over {args.steps} steps "
+              f"(about {budget:.0f} s of oracle work each), deferred schedule L={L}, fp64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * w.B * w.T / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(w, L, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(w, L, args):
+    return {"workload": w.name, "decay": "channel (KDA)" if w.decay == W.CHANNEL else "head (GDN)",
+            "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "T": w.T, "L": L,
+            "state_dtype": w.state_dtype, "in_dtype": w.in_dtype,
+            "schedule": "DeltaLog deferred, merge fused into the L-th step" if args.schedule == "fused"
+            else "DeltaLog deferred, separate merge every L steps",
+            "global_batch": w.B * max(1, dist_env()[2]), "seq_len": w.T,
+            "l2": "inputs larger than L2 (state %d MiB per GPU), no flush" % (w.state_bytes() >> 20)}
+
+
+# ---------------------------------------------------------------- GPU legs
+
+class Launcher:
+    """Issues the T steps of one decode and (optionally) brackets every launch
+    with CUDA events on the launching stream."""
+
+    def __init__(self, g, w, d, S, log, o_all, schedule, stream):
+        self.g, self.w, self.d, self.S, self.log, self.o_all = g, w, d, S, log, o_all
+        self.schedule, self.stream = schedule, stream
+        self.chan = w.decay == W.CHANNEL
+        self.L = log.L if log is not None else 0
+
+    def plan(self):
+        """(kind, n) of each launch of one decode, in order."""
+        out, n = [], 0
+        for _ in range(self.w.T):
+            if self.schedule == "eager":
+                out.append(("eager", 0))
+            elif self.schedule == "fused" and n == self.L - 1:
+                out.append(("merge_read", n))
+                n = 0
+            else:
+                out.append(("append_read", n))
+                n += 1
+                if n == self.L:
+                    out.append(("merge", n))
+                    n = 0
+        if n:
+            out.append(("merge", n))  # flush so that S holds the final state
+        return out
+
+    def run(self, events=None):
+        g, d, S, o, st = self.g, self.d, self.S, self.o_all, self.stream
+        t = 0
+        for kind, n in self.plan():
+            if events is not None:
+                events.append(self._ev())
+            if kind == "eager":
+                fn = g.dl_kda_decode_step if self.chan else g.dl_gdn_decode_step
+                fn(S, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                t += 1
+            elif kind == "append_read":
+                g.dl_log_append_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                t += 1
+            elif kind == "merge_read":
+                g.dl_log_merge_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                t += 1
+            else:
+                g.dl_log_merge(S, self.log, n, st)
+        if events is not None:
+            events.append(self._ev())
+
+    def _ev(self):
+        import torch
+
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+
+def timed(launcher, steps, warmup):
+    """Returns (ms per step (max over ranks), per-kind {durations}, launches)."""
+    import torch
+    import torch.distributed as dist
+
+    for _ in range(warmup):
+        launcher.run()
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    plan = launcher.plan()
+    all_events = []
+    for _ in range(steps):
+        ev = []
+        launcher.run(ev)
+        all_events.append(ev)
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in all_events)
+    per_kind = {}
+    for ev in all_events:
+        for i, (kind, n) in enumerate(plan):
+            per_kind.setdefault(kind, []).append((n, ev[i].elapsed_time(ev[i + 1])))
+    ms = reduce_max(total_ms / steps)
+    return ms, per_kind, steps * len(plan)
+
+
+def roofline_for(w, per_kind, kind, peak, peak_note, traffic):
+    rec = per_kind.get(kind, [])
+    if not rec:
+        return None
+    total_bytes = sum(alg_bytes(w, kind, n) for n, _ in rec)
+    total_s = sum(ms for _, ms in rec) / 1000.0
+    achieved = total_bytes / total_s / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": kind, "launches": len(rec), "avg_us": round(1e6 * total_s / len(rec), 2),
+            "alg_bytes_per_launch": round(total_bytes / len(rec)), "peak_source": peak_note,
+            "frac_of_8tbs_spec": round(achieved / SPEC_HBM_GBS, 4)}
+
+
+def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
+    """Deferred decode from pinned host buffers through the public API:
+    per step, S0 and every token's inputs H2D, every token's o and the final
+    state D2H (copy streams overlap the kernels)."""
+    import torch
+
+    dev = torch.device("cuda")
+    chan = w.decay == W.CHANNEL
+    tdt = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    B, H = w.B, w.H
+    S = torch.empty(B, H, w.d_v, w.d_k, dtype=host["S0"].dtype, device=dev)
+    log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=dev)
+    names = ("q", "k", "v", "beta", "a")
+    nslot = 3
+    slots = [{n: torch.empty_like(host[n][0], device=dev) for n in names} for _ in range(nslot)]
+    o_dev = [torch.empty(B, H, w.d_v, dtype=torch.float32, device=dev) for _ in range(nslot)]
+    o_host = torch.empty(w.T, B, H, w.d_v, dtype=torch.float32, pin_memory=True)
+    S_host = torch.empty_like(host["S0"], pin_memory=True)
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    step_in = sum(host[n][0].numel() * host[n][0].element_size() for n in names)
+    h2d_bytes = host["S0"].numel() * host["S0"].element_size() + w.T * step_in
+    d2h_bytes = o_host.numel() * 4 + S_host.numel() * S_host.element_size()
+
+    def one():
+        ev_in = [torch.cuda.Event() for _ in range(nslot)]
+        ev_used = [None] * nslot
+        ev_out = [None] * nslot
+        with torch.cuda.stream(h2d):
+            S.copy_(host["S0"], non_blocking=True)
+        s_ready = torch.cuda.Event()
+        s_ready.record(h2d)
+        stream.wait_event(s_ready)
+        dec = g.DeferredDecoder(S, log, fused_merge=(schedule == "fused"))
+        for t in range(w.T):
+            j = t % nslot
+            with torch.cuda.stream(h2d):
+                if ev_used[j] is not None:
+                    h2d.wait_event(ev_used[j])
+                for n in names:
+                    slots[j][n].copy_(host[n][t], non_blocking=True)
+                ev_in[j].record(h2d)
+            stream.wait_event(ev_in[j])
+            if ev_out[j] is not None:
+                stream.wait_event(ev_out[j])  # o slot drained
+            sl = slots[j]
+            dec.step(sl["q"], sl["k"], sl["v"], sl["beta"], sl["a"], o_dev[j], stream)
+            ev_used[j] = torch.cuda.Event()
+            ev_used[j].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_used[j])
+                o_host[t].copy_(o_dev[j], non_blocking=True)
+                ev_out[j] = torch.cuda.Event()
+                ev_out[j].record(d2h)
+        dec.flush(stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(done)
+            S_host.copy_(S, non_blocking=True)
+
+    import torch.distributed as dist
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    start_events = []
+    for _ in range(steps):
+        one()
+    # the last D2H copy ends the step: join it into the timing stream
+    end_d2h = torch.cuda.Event()
+    end_d2h.record(d2h)
+    stream.wait_event(end_d2h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    ms = reduce_max(e0.elapsed_time(e1) / steps)
+    del start_events
+    return ms, h2d_bytes, d2h_bytes
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--L", type=int, default=0, help="log capacity (default: the workload's)")
+    ap.add_argument("--schedule", choices=["fused", "unfused"], default="fused")
+    ap.add_argument("--workers", type=int, default=0, help="input-generation processes (0: auto)")
+    ap.add_argument("--cpu-seconds-per-step", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-eager", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="decode only this many tokens per step (small profiling runs; default: the workload's T)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = W.WORKLOADS[args.workload]
+    if args.tokens:
+        w = W.scaled(w, T=args.tokens)
+    L = args.L or max(w.L)
+    rank, local_rank, ws = dist_env()
+    if args.gpus != ws and ws > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+
+    if args.impl == "reference":
+        return run_reference(args, w, L)
+
+    # Inputs first (spawned generator processes start before any CUDA call).
+    workers = args.workers or W.default_workers()
+    t0 = time.time()
+    x = W.generate(w, workers=workers)
+    gen_s = time.time() - t0
+
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_104_b200 as g
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA library is the only compute path)")
+    torch.cuda.set_device(local_rank)
+    if ws > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    g.load()
+    d = W.device_inputs(w, x)
+    stream = torch.cuda.current_stream()
+    chan = w.decay == W.CHANNEL
+    tdt = d["q"].dtype
+    o_all = torch.empty(w.T, w.B, w.H, w.d_v, dtype=torch.float32, device="cuda")
+    peak, peak_note = measured_peaks()
+    traffic = profiled_traffic()
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        S_def = d["S0"].clone()
+        log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, tdt, chan)
+        lau = Launcher(g, w, d, S_def, log, o_all, args.schedule, stream)
+        ms_def, kinds_def, launches = timed(lau, args.steps, args.warmup)
+        eager = None
+        if not args.no_eager:
+            S_e = d["S0"].clone()
+            lau_e = Launcher(g, w, d, S_e, None, o_all, "eager", stream)
+            ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup)
+            eager = {"value": w.B * w.T / (ms_e / 1000.0) * ws, "unit": UNIT, "ms_per_step": round(ms_e, 3),
+                     "state_updates_per_s": w.heads * w.T / (ms_e / 1000.0) * ws,
+                     "roofline": roofline_for(w, kinds_e, "eager", peak, peak_note, None)}
+            del S_e
+    clocks = sampler.summary()
+
+    value = w.B * w.T / (ms_def / 1000.0) * ws
+    rf = roofline_for(w, kinds_def, "append_read", peak, peak_note, traffic)
+    other = {k: roofline_for(w, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != "append_read"}
+    step_time = {k: round(sum(ms for _, ms in v) / args.steps, 3) for k, v in kinds_def.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        host = {}
+        for n in ("S0", "q", "k", "v", "beta", "a"):
+            host[n] = d[n].cpu().pin_memory()
+        ms_e2e, h2d_b, d2h_b = run_e2e(g, w, host, L, args.schedule, max(2, args.steps // 4), args.warmup, stream)
+        e2e = {"value": w.B * w.T / (ms_e2e / 1000.0) * ws, "unit": UNIT, "ms_per_step": round(ms_e2e, 3),
+               "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
+               "what": "deferred decode from pinned host memory: S0 and per-token inputs in, per-token o "
+                       "and the final state out, inside the timed region"}
+        del host
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, heads, secs, threads = oracle_sample(w, L, args.cpu_seconds_per_step)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{heads} of {w.heads} (b,h) heads x all {w.T} steps, fp64 deferred schedule L={L}, "
+                         f"{secs:.1f} s on {threads} OpenMP threads; tokens = heads x T / H"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_def, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic", "config": config_block(w, L, args),
+        "state_updates_per_s": w.heads * w.T / (ms_def / 1000.0) * ws,
+        "roofline": rf, "roofline_other_kernels": other, "ms_per_step_by_kernel": step_time,
+        "eager": eager, "deferred_over_eager": (value / eager["value"]) if eager else None,
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks,
+        "input_generation_s": round(gen_s, 1),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -143,19 +143,26 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     const bool chan = kind == DL_DECAY_CHANNEL;
-    Buf b[11];
+    Buf b[12];
     int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
     if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
     nb += 4;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
     if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
-    // written: o and the log (slot n); the base is only read.
-    const Buf writers[5] = {b[6], b[7], b[8], b[9], b[10]};
-    if ((s = check_overlap(writers, 5, b, nb)) != DL_OK) return s;
+    const size_t need = dl::read_work_bytes(B, H, d_k, d_v);
+    b[nb] = {"log.work", log->work, need, 16};
+    if ((s = check_bufs(b + nb, 1)) != DL_OK) return s;
+    if (log->work_bytes < need)
+        return fail(DL_ERR_INVALID_ARG, "log.work holds %zu bytes, needs %zu", log->work_bytes, need);
+    ++nb;
+    // written: o, the log (slot n) and its workspace; the base is only read.
+    const Buf writers[6] = {b[6], b[7], b[8], b[9], b[10], b[11]};
+    if ((s = check_overlap(writers, 6, b, nb)) != DL_OK) return s;
     dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
     dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
-    return cuda_status(dl::launch_append_read(p, lg, n, stream), "append-read launch");
+    return cuda_status(dl::launch_append_read(p, lg, n, static_cast<float *>(log->work), stream),
+                       "append-read launch");
 }
 
 dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log, int n, int B, int H,
@@ -214,6 +221,11 @@ const char *dl_status_string(dl_status s) {
 }
 
 const char *dl_last_error(void) { return g_err; }
+
+size_t dl_log_work_bytes(int B, int H, int d_k, int d_v) {
+    if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return 0;
+    return dl::read_work_bytes(B, H, d_k, d_v);
+}
 
 int dl_abi_version(void) { return DL_ABI_VERSION; }
 

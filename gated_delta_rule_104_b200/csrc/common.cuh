@@ -131,6 +131,38 @@ __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// ---------------------------------------------------------------- staging
+
+// Copy a rows x cols block of IT (each row contiguous in global memory, row
+// r at src + r * src_stride; cols a multiple of 16 / sizeof(IT)) into shared
+// memory as float with row stride dst_stride. All threads of the block take
+// part; the flat chunk loop is unrolled so several 16-byte loads are in
+// flight per thread before the first shared store.
+template <class IT>
+__device__ __forceinline__ void stage_block(float *dst, int dst_stride, const IT *src, long long src_stride,
+                                            int rows, int cols, int tid, int nthreads) {
+    constexpr int E = 16 / (int)sizeof(IT);
+    const int cpr = cols / E;  // chunks per row
+    const int total = rows * cpr;
+#pragma unroll 4
+    for (int c = tid; c < total; c += nthreads) {
+        const int r = c / cpr, j = (c - r * cpr) * E;
+        float x[E];
+        load_vec<E>(src + r * src_stride + j, x);
+#pragma unroll
+        for (int e = 0; e < E; ++e) dst[r * dst_stride + j + e] = x[e];
+    }
+}
+
+// ---------------------------------------------------------------- PDL
+
+// Programmatic dependent launch: a producer lets the next kernel in the
+// stream start early; the consumer waits for the producer's completion (and
+// memory) only where it first reads the producer's results. Both are no-ops
+// when the launch did not opt in.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- async copy
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {

@@ -1,203 +1,216 @@
 // Deferred step: append this step's factors to the log and read
 // o = S_n q from the unwritten base plus the log (DeltaLog page, Technical
-// Summary, "Append Phase", and "Kernel Implementation": value-tile
-// parallelism, key-side metadata computed once and shared by the value
-// tiles, a "ReplayPrep" stage then "AppendDecode" stages).
+// Summary, "Append Phase", and "Kernel Implementation": key-side metadata
+// computed once per slot-head in a "ReplayPrep" stage and shared by the value
+// tiles, which then run in parallel "AppendDecode" stages).
 //
 // With A_i = Diag(a_i)(I - beta_i k_i k_i^T), the logical state after log
 // entries 1..n is S_n = S_bar A_1...A_n + sum_i beta_i v_i k_i^T A_{i+1}...A_n,
 // so o = S_n q needs only
 //   key side (once per head):   x_n = q; for i = n..1:
 //        c_i = k_i . x_i,  s_i = beta_i c_i,  x_{i-1} = a_i o (x_i - s_i k_i)
-//   value side (per row r):     o_r = S_bar[r] . x_0 + sum_i s_i v_i[r].
+//        and w = sum_i s_i v_i            (a d_v vector)
+//   value side (per row r):     o_r = S_bar[r] . x_0 + w_r.
 // The base is read once and never written.
 //
-// One 256-thread block per (head, value tile); a tile holds up to 64 KB of
-// the base. The block first issues all of its base loads into registers
-// (16 x 16 bytes per thread at most), then stages the log entries it needs
-// into shared memory, writes the new entry (tile 0 only), runs the key-side
-// recursion in warp 0 while the base loads are in flight, and finally every
-// warp finishes its rows with group shuffle reductions.
+// Two kernels, chained with programmatic dependent launch:
+//   replay_prep   one warp per head: appends the entry, runs the serial
+//                 recursion (lanes own d_k/32 key columns, one shuffle
+//                 reduction per entry) and w, and stores (x_0, w) in the
+//                 caller's workspace [B*H][d_k + d_v] fp32.
+//   append_decode a pure streaming pass over the base, laid out like the
+//                 eager kernel (a row spread over 16-byte lane slices, 8 loads
+//                 in flight per thread, no shared memory, no block barrier).
+//                 It may start while replay_prep still runs: it issues its
+//                 base loads first and waits for the prep grid only before
+//                 reading the workspace.
 #include "launch.h"
 
 namespace dl {
 
-template <class ST, int DK, int DV>
-struct ReadShape {
+// ------------------------------------------------------------------ prep
+
+template <class IT, int DK, int DV, bool CHAN>
+__global__ void __launch_bounds__(256)
+replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
+                   const IT *__restrict__ beta, const IT *__restrict__ a, IT *__restrict__ log_k,
+                   IT *__restrict__ log_v, IT *__restrict__ log_b, IT *__restrict__ log_a, int L, int n,
+                   float *__restrict__ work, long long heads) {
+    pdl_launch_dependents();
+    constexpr int CW = DK / 32;   // key columns per lane
+    constexpr int RV = DV / 32;   // value rows per lane
+    constexpr int CHUNK = 4;      // log entries fetched together
+    const int lane = threadIdx.x & 31;
+    const long long head = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (head >= heads) return;
+    const long long lrow = head * L;
+    const int c0 = lane * CW, r0 = lane * RV;
+
+    // This step's entry (index n), from the inputs.
+    float kc[CW], ac[CW], vc[RV], x[CW];
+    load_vec<CW>(k + head * DK + c0, kc);
+    load_vec<RV>(v + head * DV + r0, vc);
+    load_vec<CW>(q + head * DK + c0, x);
+    if constexpr (CHAN) {
+        load_vec<CW>(a + head * DK + c0, ac);
+    } else {
+        const float as = to_f(a[head]);
+#pragma unroll
+        for (int e = 0; e < CW; ++e) ac[e] = as;
+    }
+    const float bc = to_f(beta[head]);
+
+    // D1: the entry is appended unchanged (raw input elements).
+#pragma unroll
+    for (int e = 0; e < CW; ++e) log_k[(lrow + n) * DK + c0 + e] = k[head * DK + c0 + e];
+#pragma unroll
+    for (int e = 0; e < RV; ++e) log_v[(lrow + n) * DV + r0 + e] = v[head * DV + r0 + e];
+    if constexpr (CHAN) {
+#pragma unroll
+        for (int e = 0; e < CW; ++e) log_a[(lrow + n) * DK + c0 + e] = a[head * DK + c0 + e];
+    } else if (lane == 0) {
+        log_a[lrow + n] = a[head];
+    }
+    if (lane == 0) log_b[lrow + n] = beta[head];
+
+    // D2: the recursion, newest entry first.
+    float w[RV];
+#pragma unroll
+    for (int e = 0; e < RV; ++e) w[e] = 0.f;
+    auto step = [&](const float (&kk)[CW], const float (&aa)[CW], float bb, const float (&vv)[RV]) {
+        float c = 0.f;
+#pragma unroll
+        for (int e = 0; e < CW; ++e) c = fmaf(kk[e], x[e], c);
+        c = group_sum<32>(c);
+        const float s = bb * c;
+#pragma unroll
+        for (int e = 0; e < CW; ++e) x[e] = aa[e] * fmaf(-s, kk[e], x[e]);
+#pragma unroll
+        for (int e = 0; e < RV; ++e) w[e] = fmaf(s, vv[e], w[e]);
+    };
+    step(kc, ac, bc, vc);
+    for (int top = n - 1; top >= 0; top -= CHUNK) {
+        float kk[CHUNK][CW], aa[CHUNK][CW], vv[CHUNK][RV], bb[CHUNK];
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j) {
+            const int i = top - j;
+            if (i < 0) break;
+            load_vec<CW>(log_k + (lrow + i) * DK + c0, kk[j]);
+            load_vec<RV>(log_v + (lrow + i) * DV + r0, vv[j]);
+            if constexpr (CHAN) {
+                load_vec<CW>(log_a + (lrow + i) * DK + c0, aa[j]);
+            } else {
+                const float as = to_f(log_a[lrow + i]);
+#pragma unroll
+                for (int e = 0; e < CW; ++e) aa[j][e] = as;
+            }
+            bb[j] = to_f(log_b[lrow + i]);
+        }
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j) {
+            if (top - j < 0) break;
+            step(kk[j], aa[j], bb[j], vv[j]);
+        }
+    }
+
+    // (x_0, w) -> workspace.
+    float *wk = work + head * (DK + DV);
+#pragma unroll
+    for (int e = 0; e < CW; ++e) wk[c0 + e] = x[e];
+#pragma unroll
+    for (int e = 0; e < RV; ++e) wk[DK + r0 + e] = w[e];
+}
+
+// ------------------------------------------------------------------ decode
+
+template <class ST, int DK>
+struct DecodeShape {
     static constexpr int VEC = StateVec<ST>::N;
-    static constexpr int G = DK / VEC;                 // lanes per row
-    static constexpr int RPW = 32 / G;                 // rows per warp-wide load
-    static constexpr int ROW_BYTES = DK * (int)sizeof(ST);
-    static constexpr int ROWS = DV < 65536 / ROW_BYTES ? DV : 65536 / ROW_BYTES;  // rows per block
-    static constexpr int TILES = DV / ROWS;
+    static constexpr int G = DK / VEC;       // lanes per row
+    static constexpr int RPW = 32 / G;       // rows per warp-wide load
+    static constexpr int R = 8;              // loads in flight per thread
+    static constexpr int UNIT = R * RPW;     // rows per warp
     static constexpr int WARPS = 8;
-    static constexpr int THREADS = WARPS * 32;
-    static constexpr int NV = ROWS / (WARPS * RPW);    // 16-byte base loads per thread
-    static constexpr int CW = DK / 32;                 // key columns per lane in the recursion
-    static constexpr int SVS = ROWS + 1;               // padded stride of staged values
-    static_assert(NV >= 1 && NV * WARPS * RPW == ROWS, "tile shape");
 };
 
-// Shared-memory floats needed for a log holding n entries before this step.
-template <class ST, int DK, int DV, bool CHAN>
-__host__ __device__ constexpr size_t read_smem_floats(int n) {
-    using C = ReadShape<ST, DK, DV>;
-    return (size_t)(n + 1) * DK                    // k
-         + (size_t)(n + 1) * (CHAN ? DK : 1)       // a
-         + (size_t)(n + 1)                         // beta
-         + (size_t)(n + 1) * C::SVS                // v (this tile's rows)
-         + (size_t)(n + 1)                         // s
-         + DK;                                     // x_0
-}
-
-template <class IT>
-__device__ __forceinline__ void stage_contig(float *dst, const IT *src, int count, int tid, int nthreads) {
-    constexpr int E = 16 / (int)sizeof(IT);  // elements per 16-byte chunk
-    const int chunks = count / E;
-    for (int c = tid; c < chunks; c += nthreads) {
-        float x[E];
-        load_vec<E>(src + c * E, x);
-#pragma unroll
-        for (int e = 0; e < E; ++e) dst[c * E + e] = x[e];
-    }
-    for (int i = chunks * E + tid; i < count; i += nthreads) dst[i] = to_f(src[i]);
-}
-
-template <class IT>
-__device__ __forceinline__ void copy_contig(IT *dst, const IT *src, int count, int tid, int nthreads) {
-    constexpr int E = 16 / (int)sizeof(IT);
-    const int chunks = count / E;
-    for (int c = tid; c < chunks; c += nthreads)
-        *reinterpret_cast<uint4 *>(dst + c * E) = *reinterpret_cast<const uint4 *>(src + c * E);
-    for (int i = chunks * E + tid; i < count; i += nthreads) dst[i] = src[i];
-}
-
-template <class ST, class IT, int DK, int DV, bool CHAN>
-__global__ void __launch_bounds__(256, 2)
-append_read_kernel(const ST *__restrict__ Sbar, const IT *__restrict__ q, const IT *__restrict__ k,
-                   const IT *__restrict__ v, const IT *__restrict__ beta, const IT *__restrict__ a,
-                   float *__restrict__ o, IT *__restrict__ log_k, IT *__restrict__ log_v,
-                   IT *__restrict__ log_b, IT *__restrict__ log_a, int L, int n) {
-    using C = ReadShape<ST, DK, DV>;
+template <class ST, int DK, int DV>
+__global__ void __launch_bounds__(256)
+append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work, float *__restrict__ o,
+                     long long num_units) {
+    using C = DecodeShape<ST, DK>;
     constexpr int VEC = C::VEC;
-    extern __shared__ float4 smem_raw[];
-    float *sk = reinterpret_cast<float *>(smem_raw);
-    float *sa = sk + (size_t)(n + 1) * DK;
-    float *sb = sa + (size_t)(n + 1) * (CHAN ? DK : 1);
-    float *sv = sb + (n + 1);
-    float *ss = sv + (size_t)(n + 1) * C::SVS;
-    float *sx = ss + (n + 1);
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long head = blockIdx.x / C::TILES;
-    const int tile = blockIdx.x % C::TILES;
-    const int row0 = tile * C::ROWS;                 // first row of the tile within the head
+    static_assert(DV % C::UNIT == 0, "unit divides d_v");
+    const int lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * C::WARPS + (threadIdx.x >> 5);
+    const bool active = unit < num_units;
+    const long long row0 = unit * C::UNIT;
+    const long long head = row0 / DV;
+    const int rin0 = (int)(row0 - head * DV);
     const int sub = lane / C::G;
     const int col = (lane % C::G) * VEC;
 
-    // D3 operands first: this thread's slice of the base (NV rows x 16 bytes).
-    const ST *bsrc = Sbar + (head * DV + row0 + (long long)warp * C::NV * C::RPW + sub) * DK + col;
-    uint4 raw[C::NV];
+    // D3 operands: the base rows first (read only, streamed).
+    uint4 raw[C::R];
+    if (active) {
+        const ST *src = Sbar + (row0 + sub) * DK + col;
 #pragma unroll
-    for (int j = 0; j < C::NV; ++j) raw[j] = ld_ro_stream(bsrc + (long long)j * C::RPW * DK);
-
-    // Stage log entries 0..n-1 and this step's factors as entry n.
-    const long long lrow = head * L;                 // first log slot of this head
-    stage_contig(sk, log_k + lrow * DK, n * DK, tid, C::THREADS);
-    stage_contig(sk + (size_t)n * DK, k + head * DK, DK, tid, C::THREADS);
-    if constexpr (CHAN) {
-        stage_contig(sa, log_a + lrow * DK, n * DK, tid, C::THREADS);
-        stage_contig(sa + (size_t)n * DK, a + head * DK, DK, tid, C::THREADS);
-    } else {
-        for (int i = tid; i < n; i += C::THREADS) sa[i] = to_f(log_a[lrow + i]);
-        if (tid == 0) sa[n] = to_f(a[head]);
+        for (int r = 0; r < C::R; ++r) raw[r] = ld_ro_stream(src + (long long)r * C::RPW * DK);
     }
-    for (int i = tid; i < n; i += C::THREADS) sb[i] = to_f(log_b[lrow + i]);
-    if (tid == 0) sb[n] = to_f(beta[head]);
-    for (int i = 0; i < n; ++i)
-        stage_contig(sv + (size_t)i * C::SVS, log_v + (lrow + i) * DV + row0, C::ROWS, tid, C::THREADS);
-    stage_contig(sv + (size_t)n * C::SVS, v + head * DV + row0, C::ROWS, tid, C::THREADS);
-
-    // D1: append (k, v, beta, a) as entry n, unchanged. One tile per head writes it.
-    if (tile == 0) {
-        copy_contig(log_k + (lrow + n) * DK, k + head * DK, DK, tid, C::THREADS);
-        copy_contig(log_v + (lrow + n) * DV, v + head * DV, DV, tid, C::THREADS);
-        if constexpr (CHAN) copy_contig(log_a + (lrow + n) * DK, a + head * DK, DK, tid, C::THREADS);
-        else if (tid == 0) log_a[lrow + n] = a[head];
-        if (tid == 0) log_b[lrow + n] = beta[head];
-    }
-    __syncthreads();
-
-    // D2: key-side recursion (ReplayPrep), warp 0, lanes own CW key columns.
-    if (warp == 0) {
-        const int c0 = lane * C::CW;
-        float x[C::CW];
-        load_vec<C::CW>(q + head * DK + c0, x);
-        for (int i = n; i >= 0; --i) {
-            float kk[C::CW], ai[C::CW];
-            load_vec<C::CW>(sk + (size_t)i * DK + c0, kk);
-            if constexpr (CHAN) {
-                load_vec<C::CW>(sa + (size_t)i * DK + c0, ai);
-            } else {
-#pragma unroll
-                for (int e = 0; e < C::CW; ++e) ai[e] = sa[i];
-            }
-            float c = 0.f;
-#pragma unroll
-            for (int e = 0; e < C::CW; ++e) c = fmaf(kk[e], x[e], c);
-            c = group_sum<32>(c);
-            const float si = sb[i] * c;
-#pragma unroll
-            for (int e = 0; e < C::CW; ++e) x[e] = ai[e] * fmaf(-si, kk[e], x[e]);
-            if (lane == 0) ss[i] = si;
-        }
-#pragma unroll
-        for (int e = 0; e < C::CW; ++e) sx[c0 + e] = x[e];
-    }
-    __syncthreads();
-
-    // D3: o_r = S_bar[r] . x_0 + sum_i s_i v_i[r]  (AppendDecode).
+    pdl_wait();  // replay_prep's (x_0, w) are complete and visible from here on
+    if (!active) return;
+    const float *wk = work + head * (DK + DV);
     float xv[VEC];
+    load_vec<VEC>(wk + col, xv);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) xv[e] = sx[col + e];
-    const int gl = lane % C::G;
-#pragma unroll
-    for (int j = 0; j < C::NV; ++j) {
-        const int rl = (warp * C::NV + j) * C::RPW + sub;   // row within the tile
+    for (int r = 0; r < C::R; ++r) {
         float s[VEC];
-        StateVec<ST>::unpack(raw[j], s);
+        StateVec<ST>::unpack(raw[r], s);
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc = fmaf(s[e], xv[e], acc);
-        for (int i = gl; i <= n; i += C::G) acc = fmaf(ss[i], sv[(size_t)i * C::SVS + rl], acc);
         acc = group_sum<C::G>(acc);
-        if (gl == 0) o[head * DV + row0 + rl] = acc;
+        const int rr = rin0 + r * C::RPW + sub;
+        if ((lane % C::G) == 0) o[head * DV + rr] = acc + wk[DK + rr];
     }
 }
 
-cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, cudaStream_t st) {
+size_t read_work_bytes(int B, int H, int dk, int dv) { return (size_t)B * H * (dk + dv) * sizeof(float); }
+
+template <class ST, int DK, int DV>
+static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStream_t st) {
+    using C = DecodeShape<ST, DK>;
+    const long long units = (long long)p.B * p.H * DV / C::UNIT;
+    const long long blocks = (units + C::WARPS - 1) / C::WARPS;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(C::WARPS * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, append_decode_kernel<ST, DK, DV>, static_cast<const ST *>(p.S), work, p.o,
+                              units);
+}
+
+cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st) {
     return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
         using ST = decltype(st_t);
         using IT = decltype(it_t);
         constexpr int DK = decltype(dk_c)::value;
         constexpr int DV = decltype(dv_c)::value;
         constexpr bool CH = decltype(ch_c)::value;
-        using C = ReadShape<ST, DK, DV>;
-        auto kern = append_read_kernel<ST, IT, DK, DV, CH>;
-        const size_t smem = read_smem_floats<ST, DK, DV, CH>(n) * sizeof(float);
-        static size_t configured = 48 * 1024;  // per instantiation
-        if (smem > configured) {
-            const size_t want = read_smem_floats<ST, DK, DV, CH>(DL_MAX_LOG - 1) * sizeof(float);
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
-            if (e != cudaSuccess) return e;
-            configured = want;
-        }
-        const long long blocks = (long long)p.B * p.H * C::TILES;
-        kern<<<(unsigned)blocks, C::THREADS, smem, st>>>(
-            static_cast<const ST *>(p.S), static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
-            static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a),
-            p.o, static_cast<IT *>(lg.k), static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta),
-            static_cast<IT *>(lg.a), lg.L, n);
+        const long long heads = (long long)p.B * p.H;
+        replay_prep_kernel<IT, DK, DV, CH><<<(unsigned)((heads + 7) / 8), 256, 0, st>>>(
+            static_cast<const IT *>(p.q), static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
+            static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
+            static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.L, n, work, heads);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = launch_decode<ST, DK, DV>(p, work, st);
+        if (e != cudaSuccess) return e;
         return cudaGetLastError();
     });
 }

@@ -24,7 +24,9 @@ struct LogParams {
 };
 
 cudaError_t launch_eager(const StepParams &p, cudaStream_t st);
-cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, cudaStream_t st);
+// Deferred read: needs read_work_bytes() of fp32 workspace (x_0 and w per head).
+cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st);
+size_t read_work_bytes(int B, int H, int dk, int dv);
 // Merge n_log log entries (plus, if with_cur, this step's inputs as one more
 // entry, and then o = S_new q) into the base.
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,

@@ -106,27 +106,32 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     }
     cp_async_commit();
 
-    // 2. key side and values (log entries 0..n_log-1, then this step's).
+    // 2. key side and values (log entries 0..n_log-1, then this step's): flat,
+    // vectorised loads with several in flight per thread.
     const long long lrow = head * L;
-    for (int i = tid; i < n_log * DK; i += ROWS) fk[i] = ld_in(log_k, lrow * DK + i, bf);
-    if constexpr (CHAN)
-        for (int i = tid; i < n_log * DK; i += ROWS) fa[i] = ld_in(log_a, lrow * DK + i, bf);
-    else
-        for (int i = tid; i < n_log; i += ROWS) fa[i] = ld_in(log_a, lrow + i, bf);
-    for (int i = tid; i < n_log; i += ROWS) sb[i] = ld_in(log_b, lrow + i, bf);
-    for (int i = 0; i < n_log; ++i) sv[(size_t)i * ROWS + tid] = ld_in(log_v, (lrow + i) * DV + row0 + tid, bf);
-    if constexpr (WITH_CUR) {
-        const int e = n_log;
-        for (int c = tid; c < DK; c += ROWS) {
-            fk[(size_t)e * DK + c] = ld_in(k, head * DK + c, bf);
-            if constexpr (CHAN) fa[(size_t)e * DK + c] = ld_in(a, head * DK + c, bf);
-            sq[c] = ld_in(q, head * DK + c, bf);
+    auto stage = [&](auto tag) {
+        using IT = decltype(tag);
+        stage_block(fk, DK, static_cast<const IT *>(log_k) + lrow * DK, DK, n_log, DK, tid, ROWS);
+        if constexpr (CHAN) stage_block(fa, DK, static_cast<const IT *>(log_a) + lrow * DK, DK, n_log, DK, tid, ROWS);
+        stage_block(sv, ROWS, static_cast<const IT *>(log_v) + lrow * DV + row0, DV, n_log, ROWS, tid, ROWS);
+        if constexpr (WITH_CUR) {
+            stage_block(fk + (size_t)n_log * DK, DK, static_cast<const IT *>(k) + head * DK, DK, 1, DK, tid, ROWS);
+            if constexpr (CHAN)
+                stage_block(fa + (size_t)n_log * DK, DK, static_cast<const IT *>(a) + head * DK, DK, 1, DK, tid, ROWS);
+            stage_block(sq, DK, static_cast<const IT *>(q) + head * DK, DK, 1, DK, tid, ROWS);
+            stage_block(sv + (size_t)n_log * ROWS, ROWS, static_cast<const IT *>(v) + head * DV + row0, DV, 1, ROWS,
+                        tid, ROWS);
         }
-        if (tid == 0) {
-            if constexpr (!CHAN) fa[e] = ld_in(a, head, bf);
-            sb[e] = ld_in(beta, head, bf);
-        }
-        sv[(size_t)e * ROWS + tid] = ld_in(v, head * DV + row0 + tid, bf);
+    };
+    if (bf) stage(bf16{});
+    else stage(float{});
+    for (int i = tid; i < n_log; i += ROWS) {
+        if constexpr (!CHAN) fa[i] = ld_in(log_a, lrow + i, bf);
+        sb[i] = ld_in(log_b, lrow + i, bf);
+    }
+    if (WITH_CUR && tid == 0) {
+        if constexpr (!CHAN) fa[n_log] = ld_in(a, head, bf);
+        sb[n_log] = ld_in(beta, head, bf);
     }
     __syncthreads();
 

@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 1
+#define DL_ABI_VERSION 2
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -74,7 +74,9 @@ typedef enum {
 } dl_decay;
 
 /* Caller-owned bounded log of a deferred state: per (b, h) up to L entries of
- * the raw step factors, stored unchanged in `dtype` (lossless).
+ * the raw step factors, stored unchanged in `dtype` (lossless), plus a small
+ * fp32 workspace the deferred read uses to hand its per-head key-side results
+ * to the value tiles.
  * (The page's log keeps "compact update factors" plus log-decay metadata,
  * Technical Summary, "Core Mechanism: Base + Log"; here the metadata is
  * recomputed from the stored decays where it is needed.)
@@ -82,6 +84,8 @@ typedef enum {
  *   v     [B, H, L, d_v]
  *   beta  [B, H, L]
  *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL)
+ *   work  at least dl_log_work_bytes(B, H, d_k, d_v) bytes, 16-byte aligned,
+ *         contents irrelevant between calls (only dl_log_append_read uses it)
  * The number of valid entries n (the same for every head) is tracked by the
  * caller and passed to each call; entries 0..n-1 are valid. */
 typedef struct {
@@ -91,6 +95,8 @@ typedef struct {
     void *a;
     dl_dtype dtype;
     int L;
+    void *work;
+    size_t work_bytes;
 } dl_log;
 
 /* Eager GDN step (head-wise decay), in place.
@@ -113,13 +119,18 @@ dl_status dl_kda_decode_step(void *S, dl_dtype s_dtype,
                              float *o, int B, int H, int d_k, int d_v,
                              cudaStream_t stream);
 
+/* Bytes of log workspace (dl_log.work) the deferred read needs:
+ * B * H * (d_k + d_v) * 4. */
+size_t dl_log_work_bytes(int B, int H, int d_k, int d_v);
+
 /* Deferred step: append this step's (k, v, beta, a) to the log as entry n and
  * write o = S_n q, where S_n is the base with log entries 0..n replayed, read
  * without materialising it (Technical Summary, "Append Phase" and
  * "Kernel Implementation": key-side coefficients computed once per head, then
  * value tiles read the base). S_base is only read.
  *   S_base [B, H, d_v, d_k] s_dtype (read only)
- *   log    entries 0..n-1 read, entry n written
+ *   log    entries 0..n-1 read, entry n written; log->work is overwritten
+ *          (missing or smaller than dl_log_work_bytes -> DL_ERR_INVALID_ARG)
  *   n      entries already in the log, 0 <= n < L; n >= L -> DL_ERR_LOG_FULL
  *   q, k, v, beta, a, o: as the eager step of the same decay kind. */
 dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind,

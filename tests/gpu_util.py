@@ -7,35 +7,14 @@ import numpy as np
 import workloads as W
 
 
-def to_torch(arr: np.ndarray, dtype: str, device="cuda"):
-    import torch
-
-    if dtype == "bf16":
-        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
-    else:
-        t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
-    return t.to(device)
+to_torch = W.to_torch
+device_inputs = W.device_inputs
 
 
 def state_to_f64(S) -> np.ndarray:
     import torch
 
     return S.detach().to(torch.float64).cpu().numpy()
-
-
-def device_inputs(w: W.Workload, x, device="cuda"):
-    """Stored inputs -> device tensors with the [B, H] axes restored."""
-    nh = x["S0"].shape[0]
-    B, H = (w.B, w.H) if nh == w.heads else (1, nh)
-    d = {}
-    d["S0"] = to_torch(x["S0"], w.state_dtype, device).view(B, H, w.d_v, w.d_k)
-    d["q"] = to_torch(x["q"], w.in_dtype, device).view(w.T, B, H, w.d_k)
-    d["k"] = to_torch(x["k"], w.in_dtype, device).view(w.T, B, H, w.d_k)
-    d["v"] = to_torch(x["v"], w.in_dtype, device).view(w.T, B, H, w.d_v)
-    d["beta"] = to_torch(x["beta"], w.in_dtype, device).view(w.T, B, H)
-    a_shape = (w.T, B, H) if w.decay == W.HEAD else (w.T, B, H, w.d_k)
-    d["a"] = to_torch(x["a"], w.in_dtype, device).view(*a_shape)
-    return d
 
 
 def run_cuda(w: W.Workload, d, path: str, L: int = 0, fused: bool = True, keep_o: bool = True,

@@ -1,0 +1,118 @@
+"""Host-side pieces of bench.py and of the schedule driver (CPU only)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+import workloads as W
+from gated_delta_rule_104_b200.schedule import DeferredDecoder
+
+
+class FakeOps:
+    def __init__(self):
+        self.calls = []
+
+    def dl_log_append_read(self, S, log, n, *a):
+        assert 0 <= n < log.L
+        self.calls.append(("append_read", n))
+
+    def dl_log_merge_read(self, S, log, n, *a):
+        assert 0 <= n < log.L
+        self.calls.append(("merge_read", n))
+
+    def dl_log_merge(self, S, log, n, *a):
+        assert 1 <= n <= log.L
+        self.calls.append(("merge", n))
+
+
+class FakeLog:
+    def __init__(self, L):
+        self.L = L
+
+
+def run_schedule(L, T, fused):
+    ops = FakeOps()
+    dec = DeferredDecoder(None, FakeLog(L), fused_merge=fused, ops=ops)
+    for _ in range(T):
+        dec.step(None, None, None, None, None, None)
+    dec.flush()
+    return ops.calls
+
+
+def test_unfused_schedule_appends_then_merges_full_log():
+    calls = run_schedule(4, 10, False)
+    assert calls == [("append_read", 0), ("append_read", 1), ("append_read", 2), ("append_read", 3), ("merge", 4),
+                     ("append_read", 0), ("append_read", 1), ("append_read", 2), ("append_read", 3), ("merge", 4),
+                     ("append_read", 0), ("append_read", 1), ("merge", 2)]
+
+
+def test_fused_schedule_merges_on_the_filling_step():
+    calls = run_schedule(4, 10, True)
+    assert calls == [("append_read", 0), ("append_read", 1), ("append_read", 2), ("merge_read", 3),
+                     ("append_read", 0), ("append_read", 1), ("append_read", 2), ("merge_read", 3),
+                     ("append_read", 0), ("append_read", 1), ("merge", 2)]
+
+
+@pytest.mark.parametrize("L", [1, 2, 16, 64])
+@pytest.mark.parametrize("fused", [True, False])
+def test_every_step_reads_once_and_log_never_overflows(L, fused):
+    T = 131
+    calls = run_schedule(L, T, fused)
+    assert sum(1 for k, _ in calls if k in ("append_read", "merge_read")) == T
+    n = 0
+    for kind, m in calls:
+        assert m == n if kind != "merge" else m == n
+        n = 0 if kind in ("merge", "merge_read") else n + 1
+        assert n <= L
+    assert n == 0  # flushed
+
+
+def test_bench_plan_matches_the_driver():
+    w = W.scaled(W.WORKLOADS["kda_b256_h32_d128_t512"], T=40)
+    for sched in ("fused", "unfused"):
+        lau = bench.Launcher(None, w, None, None, FakeLog(16), None, sched, None)
+        assert lau.plan() == run_schedule(16, 40, sched == "fused")
+    lau = bench.Launcher(None, w, None, None, None, None, "eager", None)
+    assert lau.plan() == [("eager", 0)] * 40
+
+
+def test_byte_model_matches_the_state_sizes():
+    w = W.WORKLOADS["kda_b256_h32_d128_t512"]
+    assert w.state_bytes() == 512 << 20
+    assert bench.entry_bytes(w) == (128 + 128 + 1 + 128) * 2 == 770
+    # eager moves the state twice, the deferred read once
+    assert bench.alg_bytes(w, "eager", 0) - 2 * w.state_bytes() == w.heads * (770 + 256 + 512)
+    assert bench.alg_bytes(w, "append_read", 3) - w.state_bytes() == w.heads * (5 * 770 + 256 + 512)
+    w4 = W.WORKLOADS["gdn_b1024_h32_dk128_dv256_t256"]
+    assert w4.state_bytes() == 2 << 30 and bench.entry_bytes(w4) == (128 + 256 + 2) * 2
+
+
+def test_reduce_max_without_process_group():
+    assert bench.reduce_max(3.5) == 3.5
+
+
+GLOO_SCRIPT = r"""
+import os, sys
+sys.path.insert(0, os.environ["REPO"])
+import torch.distributed as dist
+import bench
+dist.init_process_group("gloo", init_method="env://")
+r = dist.get_rank()
+m = bench.reduce_max(10.0 + r)            # per-rank device times -> the max
+assert m == 11.0, m
+print("rank", r, "ok", m, flush=True)
+dist.destroy_process_group()
+"""
+
+
+def test_max_over_ranks_gloo_world2(tmp_path):
+    script = tmp_path / "gloo_max.py"
+    script.write_text(GLOO_SCRIPT)
+    env = dict(os.environ, REPO=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", "--master-port=29613", str(script)]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.count("ok 11.0") == 2

@@ -81,7 +81,8 @@ def test_scalar_operands_need_only_element_alignment(lib):
 
 
 def make_log(L=8, dtype=b.DL_BF16, base=10):
-    return b.dl_log(addr(base), addr(base + 1), addr(base + 2), addr(base + 3), dtype, L)
+    return b.dl_log(addr(base), addr(base + 1), addr(base + 2), addr(base + 3), dtype, L, addr(base + 4),
+                    2 * 3 * (128 + 128) * 4)
 
 
 def append(lib, fn="dl_log_append_read", log=None, n=0, kind=b.DL_DECAY_CHANNEL, S=None, dk=128, dv=128,
@@ -110,6 +111,21 @@ def test_log_step_argument_checks(lib, fn):
     lo = make_log()
     lo.k = addr(0) + 256                                                 # log inside the base
     assert append(lib, fn, log=lo) == b.DL_ERR_INVALID_ARG
+
+
+def test_append_read_workspace_checks(lib):
+    assert lib.dl_log_work_bytes(2, 3, 128, 128) == 2 * 3 * 256 * 4
+    lg = make_log()
+    lg.work = None
+    assert append(lib, log=lg) == b.DL_ERR_INVALID_ARG
+    assert "log.work is a null pointer" in lib.dl_last_error().decode()
+    lg = make_log()
+    lg.work_bytes = 100
+    assert append(lib, log=lg) == b.DL_ERR_INVALID_ARG
+    assert "needs" in lib.dl_last_error().decode()
+    lg = make_log()
+    lg.work = addr(0) + 512  # workspace inside the base
+    assert append(lib, log=lg) == b.DL_ERR_INVALID_ARG
 
 
 def test_merge_argument_checks(lib):

@@ -256,3 +256,33 @@ def as_f64(w: Workload, inputs: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
         dt = w.state_dtype if key == "S0" else w.in_dtype
         out[key] = to_f64(arr, dt)
     return out
+
+
+# ---------------------------------------------------------------- device copies
+
+def to_torch(arr: np.ndarray, dtype: str, device="cuda"):
+    """A stored array (float32, or bf16 bits as uint16) as a torch tensor."""
+    import torch
+
+    if dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+    return t.to(device)
+
+
+def device_inputs(w: Workload, x: Dict[str, np.ndarray], device="cuda"):
+    """Generated inputs as device tensors with the [B, H] head axes restored
+    (a subset of heads becomes B = 1, H = number of heads)."""
+    nh = x["S0"].shape[0]
+    B, H = (w.B, w.H) if nh == w.heads else (1, nh)
+    d = {
+        "S0": to_torch(x["S0"], w.state_dtype, device).view(B, H, w.d_v, w.d_k),
+        "q": to_torch(x["q"], w.in_dtype, device).view(w.T, B, H, w.d_k),
+        "k": to_torch(x["k"], w.in_dtype, device).view(w.T, B, H, w.d_k),
+        "v": to_torch(x["v"], w.in_dtype, device).view(w.T, B, H, w.d_v),
+        "beta": to_torch(x["beta"], w.in_dtype, device).view(w.T, B, H),
+    }
+    a_shape = (w.T, B, H) if w.decay == HEAD else (w.T, B, H, w.d_k)
+    d["a"] = to_torch(x["a"], w.in_dtype, device).view(*a_shape)
+    return d
