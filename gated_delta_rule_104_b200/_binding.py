@@ -21,7 +21,9 @@ DL_MAX_LOG = 64
 ABI_VERSION = 2
 
 EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
-           "dl_log_merge_read", "dl_log_work_bytes", "dl_status_string", "dl_last_error", "dl_abi_version")
+           "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_status_string",
+           "dl_last_error", "dl_abi_version")
+DL_NOALLOC_WORK_BYTES = 16 << 20
 
 
 class DeltaLogError(RuntimeError):
@@ -228,3 +230,16 @@ def dl_log_merge(S_base, log: Log, n: int, stream=None) -> None:
 
 def dl_status_string(status: int) -> str:
     return load().dl_status_string(int(status)).decode()
+
+
+def dl_log_append_read_noalloc(S_base, log: Log, n: int, q, k, v, beta, a, o, stream=None) -> None:
+    """As dl_log_append_read, with the scratch in the library's fixed device
+    array instead of ``log.work``: for callers that cannot allocate device
+    memory. Calls that overlap on the GPU race on that array."""
+    lib = load()
+    fn = lib.dl_log_append_read_noalloc
+    if fn.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        fn.argtypes = [vp, i, i, ctypes.POINTER(dl_log), i, vp, vp, vp, vp, vp, i, vp, i, i, i, i, vp]
+        fn.restype = ctypes.c_int
+    _log_step("dl_log_append_read_noalloc", S_base, log, n, q, k, v, beta, a, o, stream)

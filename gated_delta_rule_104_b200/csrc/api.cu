@@ -209,6 +209,34 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind, const
     return cuda_status(dl::launch_merge(p, lg, n, true, stream), "merge-read launch");
 }
 
+dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log,
+                                     int n, const void *q, const void *k, const void *v, const void *beta,
+                                     const void *a, dl_dtype in_dtype, float *o, int B, int H, int d_k, int d_v,
+                                     cudaStream_t stream) {
+    dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
+    if (s != DL_OK) return s;
+    if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
+    const bool chan = kind == DL_DECAY_CHANNEL;
+    Buf b[11];
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    nb += 4;
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
+    const size_t need = dl::read_work_bytes(B, H, d_k, d_v);
+    if (need > DL_NOALLOC_WORK_BYTES)
+        return fail(DL_ERR_UNSUPPORTED,
+                    "B*H*(d_k+d_v)*4 = %zu bytes of scratch exceeds the built-in %zu-byte array "
+                    "(DL_NOALLOC_WORK_BYTES); use dl_log_append_read with a workspace",
+                    need, (size_t)DL_NOALLOC_WORK_BYTES);
+    const Buf writers[5] = {b[6], b[7], b[8], b[9], b[10]};  // o and the log
+    if ((s = check_overlap(writers, 5, b, nb)) != DL_OK) return s;
+    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    return cuda_status(dl::launch_append_read_noalloc(p, lg, n, stream), "no-alloc append-read launch");
+}
+
 const char *dl_status_string(dl_status s) {
     switch (s) {
         case DL_OK: return "ok";

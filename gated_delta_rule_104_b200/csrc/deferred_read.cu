@@ -24,6 +24,8 @@
 //                 It may start while replay_prep still runs: it issues its
 //                 base loads first and waits for the prep grid only before
 //                 reading the workspace.
+#include <mutex>
+
 #include "launch.h"
 
 namespace dl {
@@ -213,6 +215,48 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     });
+}
+
+// ------------------------------------------------------------------ no-allocation variant
+//
+// dl_log_append_read_noalloc runs the same two kernels with their scratch in
+// this fixed module-level array instead of a caller-provided workspace, for
+// callers that cannot allocate device memory. The array belongs to the CUDA
+// module of this file, so every device that loads the library holds it until
+// the process exits. All calls share it: calls whose kernels overlap on the
+// GPU (different streams, or different host threads) race on it and must be
+// serialised by the caller. Nothing in it needs clearing between calls:
+// replay_prep writes every (x_0, w) value the decode kernel then reads.
+static __device__ __align__(256) float g_noalloc_work[DL_NOALLOC_WORK_BYTES / sizeof(float)];
+
+// Device address of g_noalloc_work on the current device. Host code may not
+// hand the symbol itself to a kernel (on the host it names a host-side
+// stand-in), so the address is looked up with cudaGetSymbolAddress once per
+// device, with that device current, and cached.
+static cudaError_t noalloc_work_address(float **out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static float *addr[kMaxDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        float *ptr = nullptr;
+        e = cudaGetSymbolAddress((void **)&ptr, g_noalloc_work);
+        if (e != cudaSuccess) return e;
+        addr[dev] = ptr;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
+cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg, int n, cudaStream_t st) {
+    float *work = nullptr;
+    cudaError_t e = noalloc_work_address(&work);
+    if (e != cudaSuccess) return e;
+    return launch_append_read(p, lg, n, work, st);
 }
 
 }  // namespace dl

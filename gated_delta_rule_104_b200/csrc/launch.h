@@ -27,6 +27,8 @@ cudaError_t launch_eager(const StepParams &p, cudaStream_t st);
 // Deferred read: needs read_work_bytes() of fp32 workspace (x_0 and w per head).
 cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st);
 size_t read_work_bytes(int B, int H, int dk, int dv);
+// The same with the scratch in a fixed module array (DL_NOALLOC_WORK_BYTES).
+cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg, int n, cudaStream_t st);
 // Merge n_log log entries (plus, if with_cur, this step's inputs as one more
 // entry, and then o = S_new q) into the base.
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,

@@ -160,6 +160,36 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind,
                             float *o, int B, int H, int d_k, int d_v,
                             cudaStream_t stream);
 
+/* Deferred step that allocates nothing and needs no workspace from the caller.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory, such as a serving engine whose caching
+ * allocator has already reserved the device's memory for its state pool, a
+ * plugin host that hands a kernel only its input and output buffers, or a
+ * latency-critical decode loop where a cudaMalloc would synchronise the
+ * device. It computes exactly what dl_log_append_read computes, with the same
+ * arguments and checks, except that log->work is ignored (it may be null):
+ * the per-head scratch lives in a fixed array of DL_NOALLOC_WORK_BYTES inside
+ * the library, which every device that loads the library keeps until the
+ * process exits.
+ *   Limit      B * H * (d_k + d_v) * 4 <= DL_NOALLOC_WORK_BYTES (16 MiB, e.g.
+ *              B * H = 8192 heads at d_k = d_v = 128); larger -> DL_ERR_UNSUPPORTED.
+ *   Set-up     the first call on each device looks up the array's device
+ *              address (cudaGetSymbolAddress) with that device current; make
+ *              that first call before any stream capture.
+ *   Sharing    every call uses the same array and leaves its contents behind;
+ *              calls whose work overlaps on the GPU (other streams or host
+ *              threads) race on it, so the caller must serialise them. No
+ *              part of the array needs clearing between calls.
+ * It calls no cudaMalloc, cudaFree or other allocating routine. */
+#define DL_NOALLOC_WORK_BYTES (16u << 20)
+dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_decay kind,
+                                     const dl_log *log, int n,
+                                     const void *q, const void *k, const void *v,
+                                     const void *beta, const void *a, dl_dtype in_dtype,
+                                     float *o, int B, int H, int d_k, int d_v,
+                                     cudaStream_t stream);
+
 /* Static text for a status code. */
 const char *dl_status_string(dl_status s);
 
