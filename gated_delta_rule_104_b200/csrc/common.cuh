@@ -131,6 +131,29 @@ __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// Sum each of N values (N a power of two, 2..32) over all 32 lanes of the
+// warp at once with a transposing butterfly: every exchange step halves the
+// values a lane keeps, so the whole reduction costs N - 1 + (5 - log2 N)
+// shuffles instead of 5 N. Afterwards v[0] of lane l holds the warp-wide sum
+// of entry l >> (5 - log2 N).
+template <int N>
+__device__ __forceinline__ void multi_sum(float (&v)[N], int lane) {
+    static_assert(N >= 2 && N <= 32 && (N & (N - 1)) == 0, "power of two");
+#pragma unroll
+    for (int half = N / 2, off = 16; half >= 1; half >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float keep = upper ? v[i + half] : v[i];
+            const float send = upper ? v[i] : v[i + half];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    constexpr int steps = (N == 2 ? 1 : N == 4 ? 2 : N == 8 ? 3 : N == 16 ? 4 : 5);
+#pragma unroll
+    for (int off = 16 >> steps; off > 0; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+}
+
 // ---------------------------------------------------------------- staging
 
 // Copy a rows x cols block of IT (each row contiguous in global memory, row
