@@ -286,3 +286,41 @@ def device_inputs(w: Workload, x: Dict[str, np.ndarray], device="cuda"):
     a_shape = (w.T, B, H) if w.decay == HEAD else (w.T, B, H, w.d_k)
     d["a"] = to_torch(x["a"], w.in_dtype, device).view(*a_shape)
     return d
+
+
+def device_inputs_chunked(w: Workload, device="cuda", workers: int = 1, chunk_heads: int = 2048):
+    """Like ``device_inputs(w, generate(w))`` for all heads, but generated
+    ``chunk_heads`` heads at a time and copied straight into the device
+    tensors, so the host never holds the whole workload."""
+    import torch
+
+    it = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    st = torch.bfloat16 if w.state_dtype == "bf16" else torch.float32
+    nh = w.heads
+    d = {
+        "S0": torch.empty(nh, w.d_v, w.d_k, dtype=st, device=device),
+        "q": torch.empty(w.T, nh, w.d_k, dtype=it, device=device),
+        "k": torch.empty(w.T, nh, w.d_k, dtype=it, device=device),
+        "v": torch.empty(w.T, nh, w.d_v, dtype=it, device=device),
+        "beta": torch.empty(w.T, nh, dtype=it, device=device),
+        "a": torch.empty(*((w.T, nh) if w.decay == HEAD else (w.T, nh, w.d_k)), dtype=it, device=device),
+    }
+    for h0 in range(0, nh, chunk_heads):
+        heads = list(range(h0, min(nh, h0 + chunk_heads)))
+        x = generate(w, heads=heads, workers=workers)
+        for key, arr in x.items():
+            dt = w.state_dtype if key == "S0" else w.in_dtype
+            t = to_torch(arr, dt, device)
+            if key == "S0":
+                d[key][h0:h0 + len(heads)] = t
+            else:
+                d[key][:, h0:h0 + len(heads)] = t
+        del x
+    B, H = w.B, w.H
+    d["S0"] = d["S0"].view(B, H, w.d_v, w.d_k)
+    d["q"] = d["q"].view(w.T, B, H, w.d_k)
+    d["k"] = d["k"].view(w.T, B, H, w.d_k)
+    d["v"] = d["v"].view(w.T, B, H, w.d_v)
+    d["beta"] = d["beta"].view(w.T, B, H)
+    d["a"] = d["a"].view(*((w.T, B, H) if w.decay == HEAD else (w.T, B, H, w.d_k)))
+    return d
