@@ -64,18 +64,22 @@ def alg_bytes(w: W.Workload, kind: str, n: int) -> int:
 
     eager:        state read + write, this step's inputs, o
     append_read:  state read (no write), n log entries read, one entry
-                  written, this step's inputs, o
-    merge_read:   state read + write, n log entries, this step's inputs, o
-    merge:        state read + write, n log entries
+                  written, this step's inputs, o, and the log metadata: the
+                  older entries' C rows read (n(n-1)/2 floats), the new row
+                  written (n floats)
+    merge_read:   state read + write, n log entries and their C rows, this
+                  step's inputs, o
+    merge:        state read + write, n log entries and their C rows
     """
     e, S = entry_bytes(w), state_bytes_head(w)
     s_in = 2 if w.in_dtype == "bf16" else 4
     q, o = w.d_k * s_in, 4 * w.d_v
+    crows = 4 * n * (n - 1) // 2
     per_head = {
         "eager": 2 * S + e + q + o,
-        "append_read": S + n * e + e + e + q + o,
-        "merge_read": 2 * S + n * e + e + q + o,
-        "merge": 2 * S + n * e,
+        "append_read": S + n * e + e + e + q + o + crows + 4 * n,
+        "merge_read": 2 * S + n * e + e + q + o + crows,
+        "merge": 2 * S + n * e + crows,
     }[kind]
     return per_head * w.heads
 

@@ -97,6 +97,7 @@ dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, i
     out[1] = {"log.v", log->v, bhl * dv * is, 16};
     out[2] = {"log.beta", log->beta, bhl * is, is};
     out[3] = chan ? Buf{"log.a", log->a, bhl * dk * is, 16} : Buf{"log.a", log->a, bhl * is, is};
+    out[4] = {"log.c", log->c, bhl * log->L * sizeof(float), 16};
     return DL_OK;
 }
 
@@ -143,10 +144,10 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     const bool chan = kind == DL_DECAY_CHANNEL;
-    Buf b[12];
+    Buf b[13];
     int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
     if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
-    nb += 4;
+    nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
     if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
@@ -156,11 +157,11 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     if (log->work_bytes < need)
         return fail(DL_ERR_INVALID_ARG, "log.work holds %zu bytes, needs %zu", log->work_bytes, need);
     ++nb;
-    // written: o, the log (slot n) and its workspace; the base is only read.
-    const Buf writers[6] = {b[6], b[7], b[8], b[9], b[10], b[11]};
-    if ((s = check_overlap(writers, 6, b, nb)) != DL_OK) return s;
+    // written: o, the log (slot n, metadata row n) and its workspace; the base is only read.
+    const Buf writers[7] = {b[6], b[7], b[8], b[9], b[10], b[11], b[12]};
+    if ((s = check_overlap(writers, 7, b, nb)) != DL_OK) return s;
     dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
     return cuda_status(dl::launch_append_read(p, lg, n, static_cast<float *>(log->work), stream),
                        "append-read launch");
 }
@@ -172,18 +173,18 @@ dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_l
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     const bool chan = kind == DL_DECAY_CHANNEL;
     if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
-    Buf b[5];
+    Buf b[6];
     b[0] = {"S_base", S_base, (size_t)B * H * d_v * d_k * elem_size(s_dtype), 16};
     if ((s = check_log(log, b + 1, log->dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
-    if ((s = check_bufs(b, 5)) != DL_OK) return s;
+    if ((s = check_bufs(b, 6)) != DL_OK) return s;
     if (n < 1 || n > log->L) return fail(DL_ERR_INVALID_ARG, "merge needs 1 <= n <= L (n=%d, L=%d)", n, log->L);
     const Buf writers[1] = {b[0]};
-    if ((s = check_overlap(writers, 1, b, 5)) != DL_OK) return s;
-    const Buf logw[4] = {b[1], b[2], b[3], b[4]};
-    if ((s = check_overlap(logw, 4, b + 1, 4)) != DL_OK) return s;
+    if ((s = check_overlap(writers, 1, b, 6)) != DL_OK) return s;
+    const Buf logw[5] = {b[1], b[2], b[3], b[4], b[5]};
+    if ((s = check_overlap(logw, 5, b + 1, 5)) != DL_OK) return s;
     dl::StepParams p{S_base, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, chan,
                      s_dtype, log->dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, false, stream), "merge launch");
 }
 
@@ -195,17 +196,17 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind, const
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     const bool chan = kind == DL_DECAY_CHANNEL;
-    Buf b[11];
+    Buf b[12];
     int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
     if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
-    nb += 4;
+    nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
     if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
     const Buf writers[2] = {b[0], b[6]};  // the base and o
     if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
     dl::StepParams p{S_base, q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, true, stream), "merge-read launch");
 }
 
@@ -217,10 +218,10 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     const bool chan = kind == DL_DECAY_CHANNEL;
-    Buf b[11];
+    Buf b[12];
     int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
     if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
-    nb += 4;
+    nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
     if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
@@ -230,10 +231,10 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
                     "B*H*(d_k+d_v)*4 = %zu bytes of scratch exceeds the built-in %zu-byte array "
                     "(DL_NOALLOC_WORK_BYTES); use dl_log_append_read with a workspace",
                     need, (size_t)DL_NOALLOC_WORK_BYTES);
-    const Buf writers[5] = {b[6], b[7], b[8], b[9], b[10]};  // o and the log
-    if ((s = check_overlap(writers, 5, b, nb)) != DL_OK) return s;
+    const Buf writers[6] = {b[6], b[7], b[8], b[9], b[10], b[11]};  // o and the log
+    if ((s = check_overlap(writers, 6, b, nb)) != DL_OK) return s;
     dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
     return cuda_status(dl::launch_append_read_noalloc(p, lg, n, stream), "no-alloc append-read launch");
 }
 

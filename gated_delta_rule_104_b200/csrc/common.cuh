@@ -119,6 +119,89 @@ __device__ __forceinline__ uint4 ld_ro_stream(const void *p) {
     return r;
 }
 
+// L2 residency policies (createpolicy). The deferred path keeps its log --
+// a few hundred bytes per head per entry -- in L2 across steps (evict_last),
+// while the base state streams through once per step (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_keep() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_stream() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// Read-only 16-byte stream load under an L2 policy, no L1 allocation.
+__device__ __forceinline__ uint4 ld_ro_hint(const void *p, uint64_t pol) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(pol));
+    return r;
+}
+// Loads / stores of small operands under an L2 policy (bytes: 2, 4, 8, 16).
+template <int BYTES> struct HintWord;
+template <> struct HintWord<2> { using T = unsigned short; };
+template <> struct HintWord<4> { using T = uint32_t; };
+template <> struct HintWord<8> { using T = uint2; };
+template <> struct HintWord<16> { using T = uint4; };
+
+__device__ __forceinline__ void st_hint(void *p, unsigned short v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(v), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_hint(void *p, uint32_t v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_hint(void *p, uint2 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_hint(void *p, uint4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void ld_hint(const void *p, unsigned short &v, uint64_t pol) {
+    asm volatile("ld.global.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(v) : "l"(p), "l"(pol));
+}
+__device__ __forceinline__ void ld_hint(const void *p, uint32_t &v, uint64_t pol) {
+    asm volatile("ld.global.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(v) : "l"(p), "l"(pol));
+}
+__device__ __forceinline__ void ld_hint(const void *p, uint2 &v, uint64_t pol) {
+    asm volatile("ld.global.L2::cache_hint.v2.b32 {%0, %1}, [%2], %3;" : "=r"(v.x), "=r"(v.y) : "l"(p), "l"(pol));
+}
+__device__ __forceinline__ void ld_hint(const void *p, uint4 &v, uint64_t pol) {
+    asm volatile("ld.global.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+}
+// Copy N elements of T (N * sizeof(T) a power of two >= 2 bytes, aligned to
+// min(16, that)) from src to dst, writing under an L2 policy.
+template <int N, class T>
+__device__ __forceinline__ void copy_hint(T *dst, const T *src, uint64_t pol) {
+    constexpr int BYTES = N * (int)sizeof(T), W = BYTES < 16 ? BYTES : 16, K = BYTES / W;
+    using Word = typename HintWord<W>::T;
+#pragma unroll
+    for (int i = 0; i < K; ++i)
+        st_hint(reinterpret_cast<unsigned char *>(dst) + i * W,
+                *reinterpret_cast<const Word *>(reinterpret_cast<const unsigned char *>(src) + i * W), pol);
+}
+// N elements of T (as load_vec) read under an L2 policy, widened to float.
+template <int N, class T>
+__device__ __forceinline__ void load_vec_hint(const T *p, float (&x)[N], uint64_t pol) {
+    constexpr int BYTES = N * (int)sizeof(T), W = BYTES < 16 ? BYTES : 16, K = BYTES / W, PER = W / (int)sizeof(T);
+    using Word = typename HintWord<W>::T;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        Word w;
+        ld_hint(reinterpret_cast<const unsigned char *>(p) + i * W, w, pol);
+        const T *e = reinterpret_cast<const T *>(&w);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) x[i * PER + j] = to_f(e[j]);
+    }
+}
+
 // ---------------------------------------------------------------- reductions
 
 // Sum over aligned groups of G consecutive lanes (G a power of two <= 32);
@@ -191,6 +274,11 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
     asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async16_hint(void *smem_dst, const void *gmem_src, uint64_t pol) {
+    uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem_src), "l"(pol)
+                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }

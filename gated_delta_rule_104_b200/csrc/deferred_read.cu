@@ -4,26 +4,35 @@
 // computed once per slot-head in a "ReplayPrep" stage and shared by the value
 // tiles, which then run in parallel "AppendDecode" stages).
 //
-// With A_i = Diag(a_i)(I - beta_i k_i k_i^T), the logical state after log
-// entries 1..n is S_n = S_bar A_1...A_n + sum_i beta_i v_i k_i^T A_{i+1}...A_n,
-// so o = S_n q needs only
-//   key side (once per head):   x_n = q; for i = n..1:
-//        c_i = k_i . x_i,  s_i = beta_i c_i,  x_{i-1} = a_i o (x_i - s_i k_i)
-//        and w = sum_i s_i v_i            (a d_v vector)
-//   value side (per row r):     o_r = S_bar[r] . x_0 + w_r.
-// The base is read once and never written.
+// With A_e = Diag(a_e)(I - beta_e k_e k_e^T), entries e = 0..n (n is this
+// step's, the newest), the logical state is S_bar A_0 ... A_n-style replayed
+// and o = S_n q needs only, per head, the vector x_0 and the scalars s_e of
+// the key-side recursion (x <- q; for e = n..0: s_e = beta_e k_e . x,
+// x <- a_e o (x - s_e k_e)), then per row r: o_r = S_bar[r] . x_0 + w_r with
+// w = sum_e s_e v_e. The base is read once and never written.
+//
+// ReplayPrep evaluates that recursion in parallel form. With the decay
+// products D(j, e) = prod_{m=e+1..j} a_m (the page's log-decay metadata as
+// products) and the decayed key inner products C(j, e) = k_e . (D(j, e) o k_j)
+// for e < j:
+//   d_e = k_e . (D(n, e) o q)                    (independent dots)
+//   s_e = beta_e (d_e - sum_{j>e} C(j, e) s_j)   (a short scalar back-substitution)
+//   x_0 = gamma_n o q - sum_e s_e (gamma_e o k_e),  gamma_e = prod_{m<=e} a_m.
+// The C rows are kept with the log: each append computes C(n, e) for the
+// new entry (the same kind of dots as d_e) and stores it in log.c, so a read
+// never recomputes older rows and the merge reuses them.
 //
 // Two kernels, chained with programmatic dependent launch:
-//   replay_prep   one warp per head: appends the entry, runs the serial
-//                 recursion (lanes own d_k/32 key columns, one shuffle
-//                 reduction per entry) and w, and stores (x_0, w) in the
+//   replay_prep   one warp per head: stages the head's log keys and decays
+//                 in shared memory (cp.async), appends the entry, forms all
+//                 d_e and C(n, e) with one transposing butterfly per 32
+//                 entries, back-substitutes s, and stores (x_0, w) in the
 //                 caller's workspace [B*H][d_k + d_v] fp32.
-//   append_decode a pure streaming pass over the base, laid out like the
-//                 eager kernel (a row spread over 16-byte lane slices, 8 loads
-//                 in flight per thread, no shared memory, no block barrier).
-//                 It may start while replay_prep still runs: it issues its
-//                 base loads first and waits for the prep grid only before
-//                 reading the workspace.
+//   append_decode a pure streaming pass over the base (a row spread over
+//                 16-byte lane slices, 8 loads in flight per thread, no
+//                 shared memory, no block barrier). It may start while
+//                 replay_prep still runs: it issues its base loads first and
+//                 waits for the prep grid only before reading the workspace.
 #include <mutex>
 
 #include "launch.h"
@@ -32,95 +41,192 @@ namespace dl {
 
 // ------------------------------------------------------------------ prep
 
-template <class IT, int DK, int DV, bool CHAN>
-__global__ void __launch_bounds__(256)
+template <class IT, int DK, int EMAX, bool CHAN>
+struct PrepSmem {  // one warp's staging area
+    static constexpr int ROWB = DK * (int)sizeof(IT);           // bytes of one key row
+    static constexpr int K_OFF = 0;
+    static constexpr int A_OFF = K_OFF + EMAX * ROWB;           // channel decays (raw)
+    static constexpr int F_OFF = A_OFF + (CHAN ? EMAX * ROWB : 0);
+    // floats from F_OFF: as[EMAX], beta[EMAX], d[EMAX], cn[EMAX], sv[EMAX], crow[EMAX][EMAX]
+    static constexpr int FLOATS = 5 * EMAX + EMAX * EMAX;
+    static constexpr int BYTES = F_OFF + FLOATS * 4;
+};
+
+template <class IT, int DK, int DV, bool CHAN, int EMAX>
+__global__ void __launch_bounds__(128)
 replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                    const IT *__restrict__ beta, const IT *__restrict__ a, IT *__restrict__ log_k,
-                   IT *__restrict__ log_v, IT *__restrict__ log_b, IT *__restrict__ log_a, int L, int n,
-                   float *__restrict__ work, long long heads) {
+                   IT *__restrict__ log_v, IT *__restrict__ log_b, IT *__restrict__ log_a,
+                   float *__restrict__ log_c, int L, int n, float *__restrict__ work, long long heads) {
     pdl_launch_dependents();
-    constexpr int CW = DK / 32;   // key columns per lane
-    constexpr int RV = DV / 32;   // value rows per lane
-    constexpr int CHUNK = 4;      // log entries fetched together
-    const int lane = threadIdx.x & 31;
-    const long long head = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    using P = PrepSmem<IT, DK, EMAX, CHAN>;
+    constexpr int CW = DK / 32;            // key columns per lane (contiguous)
+    constexpr int RV = DV / 32;            // value rows per lane
+    constexpr int CH = EMAX < 32 ? EMAX : 32;  // entries per butterfly
+    constexpr int SLOTS = (EMAX + 31) / 32;    // entries owned per lane in the back-substitution
+    constexpr int E = 16 / (int)sizeof(IT);    // elements per 16-byte chunk
+    extern __shared__ float4 smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char *base = reinterpret_cast<unsigned char *>(smem_raw) + (size_t)warp * P::BYTES;
+    IT *sk = reinterpret_cast<IT *>(base + P::K_OFF);
+    IT *sa = reinterpret_cast<IT *>(base + P::A_OFF);
+    float *fas = reinterpret_cast<float *>(base + P::F_OFF);
+    float *fbeta = fas + EMAX, *fd = fbeta + EMAX, *fcn = fd + EMAX, *fs = fcn + EMAX, *crow = fs + EMAX;
+
+    const long long head = (long long)blockIdx.x * (blockDim.x / 32) + warp;
     if (head >= heads) return;
     const long long lrow = head * L;
     const int c0 = lane * CW, r0 = lane * RV;
+    // The log stays L2-resident between steps: its reads and writes carry an
+    // evict-last policy (the base streams through with evict-first).
+    const uint64_t keep = l2_policy_keep();
 
-    // This step's entry (index n), from the inputs.
-    float kc[CW], ac[CW], vc[RV], x[CW];
-    load_vec<CW>(k + head * DK + c0, kc);
-    load_vec<RV>(v + head * DV + r0, vc);
-    load_vec<CW>(q + head * DK + c0, x);
-    if constexpr (CHAN) {
-        load_vec<CW>(a + head * DK + c0, ac);
-    } else {
-        const float as = to_f(a[head]);
-#pragma unroll
-        for (int e = 0; e < CW; ++e) ac[e] = as;
+    // Stage keys and decays of entries 0..n-1 (log) and n (this step), raw.
+    for (int u = lane; u < (n + 1) * (DK / E); u += 32) {
+        const int e = u / (DK / E), col = (u % (DK / E)) * E;
+        if (e < n) {
+            cp_async16_hint(sk + e * DK + col, log_k + (lrow + e) * DK + col, keep);
+            if constexpr (CHAN) cp_async16_hint(sa + e * DK + col, log_a + (lrow + e) * DK + col, keep);
+        } else {
+            cp_async16(sk + e * DK + col, k + head * DK + col);
+            if constexpr (CHAN) cp_async16(sa + e * DK + col, a + head * DK + col);
+        }
     }
-    const float bc = to_f(beta[head]);
-
+    cp_async_commit();
+    for (int e = lane; e <= n; e += 32) {
+        float bx[1];
+        if (e < n) load_vec_hint<1>(log_b + lrow + e, bx, keep);
+        else bx[0] = to_f(beta[head]);
+        fbeta[e] = bx[0];
+        if constexpr (!CHAN) {
+            float ax[1];
+            if (e < n) load_vec_hint<1>(log_a + lrow + e, ax, keep);
+            else ax[0] = to_f(a[head]);
+            fas[e] = ax[0];
+        }
+    }
+    // C(j, e) of the logged entries (rows j < n, columns e < j).
+    for (int u = lane; u < n * EMAX; u += 32) {
+        const int j = u / EMAX, e = u % EMAX;
+        if (e < j) {
+            float cx[1];
+            load_vec_hint<1>(log_c + (lrow + j) * L + e, cx, keep);
+            crow[j * EMAX + e] = cx[0];
+        }
+    }
     // D1: the entry is appended unchanged (raw input elements).
-#pragma unroll
-    for (int e = 0; e < CW; ++e) log_k[(lrow + n) * DK + c0 + e] = k[head * DK + c0 + e];
-#pragma unroll
-    for (int e = 0; e < RV; ++e) log_v[(lrow + n) * DV + r0 + e] = v[head * DV + r0 + e];
+    copy_hint<CW>(log_k + (lrow + n) * DK + c0, k + head * DK + c0, keep);
+    copy_hint<RV>(log_v + (lrow + n) * DV + r0, v + head * DV + r0, keep);
     if constexpr (CHAN) {
-#pragma unroll
-        for (int e = 0; e < CW; ++e) log_a[(lrow + n) * DK + c0 + e] = a[head * DK + c0 + e];
+        copy_hint<CW>(log_a + (lrow + n) * DK + c0, a + head * DK + c0, keep);
     } else if (lane == 0) {
-        log_a[lrow + n] = a[head];
+        copy_hint<1>(log_a + lrow + n, a + head, keep);
     }
-    if (lane == 0) log_b[lrow + n] = beta[head];
+    if (lane == 0) copy_hint<1>(log_b + lrow + n, beta + head, keep);
+    float qv[CW];
+    load_vec<CW>(q + head * DK + c0, qv);
+    cp_async_wait_all();
+    __syncwarp();
 
-    // D2: the recursion, newest entry first.
+    auto decay = [&](int e, float (&ae)[CW]) {
+        if constexpr (CHAN) {
+            load_vec<CW>(sa + e * DK + c0, ae);
+        } else {
+#pragma unroll
+            for (int c = 0; c < CW; ++c) ae[c] = fas[e];
+        }
+    };
+
+    // d_e = k_e . (D(n, e) o q) and C(n, e) = k_e . (D(n, e) o k_n), newest first.
+    float z[CW], y[CW];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) z[c] = qv[c];
+    load_vec<CW>(sk + n * DK + c0, y);
+    for (int top = n; top >= 0; top -= CH) {
+        float pd[CH], pc[CH];
+#pragma unroll
+        for (int jj = 0; jj < CH; ++jj) {
+            pd[jj] = 0.f;
+            pc[jj] = 0.f;
+            const int e = top - jj;
+            if (e >= 0) {
+                float ke[CW], ae[CW];
+                load_vec<CW>(sk + e * DK + c0, ke);
+                decay(e, ae);
+#pragma unroll
+                for (int c = 0; c < CW; ++c) {
+                    pd[jj] = fmaf(ke[c], z[c], pd[jj]);
+                    pc[jj] = fmaf(ke[c], y[c], pc[jj]);
+                    z[c] *= ae[c];
+                    y[c] *= ae[c];
+                }
+            }
+        }
+        multi_sum<CH>(pd, lane);
+        multi_sum<CH>(pc, lane);
+        constexpr int shift = CH == 32 ? 0 : CH == 16 ? 1 : CH == 8 ? 2 : 3;
+        const int e = top - (lane >> shift);
+        if ((lane & ((1 << shift) - 1)) == 0 && e >= 0) {
+            fd[e] = pd[0];
+            fcn[e] = pc[0];  // (C(n, n) is not used)
+        }
+    }
+    __syncwarp();
+    for (int e = lane; e < n; e += 32) copy_hint<1>(log_c + (lrow + n) * L + e, fcn + e, keep);
+
+    // s_e = beta_e (d_e - sum_{j>e} C(j, e) s_j), from the newest entry down.
+    float acc[SLOTS];
+#pragma unroll
+    for (int t = 0; t < SLOTS; ++t) acc[t] = 0.f;
+    for (int j = n; j >= 0; --j) {
+        if (lane == (j & 31)) fs[j] = fbeta[j] * (fd[j] - acc[j >> 5]);
+        __syncwarp();
+        const float sj = fs[j];
+        const float *cj = j == n ? fcn : crow + j * EMAX;
+#pragma unroll
+        for (int t = 0; t < SLOTS; ++t) {
+            const int e = lane + 32 * t;
+            if (e < j) acc[t] = fmaf(cj[e], sj, acc[t]);
+        }
+    }
+    __syncwarp();
+
+    // x_0 = gamma_n o q - sum_e s_e (gamma_e o k_e);  w = sum_e s_e v_e.
+    float g[CW], xs[CW];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+        g[c] = 1.f;
+        xs[c] = 0.f;
+    }
+    for (int e = 0; e <= n; ++e) {
+        float ke[CW], ae[CW];
+        load_vec<CW>(sk + e * DK + c0, ke);
+        decay(e, ae);
+        const float se = fs[e];
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+            g[c] *= ae[c];
+            xs[c] = fmaf(se * g[c], ke[c], xs[c]);
+        }
+    }
     float w[RV];
 #pragma unroll
-    for (int e = 0; e < RV; ++e) w[e] = 0.f;
-    auto step = [&](const float (&kk)[CW], const float (&aa)[CW], float bb, const float (&vv)[RV]) {
-        float c = 0.f;
+    for (int r = 0; r < RV; ++r) w[r] = 0.f;
+#pragma unroll 4
+    for (int e = 0; e <= n; ++e) {
+        float ve[RV];
+        if (e < n) load_vec_hint<RV>(log_v + (lrow + e) * DV + r0, ve, keep);
+        else load_vec<RV>(v + head * DV + r0, ve);
+        const float se = fs[e];
 #pragma unroll
-        for (int e = 0; e < CW; ++e) c = fmaf(kk[e], x[e], c);
-        c = group_sum<32>(c);
-        const float s = bb * c;
-#pragma unroll
-        for (int e = 0; e < CW; ++e) x[e] = aa[e] * fmaf(-s, kk[e], x[e]);
-#pragma unroll
-        for (int e = 0; e < RV; ++e) w[e] = fmaf(s, vv[e], w[e]);
-    };
-    step(kc, ac, bc, vc);
-    for (int top = n - 1; top >= 0; top -= CHUNK) {
-        float kk[CHUNK][CW], aa[CHUNK][CW], vv[CHUNK][RV], bb[CHUNK];
-#pragma unroll
-        for (int j = 0; j < CHUNK; ++j) {
-            const int i = top - j;
-            if (i < 0) break;
-            load_vec<CW>(log_k + (lrow + i) * DK + c0, kk[j]);
-            load_vec<RV>(log_v + (lrow + i) * DV + r0, vv[j]);
-            if constexpr (CHAN) {
-                load_vec<CW>(log_a + (lrow + i) * DK + c0, aa[j]);
-            } else {
-                const float as = to_f(log_a[lrow + i]);
-#pragma unroll
-                for (int e = 0; e < CW; ++e) aa[j][e] = as;
-            }
-            bb[j] = to_f(log_b[lrow + i]);
-        }
-#pragma unroll
-        for (int j = 0; j < CHUNK; ++j) {
-            if (top - j < 0) break;
-            step(kk[j], aa[j], bb[j], vv[j]);
-        }
+        for (int r = 0; r < RV; ++r) w[r] = fmaf(se, ve[r], w[r]);
     }
 
-    // (x_0, w) -> workspace.
     float *wk = work + head * (DK + DV);
 #pragma unroll
-    for (int e = 0; e < CW; ++e) wk[c0 + e] = x[e];
+    for (int c = 0; c < CW; ++c) wk[c0 + c] = fmaf(g[c], qv[c], -xs[c]);
 #pragma unroll
-    for (int e = 0; e < RV; ++e) wk[DK + r0 + e] = w[e];
+    for (int r = 0; r < RV; ++r) wk[DK + r0 + r] = w[r];
 }
 
 // ------------------------------------------------------------------ decode
@@ -154,9 +260,10 @@ append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work
     // D3 operands: the base rows first (read only, streamed).
     uint4 raw[C::R];
     if (active) {
+        const uint64_t stream = l2_policy_stream();
         const ST *src = Sbar + (row0 + sub) * DK + col;
 #pragma unroll
-        for (int r = 0; r < C::R; ++r) raw[r] = ld_ro_stream(src + (long long)r * C::RPW * DK);
+        for (int r = 0; r < C::R; ++r) raw[r] = ld_ro_hint(src + (long long)r * C::RPW * DK, stream);
     }
     pdl_wait();  // replay_prep's (x_0, w) are complete and visible from here on
     if (!active) return;
@@ -197,6 +304,26 @@ static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStr
                               units);
 }
 
+template <class IT, int DK, int DV, bool CH, int EMAX>
+static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st) {
+    using P = PrepSmem<IT, DK, EMAX, CH>;
+    constexpr int WARPS = EMAX <= 32 ? 4 : 2;
+    auto kern = replay_prep_kernel<IT, DK, DV, CH, EMAX>;
+    const size_t smem = (size_t)WARPS * P::BYTES;
+    static bool configured = false;
+    if (!configured && smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const long long heads = (long long)p.B * p.H;
+    kern<<<(unsigned)((heads + WARPS - 1) / WARPS), WARPS * 32, smem, st>>>(
+        static_cast<const IT *>(p.q), static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
+        static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
+        static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.c, lg.L, n, work, heads);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st) {
     return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
         using ST = decltype(st_t);
@@ -204,12 +331,10 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
         constexpr int DK = decltype(dk_c)::value;
         constexpr int DV = decltype(dv_c)::value;
         constexpr bool CH = decltype(ch_c)::value;
-        const long long heads = (long long)p.B * p.H;
-        replay_prep_kernel<IT, DK, DV, CH><<<(unsigned)((heads + 7) / 8), 256, 0, st>>>(
-            static_cast<const IT *>(p.q), static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
-            static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
-            static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.L, n, work, heads);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e;
+        if (lg.L <= 16) e = launch_prep<IT, DK, DV, CH, 16>(p, lg, n, work, st);
+        else if (lg.L <= 32) e = launch_prep<IT, DK, DV, CH, 32>(p, lg, n, work, st);
+        else e = launch_prep<IT, DK, DV, CH, 64>(p, lg, n, work, st);
         if (e != cudaSuccess) return e;
         e = launch_decode<ST, DK, DV>(p, work, st);
         if (e != cudaSuccess) return e;

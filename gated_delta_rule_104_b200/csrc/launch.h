@@ -20,6 +20,7 @@ struct StepParams {
 
 struct LogParams {
     void *k, *v, *beta, *a;  // [B, H, L, *]
+    float *c;                // [B, H, L, L] decayed key inner products C(j, e), e < j
     int L;
 };
 

@@ -26,9 +26,10 @@
 //  1. The block issues its base loads first (they land during 2-3).
 //  2. Per entry block, the key side is staged into shared memory: k, a,
 //     beta, the tile's values.
-//  3. C(i, j) by warps (lanes over key channels, shuffle reductions); then,
-//     one thread per key channel, running decay products turn the staged
-//     keys in place into Khat_i = gamma_i o k_i and F_j, plus gamma_n.
+//  3. One thread per key channel forms Khat_i = gamma_i o k_i, F_j and
+//     gamma_n from running decay products. C(i, j) comes from the log
+//     metadata (the append that logged entry i computed it); the fused read's
+//     current entry is the block's last, so its row is just k_n . F_j.
 //  4. Each thread contracts its columns of the row against Khat (the four
 //     lanes of a row read four adjacent chunks: one broadcast wavefront),
 //     the row's partial G are summed over its four lanes, delta is solved
@@ -62,26 +63,28 @@ __device__ __forceinline__ float ld_in(const void *p, long long i, bool bf) {
 
 __host__ __device__ constexpr size_t round4(size_t x) { return (x + 3) & ~(size_t)3; }
 
-// Shared-memory layout for one block of NB entries (all float):
-//   fk [nb][DK]  keys, turned into F in place        (16-byte aligned)
-//   fa           channel decay: [nb][DK], turned into Khat in place;
-//                head decay: nb scalars (padded to 4)
-//   kh [nb][DK]  Khat (head decay only; aliases fa otherwise)
-//   gn [DK], sq [DK]                                 (vector reads)
-//   cm [nb][nb], sb [nb], sv [nb][ROWS]              (scalar reads)
+// Shared-memory layout after the base tile, for one block of NB entries
+// (all float):
+//   fk [nb][DK]  keys                                 (16-byte aligned)
+//   fa           channel decay: [nb][DK]; head decay: nb scalars (padded to 4)
+//   kh [nb][DK]  Khat_i = gamma_i o k_i
+//   ff [nb][DK]  F_j = k_j o D(nb, j)
+//   gn [DK], sq [DK]                                  (vector reads)
+//   cm [nb][nb], sb [nb], sv [nb][ROWS]               (scalar reads)
 template <class ST, int DK, bool CHAN, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
     using C = MergeShape<ST, DK>;
     constexpr int nb = NB, rows = C::ROWS;
-    const size_t floats = (size_t)nb * DK + (CHAN ? (size_t)nb * DK : round4(nb)) + (CHAN ? 0 : (size_t)nb * DK) +
-                          DK + DK + (size_t)nb * nb + nb + (size_t)nb * rows;
+    const size_t floats = (size_t)nb * DK + (CHAN ? (size_t)nb * DK : round4(nb)) + 2 * (size_t)nb * DK + DK +
+                          DK + (size_t)nb * nb + nb + (size_t)nb * rows;
     return (size_t)C::TILE_BYTES + floats * sizeof(float);
 }
 
 template <class ST, int DK, bool CHAN, bool WITH_CUR, int NB>
 __global__ void __launch_bounds__(256, 2)
 merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__restrict__ log_v,
-             const void *__restrict__ log_b, const void *__restrict__ log_a, int L, int n_log,
+             const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_c,
+             int L, int n_log,
              const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
              const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV,
              bool bf) {
@@ -91,10 +94,11 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 
     extern __shared__ float4 smem_raw[];
     unsigned char *tile = reinterpret_cast<unsigned char *>(smem_raw);         // the base tile
-    float *fk = reinterpret_cast<float *>(tile + C::TILE_BYTES);               // k, then F
-    float *fa = fk + (size_t)NB * DK;                 // a (channel: then Khat)
-    float *kh = CHAN ? fa : fa + round4(NB);          // Khat
-    float *gn = kh + (size_t)NB * DK;
+    float *fk = reinterpret_cast<float *>(tile + C::TILE_BYTES);  // keys
+    float *fa = fk + (size_t)NB * DK;                             // decays
+    float *kh = fa + (CHAN ? (size_t)NB * DK : round4(NB));       // Khat
+    float *ff = kh + (size_t)NB * DK;                             // F
+    float *gn = ff + (size_t)NB * DK;
     float *sq = gn + DK;
     float *cm = sq + DK;
     float *sb = cm + (size_t)NB * NB;
@@ -108,8 +112,10 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     ST *grow = S + (head * DV + row0 + rl) * DK;
     const long long lrow = head * L;
 
-    // 1. the base tile -> padded shared rows, asynchronously (no registers held).
-    {
+    // 1. the base tile -> padded shared rows, asynchronously (no registers held);
+    // issued right after the first entry block's key-side loads, so the small
+    // operands are not queued behind the 32-64 KB of state.
+    auto issue_tile = [&]() {
         const unsigned char *gt = reinterpret_cast<const unsigned char *>(S + (head * DV + row0) * DK);
 #pragma unroll
         for (int u = 0; u < C::CPT; ++u) {
@@ -117,7 +123,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             cp_async16(tile + r * C::TSTRIDE + c * 16, gt + (size_t)r * (C::CPR * 16) + c * 16);
         }
         cp_async_commit();
-    }
+    };
     if constexpr (WITH_CUR) {
         if (bf) stage_block(sq, DK, static_cast<const bf16 *>(q) + head * DK, DK, 1, DK, tid, C::THREADS);
         else stage_block(sq, DK, static_cast<const float *>(q) + head * DK, DK, 1, DK, tid, C::THREADS);
@@ -168,6 +174,12 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                     asc = tid < nl ? to_f(static_cast<const IT *>(log_a)[lrow + b0 + tid])
                                    : to_f(static_cast<const IT *>(a)[head]);
             }
+            // C(i, j) for the logged entries of the block (the current entry's row,
+            // if any, is formed below); zero elsewhere.
+            float cval = 0.f;
+            const int ci = tid / NB, cj = tid % NB;
+            if (tid < NB * NB && cj < ci && ci < nl) cval = log_c[(lrow + b0 + ci) * L + b0 + cj];
+            if (b0 == 0) issue_tile();
 #pragma unroll
             for (int u = 0; u < KN; ++u) {
                 const int c = tid + u * C::THREADS, r = c / KC, col = (c % KC) * E;
@@ -191,6 +203,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 sb[tid] = bsc;
                 if constexpr (!CHAN) fa[tid] = asc;
             }
+            if (tid < NB * NB && !(WITH_CUR && nl < nb && ci == nl && cj < nl)) cm[tid] = cval;
         };
         if (bf) stage(bf16{});
         else stage(float{});
@@ -208,33 +221,8 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         for (int i = nb * ROWS + tid; i < NB * ROWS; i += C::THREADS) sv[i] = 0.f;
         __syncthreads();
 
-        // 3a. C(i, j) = sum_c k_i[c] k_j[c] prod_{m=j+1..i} a_m[c], for j < i (within the block):
-        // one warp per j, a running decay product over i, every partial dot kept
-        // in registers and all of them reduced in one transposing butterfly.
-        for (int j = warp; j < NB - 1; j += C::WARPS) {
-            float y[C::CW], p[NB];
-#pragma unroll
-            for (int e = 0; e < C::CW; ++e) y[e] = fk[j * DK + e * 32 + lane];
-#pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                p[i] = 0.f;
-                if (i > j) {
-#pragma unroll
-                    for (int e = 0; e < C::CW; ++e) {
-                        const int c = e * 32 + lane;
-                        y[e] *= CHAN ? fa[i * DK + c] : fa[i];
-                        p[i] = fmaf(fk[i * DK + c], y[e], p[i]);
-                    }
-                }
-            }
-            multi_sum<NB>(p, lane);
-            constexpr int shift = (NB == 4 ? 3 : NB == 8 ? 2 : 1);
-            const int i = lane >> shift;
-            if ((lane & ((1 << shift) - 1)) == 0 && i > j) cm[i * NB + j] = p[0];
-        }
-        __syncthreads();
-
-        // 3b. per key channel: Khat_i = gamma_i o k_i, gamma_nb, F_j = k_j o D(nb, j).
+        // 3. Per key channel: Khat_i = gamma_i o k_i, gamma_nb and F_j = k_j o D(nb, j)
+        // (running decay products; padded entries have a = 1).
         for (int c = tid; c < DK; c += C::THREADS) {
             float ac[NB];
 #pragma unroll
@@ -249,11 +237,28 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             float f = 1.f;
 #pragma unroll
             for (int j = NB - 1; j >= 0; --j) {
-                fk[j * DK + c] *= f;
+                ff[j * DK + c] = fk[j * DK + c] * f;
                 f *= ac[j];
             }
         }
         __syncthreads();
+        // C(i, j) = sum_c k_i[c] k_j[c] prod_{m=j+1..i} a_m[c] for j < i came with the
+        // staging (logged entries carry their rows). The fused read's current
+        // entry is the block's last real entry nl, so D(nl, j) is the suffix
+        // product of F_j and its row is a plain dot: C(nl, j) = k_nl . F_j.
+        const bool cur_here = WITH_CUR && nl < nb;
+        if (cur_here) {
+            for (int j = warp; j < nl; j += C::WARPS) {
+                float pj = 0.f;
+#pragma unroll
+                for (int e = 0; e < C::CW; ++e) {
+                    const int c = e * 32 + lane;
+                    pj = fmaf(fk[nl * DK + c], ff[j * DK + c], pj);
+                }
+                pj = group_sum<32>(pj);
+                if (lane == 0) cm[nl * NB + j] = pj;
+            }
+        }
 
         if (b0 == 0) {  // this thread's chunks of its row: chunk part + 4 m
             cp_async_wait_all();
@@ -271,7 +276,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         // 4. G_i = s . Khat_i over this thread's columns, then over the row's 4 lanes.
         // Entry-outer loops: one uniform bound check per entry, and every shared
         // load a compile-time offset from one per-thread base.
-        const float *khp = kh + part * VEC, *fkp = fk + part * VEC;
+        const float *khp = kh + part * VEC, *fkp = ff + part * VEC;
         float acc[NB];
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
@@ -288,6 +293,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             }
             acc[i] = group_sum<C::TPR>(p0 + p1);
         }
+        if (cur_here) __syncthreads();  // the current entry's C row is complete
         // forward substitution (each of the 4 lanes redundantly): acc <- delta
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
@@ -352,8 +358,8 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
         configured = true;
     }
     const long long blocks = (long long)p.B * p.H * (p.dv / C::ROWS);
-    kern<<<(unsigned)blocks, C::THREADS, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.L,
-                                                    n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
+    kern<<<(unsigned)blocks, C::THREADS, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.c,
+                                                    lg.L, n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
                                                     p.in_dt == DL_BF16);
     return cudaGetLastError();
 }

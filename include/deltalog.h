@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 2
+#define DL_ABI_VERSION 3
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -74,9 +74,9 @@ typedef enum {
 } dl_decay;
 
 /* Caller-owned bounded log of a deferred state: per (b, h) up to L entries of
- * the raw step factors, stored unchanged in `dtype` (lossless), plus a small
- * fp32 workspace the deferred read uses to hand its per-head key-side results
- * to the value tiles.
+ * the raw step factors, stored unchanged in `dtype` (lossless), their
+ * log-decay metadata, and a small fp32 workspace the deferred read uses to
+ * hand its per-head key-side results to the value tiles.
  * (The page's log keeps "compact update factors" plus log-decay metadata,
  * Technical Summary, "Core Mechanism: Base + Log"; here the metadata is
  * recomputed from the stored decays where it is needed.)
@@ -84,6 +84,13 @@ typedef enum {
  *   v     [B, H, L, d_v]
  *   beta  [B, H, L]
  *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL)
+ *   c     [B, H, L, L] float: row j holds C(j, e) = sum_c k_e[c] k_j[c]
+ *         prod_{m=e+1..j} a_m[c] for e < j, the decayed key inner products of
+ *         entry j with the older entries (the page's "log-decay metadata",
+ *         Technical Summary, "Core Mechanism: Base + Log", kept as products
+ *         rather than logarithms). Written by dl_log_append_read for the entry
+ *         it appends and read by the deferred read and the merge, so log
+ *         entries must be written by dl_log_append_read. 16-byte aligned.
  *   work  at least dl_log_work_bytes(B, H, d_k, d_v) bytes, 16-byte aligned,
  *         contents irrelevant between calls (only dl_log_append_read uses it)
  * The number of valid entries n (the same for every head) is tracked by the
@@ -93,6 +100,7 @@ typedef struct {
     void *v;
     void *beta;
     void *a;
+    float *c;
     dl_dtype dtype;
     int L;
     void *work;

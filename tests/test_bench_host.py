@@ -84,7 +84,7 @@ def test_byte_model_matches_the_state_sizes():
     assert bench.entry_bytes(w) == (128 + 128 + 1 + 128) * 2 == 770
     # eager moves the state twice, the deferred read once
     assert bench.alg_bytes(w, "eager", 0) - 2 * w.state_bytes() == w.heads * (770 + 256 + 512)
-    assert bench.alg_bytes(w, "append_read", 3) - w.state_bytes() == w.heads * (5 * 770 + 256 + 512)
+    assert bench.alg_bytes(w, "append_read", 3) - w.state_bytes() == w.heads * (5 * 770 + 256 + 512 + 4 * 3 + 4 * 3)
     w4 = W.WORKLOADS["gdn_b1024_h32_dk128_dv256_t256"]
     assert w4.state_bytes() == 2 << 30 and bench.entry_bytes(w4) == (128 + 256 + 2) * 2
 

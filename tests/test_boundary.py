@@ -81,8 +81,8 @@ def test_scalar_operands_need_only_element_alignment(lib):
 
 
 def make_log(L=8, dtype=b.DL_BF16, base=10):
-    return b.dl_log(addr(base), addr(base + 1), addr(base + 2), addr(base + 3), dtype, L, addr(base + 4),
-                    2 * 3 * (128 + 128) * 4)
+    return b.dl_log(addr(base), addr(base + 1), addr(base + 2), addr(base + 3), addr(base + 5), dtype, L,
+                    addr(base + 4), 2 * 3 * (128 + 128) * 4)
 
 
 def append(lib, fn="dl_log_append_read", log=None, n=0, kind=b.DL_DECAY_CHANNEL, S=None, dk=128, dv=128,
@@ -111,6 +111,10 @@ def test_log_step_argument_checks(lib, fn):
     lo = make_log()
     lo.k = addr(0) + 256                                                 # log inside the base
     assert append(lib, fn, log=lo) == b.DL_ERR_INVALID_ARG
+    lc = make_log()
+    lc.c = None                                                          # metadata missing
+    assert append(lib, fn, log=lc) == b.DL_ERR_INVALID_ARG
+    assert "log.c is a null pointer" in lib.dl_last_error().decode()
 
 
 def test_append_read_workspace_checks(lib):

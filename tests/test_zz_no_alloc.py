@@ -31,7 +31,8 @@ def test_noalloc_refuses_sizes_beyond_its_array():
     fn.restype = ctypes.c_int
     A = 0x7f0000000000
     B, H = 1024, 32  # 32768 heads * 384 floats * 4 bytes = 48 MiB of scratch
-    log = b.dl_log(A + (1 << 40), A + (2 << 40), A + (3 << 40), A + (4 << 40), b.DL_BF16, 8, None, 0)
+    log = b.dl_log(A + (1 << 40), A + (2 << 40), A + (3 << 40), A + (4 << 40), A + (5 << 40), b.DL_BF16, 8,
+                   None, 0)
     big = 1 << 36
     rc = fn(A, b.DL_BF16, b.DL_DECAY_HEAD, ctypes.byref(log), 0, A + big, A + 2 * big, A + 3 * big,
             A + 4 * big, A + 5 * big, b.DL_BF16, A + 6 * big, B, H, 128, 256, None)
