@@ -18,7 +18,7 @@ DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = ra
 DL_F32, DL_BF16 = 0, 1
 DL_DECAY_HEAD, DL_DECAY_CHANNEL = 0, 1
 DL_MAX_LOG = 64
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
            "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_status_string",
@@ -34,7 +34,7 @@ class DeltaLogError(RuntimeError):
 
 class dl_log(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("beta", ctypes.c_void_p),
-                ("a", ctypes.c_void_p), ("c", ctypes.c_void_p), ("dtype", ctypes.c_int), ("L", ctypes.c_int),
+                ("a", ctypes.c_void_p), ("x", ctypes.c_void_p), ("dtype", ctypes.c_int), ("L", ctypes.c_int),
                 ("work", ctypes.c_void_p), ("work_bytes", ctypes.c_size_t)]
 
 
@@ -170,10 +170,10 @@ def _eager(fn, S, q, k, v, beta, a, o, stream, chan):
 class Log:
     """Caller-owned bounded log buffers of a deferred state (device tensors):
     k [B,H,L,d_k], v [B,H,L,d_v], beta [B,H,L], a [B,H,L] or [B,H,L,d_k],
-    c [B,H,L,L] float32 (decayed key inner products), work (fp32 workspace)."""
+    x [B,H,L,L] float32 (the log's triangular solve matrix), work (fp32 workspace)."""
 
-    def __init__(self, k, v, beta, a, c, L: int, channel_decay: bool, work=None):
-        self.k, self.v, self.beta, self.a, self.c = k, v, beta, a, c
+    def __init__(self, k, v, beta, a, x, L: int, channel_decay: bool, work=None):
+        self.k, self.v, self.beta, self.a, self.x = k, v, beta, a, x
         self.L = int(L)
         self.channel_decay = bool(channel_decay)
         self.dtype = _in_dtype(k, v, beta, a)
@@ -185,14 +185,14 @@ class Log:
         z = lambda *s: torch.zeros(*s, dtype=dtype, device=device)  # noqa: E731
         a = z(B, H, L, d_k) if channel_decay else z(B, H, L)
         work = torch.empty(B * H * (d_k + d_v), dtype=torch.float32, device=device)
-        c = torch.zeros(B, H, L, L, dtype=torch.float32, device=device)
-        return cls(z(B, H, L, d_k), z(B, H, L, d_v), z(B, H, L), a, c, L, channel_decay, work)
+        x = torch.zeros(B, H, L, L, dtype=torch.float32, device=device)
+        return cls(z(B, H, L, d_k), z(B, H, L, d_v), z(B, H, L), a, x, L, channel_decay, work)
 
     def struct(self) -> dl_log:
         wp = _ptr(self.work, "log.work") if self.work is not None else None
         wb = self.work.numel() * self.work.element_size() if self.work is not None else 0
         return dl_log(_ptr(self.k, "log.k"), _ptr(self.v, "log.v"), _ptr(self.beta, "log.beta"),
-                      _ptr(self.a, "log.a"), _ptr(self.c, "log.c"), self.dtype, self.L, wp, wb)
+                      _ptr(self.a, "log.a"), _ptr(self.x, "log.x"), self.dtype, self.L, wp, wb)
 
     @property
     def kind(self) -> int:

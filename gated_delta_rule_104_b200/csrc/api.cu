@@ -97,7 +97,7 @@ dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, i
     out[1] = {"log.v", log->v, bhl * dv * is, 16};
     out[2] = {"log.beta", log->beta, bhl * is, is};
     out[3] = chan ? Buf{"log.a", log->a, bhl * dk * is, 16} : Buf{"log.a", log->a, bhl * is, is};
-    out[4] = {"log.c", log->c, bhl * log->L * sizeof(float), 16};
+    out[4] = {"log.x", log->x, bhl * log->L * sizeof(float), 16};
     return DL_OK;
 }
 
@@ -161,7 +161,7 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     const Buf writers[7] = {b[6], b[7], b[8], b[9], b[10], b[11], b[12]};
     if ((s = check_overlap(writers, 7, b, nb)) != DL_OK) return s;
     dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_append_read(p, lg, n, static_cast<float *>(log->work), stream),
                        "append-read launch");
 }
@@ -184,7 +184,7 @@ dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_l
     if ((s = check_overlap(logw, 5, b + 1, 5)) != DL_OK) return s;
     dl::StepParams p{S_base, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, chan,
                      s_dtype, log->dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, false, stream), "merge launch");
 }
 
@@ -206,7 +206,7 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind, const
     const Buf writers[2] = {b[0], b[6]};  // the base and o
     if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
     dl::StepParams p{S_base, q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, true, stream), "merge-read launch");
 }
 
@@ -234,7 +234,7 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
     const Buf writers[6] = {b[6], b[7], b[8], b[9], b[10], b[11]};  // o and the log
     if ((s = check_overlap(writers, 6, b, nb)) != DL_OK) return s;
     dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
-    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->c, log->L};
+    dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_append_read_noalloc(p, lg, n, stream), "no-alloc append-read launch");
 }
 

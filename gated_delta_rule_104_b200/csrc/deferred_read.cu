@@ -16,11 +16,15 @@
 // products) and the decayed key inner products C(j, e) = k_e . (D(j, e) o k_j)
 // for e < j:
 //   d_e = k_e . (D(n, e) o q)                    (independent dots)
-//   s_e = beta_e (d_e - sum_{j>e} C(j, e) s_j)   (a short scalar back-substitution)
+//   s_e = beta_e (d_e - sum_{j>e} C(j, e) s_j), i.e. s = X^T d with
+//   X = (I + Diag(beta) C)^{-1} Diag(beta)       (lower triangular)
 //   x_0 = gamma_n o q - sum_e s_e (gamma_e o k_e),  gamma_e = prod_{m<=e} a_m.
-// The C rows are kept with the log: each append computes C(n, e) for the
-// new entry (the same kind of dots as d_e) and stores it in log.c, so a read
-// never recomputes older rows and the merge reuses them.
+// X only ever gains a row when an entry is appended,
+//   X(n, n) = beta_n,  X(n, j) = -beta_n sum_{m=j..n-1} C(n, m) X(m, j),
+// so it is kept with the log (log.x): each append forms the new entry's C
+// row (the same kind of dots as d_e), extends X by one row and stores it. A
+// read is then two parallel dot passes with no serial solve, and the merge
+// uses the same X.
 //
 // Two kernels, chained with programmatic dependent launch:
 //   replay_prep   one warp per head: stages the head's log keys and decays
@@ -47,7 +51,7 @@ struct PrepSmem {  // one warp's staging area
     static constexpr int K_OFF = 0;
     static constexpr int A_OFF = K_OFF + EMAX * ROWB;           // channel decays (raw)
     static constexpr int F_OFF = A_OFF + (CHAN ? EMAX * ROWB : 0);
-    // floats from F_OFF: as[EMAX], beta[EMAX], d[EMAX], cn[EMAX], sv[EMAX], crow[EMAX][EMAX]
+    // floats from F_OFF: as[EMAX], beta[EMAX], d[EMAX], cn[EMAX], sv[EMAX], xrow[EMAX][EMAX]
     static constexpr int FLOATS = 5 * EMAX + EMAX * EMAX;
     static constexpr int BYTES = F_OFF + FLOATS * 4;
 };
@@ -57,13 +61,12 @@ __global__ void __launch_bounds__(128)
 replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                    const IT *__restrict__ beta, const IT *__restrict__ a, IT *__restrict__ log_k,
                    IT *__restrict__ log_v, IT *__restrict__ log_b, IT *__restrict__ log_a,
-                   float *__restrict__ log_c, int L, int n, float *__restrict__ work, long long heads) {
+                   float *__restrict__ log_x, int L, int n, float *__restrict__ work, long long heads) {
     pdl_launch_dependents();
     using P = PrepSmem<IT, DK, EMAX, CHAN>;
     constexpr int CW = DK / 32;            // key columns per lane (contiguous)
     constexpr int RV = DV / 32;            // value rows per lane
     constexpr int CH = EMAX < 32 ? EMAX : 32;  // entries per butterfly
-    constexpr int SLOTS = (EMAX + 31) / 32;    // entries owned per lane in the back-substitution
     constexpr int E = 16 / (int)sizeof(IT);    // elements per 16-byte chunk
     extern __shared__ float4 smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -71,7 +74,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     IT *sk = reinterpret_cast<IT *>(base + P::K_OFF);
     IT *sa = reinterpret_cast<IT *>(base + P::A_OFF);
     float *fas = reinterpret_cast<float *>(base + P::F_OFF);
-    float *fbeta = fas + EMAX, *fd = fbeta + EMAX, *fcn = fd + EMAX, *fs = fcn + EMAX, *crow = fs + EMAX;
+    float *fbeta = fas + EMAX, *fd = fbeta + EMAX, *fcn = fd + EMAX, *fs = fcn + EMAX, *xrow = fs + EMAX;
 
     const long long head = (long long)blockIdx.x * (blockDim.x / 32) + warp;
     if (head >= heads) return;
@@ -105,13 +108,13 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
             fas[e] = ax[0];
         }
     }
-    // C(j, e) of the logged entries (rows j < n, columns e < j).
+    // X rows of the logged entries (rows j < n, columns e <= j).
     for (int u = lane; u < n * EMAX; u += 32) {
         const int j = u / EMAX, e = u % EMAX;
-        if (e < j) {
-            float cx[1];
-            load_vec_hint<1>(log_c + (lrow + j) * L + e, cx, keep);
-            crow[j * EMAX + e] = cx[0];
+        if (e <= j) {
+            float xx[1];
+            load_vec_hint<1>(log_x + (lrow + j) * L + e, xx, keep);
+            xrow[j * EMAX + e] = xx[0];
         }
     }
     // D1: the entry is appended unchanged (raw input elements).
@@ -172,22 +175,21 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         }
     }
     __syncwarp();
-    for (int e = lane; e < n; e += 32) copy_hint<1>(log_c + (lrow + n) * L + e, fcn + e, keep);
-
-    // s_e = beta_e (d_e - sum_{j>e} C(j, e) s_j), from the newest entry down.
-    float acc[SLOTS];
-#pragma unroll
-    for (int t = 0; t < SLOTS; ++t) acc[t] = 0.f;
-    for (int j = n; j >= 0; --j) {
-        if (lane == (j & 31)) fs[j] = fbeta[j] * (fd[j] - acc[j >> 5]);
-        __syncwarp();
-        const float sj = fs[j];
-        const float *cj = j == n ? fcn : crow + j * EMAX;
-#pragma unroll
-        for (int t = 0; t < SLOTS; ++t) {
-            const int e = lane + 32 * t;
-            if (e < j) acc[t] = fmaf(cj[e], sj, acc[t]);
-        }
+    // X row n: X(n, n) = beta_n, X(n, j) = -beta_n sum_{m=j..n-1} C(n, m) X(m, j).
+    const float bn = fbeta[n];
+    for (int j = lane; j <= n; j += 32) {
+        float acc = 0.f;
+        for (int m = j; m < n; ++m) acc = fmaf(fcn[m], xrow[m * EMAX + j], acc);
+        const float xnj = j == n ? bn : -bn * acc;
+        xrow[n * EMAX + j] = xnj;
+        st_hint(log_x + (lrow + n) * L + j, __float_as_uint(xnj), keep);
+    }
+    __syncwarp();
+    // s_e = sum_{i=e..n} X(i, e) d_i (the back-substitution, as one dot per entry).
+    for (int e = lane; e <= n; e += 32) {
+        float acc = 0.f;
+        for (int i = e; i <= n; ++i) acc = fmaf(xrow[i * EMAX + e], fd[i], acc);
+        fs[e] = acc;
     }
     __syncwarp();
 
@@ -320,7 +322,7 @@ static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, 
     kern<<<(unsigned)((heads + WARPS - 1) / WARPS), WARPS * 32, smem, st>>>(
         static_cast<const IT *>(p.q), static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
         static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
-        static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.c, lg.L, n, work, heads);
+        static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.x, lg.L, n, work, heads);
     return cudaGetLastError();
 }
 

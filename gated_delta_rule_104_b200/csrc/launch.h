@@ -20,7 +20,7 @@ struct StepParams {
 
 struct LogParams {
     void *k, *v, *beta, *a;  // [B, H, L, *]
-    float *c;                // [B, H, L, L] decayed key inner products C(j, e), e < j
+    float *x;                // [B, H, L, L] rows of X = (I + Diag(beta) C)^{-1} Diag(beta), e <= j
     int L;
 };
 

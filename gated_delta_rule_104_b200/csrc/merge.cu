@@ -3,145 +3,191 @@
 // plus replayed log entries -- is materialised back into the base), and the
 // same merge fused with one step's read.
 //
-// Log-decay form. For log entries 1..n (decays a_i, keys k_i, values v_i,
+// Log-decay form. For log entries 0..n-1 (decays a_i, keys k_i, values v_i,
 // strengths beta_i) write D(i, j) = prod_{m=j+1..i} a_m (= exp(Lambda_i -
-// Lambda_j) with the page's log-decay metadata Lambda), gamma_i = D(i, 0).
-// Every row s_bar of the base evolves independently:
-//   s_i = s_bar o gamma_i + sum_{j<=i} delta_j (k_j o D(i, j)),
-//   delta_i = beta_i (v_i[r] - G_i - sum_{j<i} C(i, j) delta_j),
-//   G_i = s_bar . (gamma_i o k_i),   C(i, j) = sum_c k_i[c] D(i, j)[c] k_j[c],
-// and the merged row is s_n = s_bar o gamma_n + sum_j delta_j F_j with
-// F_j = k_j o D(n, j). Per head this is two thin contractions of the base
-// (G = S_bar Khat^T, then delta F) around an n x n triangular solve per row:
-// 4 n d_k d_v FLOP against 2 d_k d_v state elements moved, about 4 FMA per
-// state byte at n = 16 -- close to the B200's CUDA-core/HBM balance.
+// Lambda_j) with the page's log-decay metadata Lambda), gamma = D(n-1, -1).
+// Every row s of the base evolves independently: with
+//   G_i = s . Khat_i,  Khat_i = gamma_i o k_i          (a thin contraction)
+//   C(i, j) = k_j . (D(i, j) o k_i), j < i
+//   delta_i = beta_i (v_i[r] - G_i - sum_{j<i} C(i, j) delta_j)
+// the merged row is s o gamma + sum_j delta_j F_j with F_j = k_j o D(n-1, j).
+// The triangular solve is the same for every row: delta = X (v_r - G) with
+// X = (I + Diag(beta) C)^{-1} Diag(beta), which the log keeps (each append
+// adds its row), so the merge is two thin products
+//   G = S Khat^T                 [rows x d_k] x [d_k x n]
+//   S <- S o gamma + (V - G) W,  W = X^T F     [rows x n] x [n x d_k]
+// with W formed once per head. That is 4 n d_k d_v FLOP against 2 d_k d_v
+// state elements moved: a small dense contraction. For a block of entries
+// [b, b + 16) of a longer log, X's diagonal block is the block's own X.
 //
-// Kernel: one 256-thread block per (head, 64-row value tile); four adjacent
-// lanes share a row, each holding every fourth 16-byte chunk of it in
-// registers, so the base is read and written with coalesced 64-byte runs and
-// never staged in shared memory. The n entries are merged in blocks of at
-// most 16 -- merging n entries is the same as merging the first 16 and then
-// the next 16 into the result -- with the row kept in fp32 registers between
-// blocks and rounded to the state dtype once, at the end.
-//  1. The block issues its base loads first (they land during 2-3).
-//  2. Per entry block, the key side is staged into shared memory: k, a,
-//     beta, the tile's values.
-//  3. One thread per key channel forms Khat_i = gamma_i o k_i, F_j and
-//     gamma_n from running decay products. C(i, j) comes from the log
-//     metadata (the append that logged entry i computed it); the fused read's
-//     current entry is the block's last, so its row is just k_n . F_j.
-//  4. Each thread contracts its columns of the row against Khat (the four
-//     lanes of a row read four adjacent chunks: one broadcast wavefront),
-//     the row's partial G are summed over its four lanes, delta is solved
-//     in registers and the row updated. After the last block the row is
-//     streamed out; the fused read also forms o = s_new . q.
+// Both products run on the tensor cores (mma.sync m16n8k8, TF32 in fp32
+// accumulators). Plain TF32 keeps 10 mantissa bits, too few for the fp32
+// state, so every operand is split as x = hi + lo (two TF32 values) and each
+// product is formed as hi*hi + hi*lo + lo*hi, which recovers ~fp32 accuracy.
+//
+// Kernel: one block per (head, tile of up to 128 rows); warp w owns rows
+// 16w..16w+15 of the tile. The entries are merged in blocks of NB = 8 or 16
+// (a longer log is a chain of sub-merges; short blocks are padded with
+// neutral entries k = 0, a = 1, beta = 0, v = 0). Per block:
+//  1. stage the block's keys, decays, beta, X rows and the tile's values in
+//     shared memory (all global loads issued before any shared store);
+//  2. per key channel, running decay products give Khat, F and gamma; the
+//     fused read's current entry (the block's last) has C(n, j) = k_n . F_j,
+//     from which its X row follows;
+//  3. W = X^T F;
+//  4. per warp: G by tensor-core tiles, E = V - G moved from accumulator to
+//     operand layout with quad shuffles, S o gamma + E W by tensor-core
+//     tiles, the merged rows written back (and o = s_new . q for the fused
+//     read) straight from the accumulator layout.
 #include "launch.h"
 
 namespace dl {
 
-template <class ST, int DK>
-struct MergeShape {
-    static constexpr int VEC = StateVec<ST>::N;              // elements per 16-byte chunk
-    static constexpr int CPR = DK * (int)sizeof(ST) / 16;     // chunks per row
-    static constexpr int TPR = 4;                             // threads per row
-    static constexpr int CPT = CPR / TPR;                     // chunks per thread
-    static constexpr int ROWS = 64;                           // rows per block
-    static constexpr int THREADS = ROWS * TPR;
-    static constexpr int WARPS = THREADS / 32;
-    static constexpr int CW = DK / 32;                        // key channels per lane (C matrix)
-    // base tile rows in shared memory, padded by 64 bytes so that the eight
-    // lanes of a quarter-warp (two rows x four chunks) hit distinct banks
-    static constexpr int TSTRIDE = CPR * 16 + 64;
-    static constexpr int TILE_BYTES = ROWS * TSTRIDE;
-    static_assert(CPT >= 1 && CPT * TPR == CPR, "row split");
-};
+// ------------------------------------------------------------------ tensor-core helpers
 
-// One input element (fp32 or bf16, chosen at run time) widened to float.
-__device__ __forceinline__ float ld_in(const void *p, long long i, bool bf) {
-    return bf ? to_f(static_cast<const bf16 *>(p)[i]) : static_cast<const float *>(p)[i];
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
+// x = hi + lo, both TF32 (x - hi is exact in fp32).
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tf32_of(x);
+    lo = tf32_of(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// d += a b with a = ah + al, b = bh + bl (the al bl term is below fp32 resolution).
+__device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4], float b0,
+                                     float b1) {
+    uint32_t b0h, b0l, b1h, b1l;
+    split_tf32(b0, b0h, b0l);
+    split_tf32(b1, b1h, b1l);
+    mma_tf32(d, al, b0h, b1h);
+    mma_tf32(d, ah, b0l, b1l);
+    mma_tf32(d, ah, b0h, b1h);
+}
+
+__device__ __forceinline__ float ld_state(const float *p) { return *p; }
+__device__ __forceinline__ float ld_state(const bf16 *p) { return to_f(*p); }
+__device__ __forceinline__ void ld_state2(const float *p, float &x, float &y) {
+    const float2 v = *reinterpret_cast<const float2 *>(p);
+    x = v.x;
+    y = v.y;
+}
+__device__ __forceinline__ void ld_state2(const bf16 *p, float &x, float &y) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+    x = bf_lo(w);
+    y = bf_hi(w);
+}
+__device__ __forceinline__ void st_state2(float *p, float x, float y) {
+    __stcs(reinterpret_cast<float2 *>(p), make_float2(x, y));
+}
+__device__ __forceinline__ void st_state2(bf16 *p, float x, float y) {
+    __stcs(reinterpret_cast<unsigned int *>(p), pack_bf2(x, y));
+}
+
+// ------------------------------------------------------------------ layout
 
 __host__ __device__ constexpr size_t round4(size_t x) { return (x + 3) & ~(size_t)3; }
 
-// Shared-memory layout after the base tile, for one block of NB entries
-// (all float):
-//   fk [nb][DK]  keys                                 (16-byte aligned)
-//   fa           channel decay: [nb][DK]; head decay: nb scalars (padded to 4)
-//   kh [nb][DK]  Khat_i = gamma_i o k_i
-//   ff [nb][DK]  F_j = k_j o D(nb, j)
-//   gn [DK], sq [DK]                                  (vector reads)
-//   cm [nb][nb], sb [nb], sv [nb][ROWS]               (scalar reads)
-template <class ST, int DK, bool CHAN, int NB>
-__host__ __device__ constexpr size_t merge_smem_bytes() {
-    using C = MergeShape<ST, DK>;
-    constexpr int nb = NB, rows = C::ROWS;
-    const size_t floats = (size_t)nb * DK + (CHAN ? (size_t)nb * DK : round4(nb)) + 2 * (size_t)nb * DK + DK +
-                          DK + (size_t)nb * nb + nb + (size_t)nb * rows;
-    return (size_t)C::TILE_BYTES + floats * sizeof(float);
+template <int DK>
+struct MergeShape {
+    static constexpr int KH = DK + 4;   // Khat row stride (conflict-free B-fragment reads)
+    static constexpr int WS = DK + 8;   // W row stride (conflict-free B-fragment reads)
+    static constexpr int CW = DK / 32;  // key channels per lane (warp-wide dots)
+    __host__ __device__ static constexpr int rows(int dv) { return 64; }  // 4 warps per block
+};
+
+// Shared memory for one block of NB entries (all float):
+//   fk [NB][DK] keys   fa: channel decay [NB][DK] or head decay [NB] (padded to 4)
+//   ff [NB][DK] F      kh [NB][KH] Khat   sw [NB][WS] W
+//   gn [DK] gamma      sq [DK] q          cm [NB] C row   sx [NB][NB] X   sb [NB] beta
+//   sv [NB][rows] the tile's values
+template <int DK, bool CHAN, int NB>
+__host__ __device__ constexpr size_t merge_smem_bytes(int rows) {
+    using C = MergeShape<DK>;
+    const size_t floats = (size_t)NB * DK + (CHAN ? (size_t)NB * DK : round4(NB)) + (size_t)NB * DK +
+                          (size_t)NB * C::KH + (size_t)NB * C::WS + DK + DK + round4(NB) + (size_t)NB * NB + round4(NB) +
+                          (size_t)NB * rows;
+    return floats * sizeof(float);
 }
+
+// ------------------------------------------------------------------ kernel
 
 template <class ST, int DK, bool CHAN, bool WITH_CUR, int NB>
 __global__ void __launch_bounds__(256, 2)
 merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__restrict__ log_v,
-             const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_c,
-             int L, int n_log,
-             const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
-             const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV,
-             bool bf) {
-    using C = MergeShape<ST, DK>;
-    constexpr int VEC = C::VEC, ROWS = C::ROWS, EPT = C::CPT * VEC;
-    const int NT = n_log + (WITH_CUR ? 1 : 0);  // entries merged
+             const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_x,
+             int L, int n_log, const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
+             const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV, bool bf) {
+    using C = MergeShape<DK>;
+    constexpr int KS = DK / 8;   // k-steps of the first product / column tiles of the second
+    constexpr int NT = NB / 8;   // entry tiles
+    const int ROWS = blockDim.x / 2;  // 16 rows per warp
+    const int nthr = blockDim.x;
+    const int NTOT = n_log + (WITH_CUR ? 1 : 0);
 
     extern __shared__ float4 smem_raw[];
-    unsigned char *tile = reinterpret_cast<unsigned char *>(smem_raw);         // the base tile
-    float *fk = reinterpret_cast<float *>(tile + C::TILE_BYTES);  // keys
-    float *fa = fk + (size_t)NB * DK;                             // decays
-    float *kh = fa + (CHAN ? (size_t)NB * DK : round4(NB));       // Khat
-    float *ff = kh + (size_t)NB * DK;                             // F
-    float *gn = ff + (size_t)NB * DK;
+    float *fk = reinterpret_cast<float *>(smem_raw);
+    float *fa = fk + NB * DK;
+    float *ff = fa + (CHAN ? NB * DK : (int)round4(NB));
+    float *kh = ff + NB * DK;
+    float *sw = kh + NB * C::KH;
+    float *gn = sw + NB * C::WS;
     float *sq = gn + DK;
     float *cm = sq + DK;
-    float *sb = cm + (size_t)NB * NB;
-    float *sv = sb + NB;
+    float *sx = cm + round4(NB);
+    float *sb = sx + NB * NB;
+    float *sv = sb + round4(NB);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;  // fragment coordinates
     const int tiles = DV / ROWS;
     const long long head = blockIdx.x / tiles;
     const int row0 = (blockIdx.x % tiles) * ROWS;
-    const int rl = tid / C::TPR, part = tid % C::TPR;  // row in tile, which quarter of the chunks
-    ST *grow = S + (head * DV + row0 + rl) * DK;
     const long long lrow = head * L;
+    ST *Sw = S + (head * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
 
-    // 1. the base tile -> padded shared rows, asynchronously (no registers held);
-    // issued right after the first entry block's key-side loads, so the small
-    // operands are not queued behind the 32-64 KB of state.
-    auto issue_tile = [&]() {
-        const unsigned char *gt = reinterpret_cast<const unsigned char *>(S + (head * DV + row0) * DK);
+    // First-product operand fragments of the warp's rows, fetched before anything
+    // else (they land while the key side is prepared): a0 = S[g][8s + t],
+    // a1 = S[g + 8][8s + t], a2 = S[g][8s + t + 4], a3 = S[g + 8][8s + t + 4].
+    float afr[KS][4];
+    auto load_afr = [&]() {
 #pragma unroll
-        for (int u = 0; u < C::CPT; ++u) {
-            const int g = tid + u * C::THREADS, r = g / C::CPR, c = g % C::CPR;
-            cp_async16(tile + r * C::TSTRIDE + c * 16, gt + (size_t)r * (C::CPR * 16) + c * 16);
+        for (int s = 0; s < KS; ++s) {
+            afr[s][0] = ld_state(Sw + g * DK + 8 * s + t);
+            afr[s][1] = ld_state(Sw + (g + 8) * DK + 8 * s + t);
+            afr[s][2] = ld_state(Sw + g * DK + 8 * s + t + 4);
+            afr[s][3] = ld_state(Sw + (g + 8) * DK + 8 * s + t + 4);
         }
-        cp_async_commit();
     };
     if constexpr (WITH_CUR) {
-        if (bf) stage_block(sq, DK, static_cast<const bf16 *>(q) + head * DK, DK, 1, DK, tid, C::THREADS);
-        else stage_block(sq, DK, static_cast<const float *>(q) + head * DK, DK, 1, DK, tid, C::THREADS);
+        if (bf) stage_block(sq, DK, static_cast<const bf16 *>(q) + head * DK, DK, 1, DK, tid, nthr);
+        else stage_block(sq, DK, static_cast<const float *>(q) + head * DK, DK, 1, DK, tid, nthr);
     }
 
-    float srow[EPT];  // this thread's columns of the row, fp32, across entry blocks
-    for (int b0 = 0; b0 < NT; b0 += NB) {
-        const int nb = NT - b0 < NB ? NT - b0 : NB;
+    float oacc[2] = {0.f, 0.f};  // o for rows g and g + 8 (fused read), partial over this lane's columns
+    for (int b0 = 0; b0 < NTOT; b0 += NB) {
+        const int nb = NTOT - b0 < NB ? NTOT - b0 : NB;
         const int nl = (n_log - b0 < nb ? n_log - b0 : nb);  // of which from the log (the rest: this step)
+        const bool cur_here = WITH_CUR && nl < nb;
+        const bool last = b0 + NB >= NTOT;
 
-        // 2. entries b0 .. b0+nb-1: log entries, then (fused read) this step's.
-        // Every global load of the block is issued before the first shared store.
+        // 1. entries b0 .. b0+nb-1 (log entries, then the fused read's own); all
+        // global loads are issued before the first shared store.
         auto stage = [&](auto tag) {
             using IT = decltype(tag);
-            constexpr int E = 16 / (int)sizeof(IT);      // elements per 16-byte chunk
-            constexpr int KC = DK / E, VC = ROWS / E;     // chunks per key row / per value slice
-            constexpr int KN = (NB * KC + C::THREADS - 1) / C::THREADS;
-            constexpr int VN = (NB * VC + C::THREADS - 1) / C::THREADS;
+            constexpr int E = 16 / (int)sizeof(IT);
+            constexpr int KC = DK / E;
+            constexpr int KN = (NB * KC + 127) / 128;       // >= 128 threads per block
+            constexpr int VN = (NB * 128 / E + 127) / 128;  // rows <= 128
+            const int VC = ROWS / E;
             float kx[KN][E], ax[KN][E], vx[VN][E];
             (void)ax;
             auto key_src = [&](const void *logp, const void *cur, int r) -> const IT * {
@@ -150,16 +196,16 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             };
 #pragma unroll
             for (int u = 0; u < KN; ++u) {
-                const int c = tid + u * C::THREADS, r = c / KC, col = (c % KC) * E;
-                if (r < nb) {
+                const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
+                if (c < NB * KC && r < nb) {
                     load_vec<E>(key_src(log_k, k, r) + col, kx[u]);
                     if constexpr (CHAN) load_vec<E>(key_src(log_a, a, r) + col, ax[u]);
                 }
             }
 #pragma unroll
             for (int u = 0; u < VN; ++u) {
-                const int c = tid + u * C::THREADS, r = c / VC, col = (c % VC) * E;
-                if (r < nb) {
+                const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
+                if (c < NB * VC && r < nb) {
                     const IT *src = r < nl ? static_cast<const IT *>(log_v) + (lrow + b0 + r) * DV
                                            : static_cast<const IT *>(v) + head * DV;
                     load_vec<E>(src + row0 + col, vx[u]);
@@ -174,66 +220,61 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                     asc = tid < nl ? to_f(static_cast<const IT *>(log_a)[lrow + b0 + tid])
                                    : to_f(static_cast<const IT *>(a)[head]);
             }
-            // C(i, j) for the logged entries of the block (the current entry's row,
-            // if any, is formed below); zero elsewhere.
-            float cval = 0.f;
-            const int ci = tid / NB, cj = tid % NB;
-            if (tid < NB * NB && cj < ci && ci < nl) cval = log_c[(lrow + b0 + ci) * L + b0 + cj];
-            if (b0 == 0) issue_tile();
+            // X(i, j), j <= i, of the logged entries (the block's diagonal block; the
+            // current entry's row is formed below; padded entries are zero)
+            constexpr int CN = (NB * NB + 127) / 128;
+            float cval[CN];
+#pragma unroll
+            for (int u = 0; u < CN; ++u) {
+                const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
+                cval[u] = (idx < NB * NB && cj <= ci && ci < nl) ? log_x[(lrow + b0 + ci) * L + b0 + cj] : 0.f;
+            }
 #pragma unroll
             for (int u = 0; u < KN; ++u) {
-                const int c = tid + u * C::THREADS, r = c / KC, col = (c % KC) * E;
-                if (r < nb) {
+                const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
+                if (c < NB * KC) {
+                    const bool real = r < nb;  // padded entries: k = 0, a = 1
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
-                        fk[r * DK + col + e] = kx[u][e];
-                        if constexpr (CHAN) fa[r * DK + col + e] = ax[u][e];
+                        fk[r * DK + col + e] = real ? kx[u][e] : 0.f;
+                        if constexpr (CHAN) fa[r * DK + col + e] = real ? ax[u][e] : 1.f;
                     }
                 }
             }
 #pragma unroll
             for (int u = 0; u < VN; ++u) {
-                const int c = tid + u * C::THREADS, r = c / VC, col = (c % VC) * E;
-                if (r < nb) {
+                const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
+                if (c < NB * VC) {
 #pragma unroll
-                    for (int e = 0; e < E; ++e) sv[r * ROWS + col + e] = vx[u][e];
+                    for (int e = 0; e < E; ++e) sv[r * ROWS + col + e] = r < nb ? vx[u][e] : 0.f;
                 }
             }
-            if (tid < nb) {
-                sb[tid] = bsc;
+            if (tid < NB) {
+                sb[tid] = bsc;  // 0 for padded entries
                 if constexpr (!CHAN) fa[tid] = asc;
             }
-            if (tid < NB * NB && !(WITH_CUR && nl < nb && ci == nl && cj < nl)) cm[tid] = cval;
+#pragma unroll
+            for (int u = 0; u < CN; ++u) {
+                const int idx = tid + u * nthr, ci = idx / NB;
+                if (idx < NB * NB && !(cur_here && ci == nl)) sx[idx] = cval[u];
+            }
         };
         if (bf) stage(bf16{});
         else stage(float{});
-        // Entries nb..NB-1 of a short block are neutral: k = 0, a = 1, beta = 0,
-        // v = 0 leave gamma, F and every delta unchanged, so all loops below run
-        // over the full compile-time NB without bound checks.
-        for (int i = nb * DK + tid; i < NB * DK; i += C::THREADS) {
-            fk[i] = 0.f;
-            if constexpr (CHAN) fa[i] = 1.f;
-        }
-        for (int i = nb + tid; i < NB; i += C::THREADS) {
-            if constexpr (!CHAN) fa[i] = 1.f;
-            sb[i] = 0.f;
-        }
-        for (int i = nb * ROWS + tid; i < NB * ROWS; i += C::THREADS) sv[i] = 0.f;
         __syncthreads();
 
-        // 3. Per key channel: Khat_i = gamma_i o k_i, gamma_nb and F_j = k_j o D(nb, j)
-        // (running decay products; padded entries have a = 1).
-        for (int c = tid; c < DK; c += C::THREADS) {
+        // 2. per key channel: Khat_i = gamma_i o k_i, gamma, F_j = k_j o D(nb-1, j).
+        for (int c = tid; c < DK; c += nthr) {
             float ac[NB];
 #pragma unroll
             for (int i = 0; i < NB; ++i) ac[i] = CHAN ? fa[i * DK + c] : fa[i];
-            float g = 1.f;
+            float gm = 1.f;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
-                g *= ac[i];
-                kh[i * DK + c] = g * fk[i * DK + c];
+                gm *= ac[i];
+                kh[i * C::KH + c] = gm * fk[i * DK + c];
             }
-            gn[c] = g;
+            gn[c] = gm;
             float f = 1.f;
 #pragma unroll
             for (int j = NB - 1; j >= 0; --j) {
@@ -242,13 +283,10 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             }
         }
         __syncthreads();
-        // C(i, j) = sum_c k_i[c] k_j[c] prod_{m=j+1..i} a_m[c] for j < i came with the
-        // staging (logged entries carry their rows). The fused read's current
-        // entry is the block's last real entry nl, so D(nl, j) is the suffix
-        // product of F_j and its row is a plain dot: C(nl, j) = k_nl . F_j.
-        const bool cur_here = WITH_CUR && nl < nb;
+        // The fused read's current entry is the block's last real one, so
+        // D(nl, j) is F_j's suffix product: C(nl, j) = k_nl . F_j.
         if (cur_here) {
-            for (int j = warp; j < nl; j += C::WARPS) {
+            for (int j = warp; j < nl; j += nthr / 32) {
                 float pj = 0.f;
 #pragma unroll
                 for (int e = 0; e < C::CW; ++e) {
@@ -256,120 +294,139 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                     pj = fmaf(fk[nl * DK + c], ff[j * DK + c], pj);
                 }
                 pj = group_sum<32>(pj);
-                if (lane == 0) cm[nl * NB + j] = pj;
+                if (lane == 0) cm[j] = pj;
             }
-        }
-
-        if (b0 == 0) {  // this thread's chunks of its row: chunk part + 4 m
-            cp_async_wait_all();
             __syncthreads();
-#pragma unroll
-            for (int m = 0; m < C::CPT; ++m) {
-                float x[VEC];
-                StateVec<ST>::unpack(
-                    *reinterpret_cast<const uint4 *>(tile + rl * C::TSTRIDE + (part + C::TPR * m) * 16), x);
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) srow[m * VEC + e] = x[e];
+            // its X row: X(nl, nl) = beta, X(nl, j) = -beta sum_{m=j..nl-1} C(nl, m) X(m, j)
+            if (tid < NB) {
+                const int j = tid;
+                float acc = 0.f;
+                for (int m = j; m < nl; ++m) acc = fmaf(cm[m], sx[m * NB + j], acc);
+                sx[nl * NB + j] = j < nl ? -sb[nl] * acc : (j == nl ? sb[nl] : 0.f);
             }
+            __syncthreads();
         }
 
-        // 4. G_i = s . Khat_i over this thread's columns, then over the row's 4 lanes.
-        // Entry-outer loops: one uniform bound check per entry, and every shared
-        // load a compile-time offset from one per-thread base.
-        const float *khp = kh + part * VEC, *fkp = ff + part * VEC;
-        float acc[NB];
+        // 3. W = X^T F: W[j][c] = sum_{i>=j} X(i, j) F[i][c].
+        for (int u = tid; u < NB * DK; u += nthr) {
+            const int j = u / DK, c = u % DK;
+            float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < NB; ++i) {
-            float p0 = 0.f, p1 = 0.f;  // two partial chains per entry
+            for (int i = 0; i < NB; ++i) acc = fmaf(sx[i * NB + j], ff[i * DK + c], acc);
+            sw[j * C::WS + c] = acc;
+        }
+        __syncthreads();
+
+        // 4. this warp's 16 rows. G = S Khat^T.
+        __syncwarp();  // a previous block's rows, written by this warp, are visible
+        load_afr();
+        float acc1[NT][4];
 #pragma unroll
-            for (int m = 0; m < C::CPT; ++m) {
-                float kv[VEC];
-                load_vec<VEC>(khp + i * DK + m * C::TPR * VEC, kv);
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    if ((m + e) & 1) p1 = fmaf(srow[m * VEC + e], kv[e], p1);
-                    else p0 = fmaf(srow[m * VEC + e], kv[e], p0);
-                }
+            for (int x = 0; x < 4; ++x) acc1[nt][x] = 0.f;
+#pragma unroll
+        for (int s = 0; s < KS; ++s) {
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) split_tf32(afr[s][x], ah[x], al[x]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float *kp = kh + (8 * nt + g) * C::KH + 8 * s + t;
+                mma3(acc1[nt], ah, al, kp[0], kp[4]);
             }
-            acc[i] = group_sum<C::TPR>(p0 + p1);
         }
-        if (cur_here) __syncthreads();  // the current entry's C row is complete
-        // forward substitution (each of the 4 lanes redundantly): acc <- delta
+        // E = V - G (accumulator layout: rows g, g + 8; entries 8nt + 2t, 8nt + 2t + 1),
+        // then moved to operand layout (entries 8nt + t, 8nt + t + 4) within each quad.
+        const int rg = 16 * warp + g;
+        uint32_t eh[NT][4], el[NT][4];
 #pragma unroll
-        for (int i = 0; i < NB; ++i) {
-            float t = sv[i * ROWS + rl] - acc[i];
-#pragma unroll
-            for (int j = 0; j < i; ++j) t = fmaf(-cm[i * NB + j], acc[j], t);
-            acc[i] = sb[i] * t;
+        for (int nt = 0; nt < NT; ++nt) {
+            const int i0 = 8 * nt + 2 * t;
+            const float e0 = sv[i0 * ROWS + rg] - acc1[nt][0];
+            const float e1 = sv[(i0 + 1) * ROWS + rg] - acc1[nt][1];
+            const float e2 = sv[i0 * ROWS + rg + 8] - acc1[nt][2];
+            const float e3 = sv[(i0 + 1) * ROWS + rg + 8] - acc1[nt][3];
+            const int s0 = (lane & ~3) | (t >> 1), s1 = s0 + 2;  // quad lanes holding entries t, t + 4
+            const float x00 = __shfl_sync(0xffffffffu, e0, s0), x01 = __shfl_sync(0xffffffffu, e1, s0);
+            const float x10 = __shfl_sync(0xffffffffu, e2, s0), x11 = __shfl_sync(0xffffffffu, e3, s0);
+            const float y00 = __shfl_sync(0xffffffffu, e0, s1), y01 = __shfl_sync(0xffffffffu, e1, s1);
+            const float y10 = __shfl_sync(0xffffffffu, e2, s1), y11 = __shfl_sync(0xffffffffu, e3, s1);
+            const bool odd = t & 1;
+            split_tf32(odd ? x01 : x00, eh[nt][0], el[nt][0]);  // E[g][8nt + t]
+            split_tf32(odd ? x11 : x10, eh[nt][1], el[nt][1]);  // E[g + 8][8nt + t]
+            split_tf32(odd ? y01 : y00, eh[nt][2], el[nt][2]);  // E[g][8nt + t + 4]
+            split_tf32(odd ? y11 : y10, eh[nt][3], el[nt][3]);  // E[g + 8][8nt + t + 4]
         }
-        // s <- s o gamma_nb + sum_j delta_j F_j
+        // S <- S o gamma + E W, one 16 x 8 column tile at a time, written straight
+        // from the accumulator layout (rows g, g + 8; columns 8c + 2t, 8c + 2t + 1).
+#pragma unroll 4
+        for (int cb = 0; cb < KS; ++cb) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int m = 0; m < C::CPT; ++m) {
-            float gv[VEC];
-            load_vec<VEC>(gn + part * VEC + m * C::TPR * VEC, gv);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) srow[m * VEC + e] *= gv[e];
-        }
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-            const float dj = acc[j];
-#pragma unroll
-            for (int m = 0; m < C::CPT; ++m) {
-                float fv[VEC];
-                load_vec<VEC>(fkp + j * DK + m * C::TPR * VEC, fv);
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) srow[m * VEC + e] = fmaf(dj, fv[e], srow[m * VEC + e]);
+            for (int nt = 0; nt < NT; ++nt) {
+                const float *wp = sw + (8 * nt + t) * C::WS + 8 * cb + g;
+                mma3(d, eh[nt], el[nt], wp[0], wp[4 * C::WS]);
             }
+            const int col = 8 * cb + 2 * t;
+            float s00, s01, s10, s11;
+            ld_state2(Sw + g * DK + col, s00, s01);
+            ld_state2(Sw + (g + 8) * DK + col, s10, s11);
+            const float2 gv = *reinterpret_cast<const float2 *>(gn + col);
+            s00 = fmaf(s00, gv.x, d[0]);
+            s01 = fmaf(s01, gv.y, d[1]);
+            s10 = fmaf(s10, gv.x, d[2]);
+            s11 = fmaf(s11, gv.y, d[3]);
+            if (WITH_CUR && last) {
+                const float2 qv = *reinterpret_cast<const float2 *>(sq + col);
+                oacc[0] = fmaf(s00, qv.x, fmaf(s01, qv.y, oacc[0]));
+                oacc[1] = fmaf(s10, qv.x, fmaf(s11, qv.y, oacc[1]));
+            }
+            st_state2(Sw + g * DK + col, s00, s01);
+            st_state2(Sw + (g + 8) * DK + col, s10, s11);
         }
         __syncthreads();  // the next entry block reuses the shared buffers
     }
 
-    // 5. the merged row, streamed back (rounded once for a bf16 state); o = s_new . q (fused read).
-    float oacc = 0.f;
-#pragma unroll
-    for (int m = 0; m < C::CPT; ++m) {
-        const int c0 = (part + C::TPR * m) * VEC;
-        float x[VEC];
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) x[e] = srow[m * VEC + e];
-        if constexpr (WITH_CUR) {
-            float qv[VEC];
-            load_vec<VEC>(sq + c0, qv);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) oacc = fmaf(x[e], qv[e], oacc);
-        }
-        st_stream(grow + c0, StateVec<ST>::pack(x));
-    }
     if constexpr (WITH_CUR) {
-        oacc = group_sum<C::TPR>(oacc);
-        if (part == 0) o[head * DV + row0 + rl] = oacc;
+        oacc[0] = group_sum<4>(oacc[0]);
+        oacc[1] = group_sum<4>(oacc[1]);
+        if (t == 0) {
+            o[head * DV + row0 + 16 * warp + g] = oacc[0];
+            o[head * DV + row0 + 16 * warp + g + 8] = oacc[1];
+        }
     }
 }
+
+// ------------------------------------------------------------------ launch
 
 template <class ST, int DK, bool CHAN, bool WC, int NB>
 static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
-    using C = MergeShape<ST, DK>;
+    using C = MergeShape<DK>;
     auto kern = merge_kernel<ST, DK, CHAN, WC, NB>;
-    const size_t smem = merge_smem_bytes<ST, DK, CHAN, NB>();
+    const int rows = C::rows(p.dv);
+    const size_t smem = merge_smem_bytes<DK, CHAN, NB>(rows);
     static bool configured = false;
-    if (!configured && smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
+    if (!configured) {
+        const size_t want = merge_smem_bytes<DK, CHAN, NB>(rows);
+        if (want > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
+            if (e != cudaSuccess) return e;
+        }
         configured = true;
     }
-    const long long blocks = (long long)p.B * p.H * (p.dv / C::ROWS);
-    kern<<<(unsigned)blocks, C::THREADS, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.c,
-                                                    lg.L, n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
-                                                    p.in_dt == DL_BF16);
+    const long long blocks = (long long)p.B * p.H * (p.dv / rows);
+    kern<<<(unsigned)blocks, rows * 2, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.x, lg.L,
+                                                   n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
+                                                   p.in_dt == DL_BF16);
     return cudaGetLastError();
 }
 
-// Entry-block size: the smallest of 4, 8, 16 that holds all entries (16 for
-// longer logs, whose last block is padded).
+// Entry-block size: 8 when all entries fit, else 16 (a longer log runs as a
+// chain of 16-entry sub-merges, the last one padded).
 template <class ST, int DK, bool CHAN, bool WC>
 static cudaError_t launch_merge_nb(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
     const int nt = n_log + (WC ? 1 : 0);
-    if (nt <= 4) return launch_merge_t<ST, DK, CHAN, WC, 4>(p, lg, n_log, st);
     if (nt <= 8) return launch_merge_t<ST, DK, CHAN, WC, 8>(p, lg, n_log, st);
     return launch_merge_t<ST, DK, CHAN, WC, 16>(p, lg, n_log, st);
 }

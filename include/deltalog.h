@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 3
+#define DL_ABI_VERSION 4
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -84,13 +84,15 @@ typedef enum {
  *   v     [B, H, L, d_v]
  *   beta  [B, H, L]
  *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL)
- *   c     [B, H, L, L] float: row j holds C(j, e) = sum_c k_e[c] k_j[c]
- *         prod_{m=e+1..j} a_m[c] for e < j, the decayed key inner products of
- *         entry j with the older entries (the page's "log-decay metadata",
+ *   x     [B, H, L, L] float: the log's metadata, row j holding X(j, e) for
+ *         e <= j, where X = (I + Diag(beta) C)^{-1} Diag(beta) and
+ *         C(j, e) = sum_c k_e[c] k_j[c] prod_{m=e+1..j} a_m[c] for e < j (the
+ *         decayed key inner products: the page's "log-decay metadata",
  *         Technical Summary, "Core Mechanism: Base + Log", kept as products
- *         rather than logarithms). Written by dl_log_append_read for the entry
- *         it appends and read by the deferred read and the merge, so log
- *         entries must be written by dl_log_append_read. 16-byte aligned.
+ *         rather than logarithms). X is lower triangular and gains one row per
+ *         append, so dl_log_append_read writes row n for the entry it appends;
+ *         the deferred read and the merge read it. Log entries must therefore
+ *         be written by dl_log_append_read. 16-byte aligned.
  *   work  at least dl_log_work_bytes(B, H, d_k, d_v) bytes, 16-byte aligned,
  *         contents irrelevant between calls (only dl_log_append_read uses it)
  * The number of valid entries n (the same for every head) is tracked by the
@@ -100,7 +102,7 @@ typedef struct {
     void *v;
     void *beta;
     void *a;
-    float *c;
+    float *x;
     dl_dtype dtype;
     int L;
     void *work;

@@ -112,9 +112,9 @@ def test_log_step_argument_checks(lib, fn):
     lo.k = addr(0) + 256                                                 # log inside the base
     assert append(lib, fn, log=lo) == b.DL_ERR_INVALID_ARG
     lc = make_log()
-    lc.c = None                                                          # metadata missing
+    lc.x = None                                                          # metadata missing
     assert append(lib, fn, log=lc) == b.DL_ERR_INVALID_ARG
-    assert "log.c is a null pointer" in lib.dl_last_error().decode()
+    assert "log.x is a null pointer" in lib.dl_last_error().decode()
 
 
 def test_append_read_workspace_checks(lib):
