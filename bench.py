@@ -50,9 +50,10 @@ KERNEL_SOURCES = ["gated_delta_rule_104_b200/csrc/deferred_read.cu", "gated_delt
 # ---------------------------------------------------------------- byte model
 
 def entry_bytes(w: W.Workload) -> int:
-    """Bytes of one log entry / one step's (k, v, beta, a)."""
+    """Bytes of one log entry / one step's (k, v, beta, a); RWKV6 has no beta."""
     s_in = 2 if w.in_dtype == "bf16" else 4
-    return (w.d_k + w.d_v + 1 + (w.d_k if w.decay == W.CHANNEL else 1)) * s_in
+    beta = 0 if w.decay == W.RWKV6 else 1
+    return (w.d_k + w.d_v + beta + (1 if w.decay == W.HEAD else w.d_k)) * s_in
 
 
 def state_bytes_head(w: W.Workload) -> int:
@@ -66,22 +67,37 @@ def alg_bytes(w: W.Workload, kind: str, n: int) -> int:
     append_read:  state read (no write), n log entries read, one entry
                   written, this step's inputs, o, and the log metadata: the
                   older entries' C rows read (n(n-1)/2 floats), the new row
-                  written (n floats)
+                  written (n floats); RWKV6 keeps no such rows
     merge_read:   state read + write, n log entries and their C rows, this
                   step's inputs, o
     merge:        state read + write, n log entries and their C rows
+    pool:         one slot-pool step of the whole batch with staggered fills
+                  (sequence b holds (b + step) mod L entries, n = L): the
+                  rows at L - 1 merge (merge_read), the others append_read
     """
+    if kind == "pool":
+        L = n
+        tot = 0
+        for c in range(L):
+            nseq = len(range(c, w.B, L))
+            sub = "merge_read" if c == L - 1 else "append_read"
+            tot += nseq * alg_bytes(w, sub, c) // w.B
+        return tot
     e, S = entry_bytes(w), state_bytes_head(w)
     s_in = 2 if w.in_dtype == "bf16" else 4
     q, o = w.d_k * s_in, 4 * w.d_v
-    crows = 4 * n * (n - 1) // 2
+    delta = w.decay != W.RWKV6
+    crows = 4 * n * (n - 1) // 2 if delta else 0
     per_head = {
         "eager": 2 * S + e + q + o,
-        "append_read": S + n * e + e + e + q + o + crows + 4 * n,
+        "append_read": S + n * e + e + e + q + o + crows + (4 * n if delta else 0),
         "merge_read": 2 * S + n * e + e + q + o + crows,
         "merge": 2 * S + n * e + crows,
     }[kind]
     return per_head * w.heads
+
+
+KERNELS_PER_CALL = {"eager": 1, "append_read": 2, "merge_read": 1, "merge": 1, "pool": 4}
 
 
 # ---------------------------------------------------------------- helpers
@@ -245,11 +261,14 @@ def run_reference(args, w, L):
 
 
 def config_block(w, L, args):
-    return {"workload": w.name, "decay": "channel (KDA)" if w.decay == W.CHANNEL else "head (GDN)",
+    decay = {W.CHANNEL: "channel (KDA)", W.HEAD: "head (GDN)",
+             W.RWKV6: "channel, raw-value update without delta correction (RWKV6)"}[w.decay]
+    return {"workload": w.name, "decay": decay,
             "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "T": w.T, "L": L,
             "state_dtype": w.state_dtype, "in_dtype": w.in_dtype,
-            "schedule": "DeltaLog deferred, merge fused into the L-th step" if args.schedule == "fused"
-            else "DeltaLog deferred, separate merge every L steps",
+            "schedule": {"fused": "DeltaLog deferred, merge fused into the L-th step",
+                         "unfused": "DeltaLog deferred, separate merge every L steps",
+                         "pool": "slot pool, staggered log fills (each step 1/L of the rows merge)"}[args.schedule],
             "global_batch": w.B * max(1, dist_env()[2]), "seq_len": w.T,
             "l2": "inputs larger than L2 (state %d MiB per GPU), no flush" % (w.state_bytes() >> 20)}
 
@@ -260,15 +279,18 @@ class Launcher:
     """Issues the T steps of one decode and (optionally) brackets every launch
     with CUDA events on the launching stream."""
 
-    def __init__(self, g, w, d, S, log, o_all, schedule, stream):
+    def __init__(self, g, w, d, S, log, o_all, schedule, stream, pool=None):
         self.g, self.w, self.d, self.S, self.log, self.o_all = g, w, d, S, log, o_all
-        self.schedule, self.stream = schedule, stream
-        self.chan = w.decay == W.CHANNEL
+        self.schedule, self.stream, self.pool = schedule, stream, pool
+        self.chan = w.decay != W.HEAD
+        self.rwkv6 = w.decay == W.RWKV6
         self.L = log.L if log is not None else 0
 
     def plan(self):
         """(kind, n) of each launch of one decode, in order."""
         out, n = [], 0
+        if self.schedule == "pool":
+            return [("pool", self.L)] * self.w.T
         for _ in range(self.w.T):
             if self.schedule == "eager":
                 out.append(("eager", 0))
@@ -285,21 +307,53 @@ class Launcher:
             out.append(("merge", n))  # flush so that S holds the final state
         return out
 
+    def pool_join(self):
+        """Untimed: sequence b joins at step (L-1) - (b mod L), so after L-1
+        steps it holds b mod L entries and the fills are staggered."""
+        import torch
+
+        g, d, L = self.g, self.d, self.L
+        B = self.w.B
+        for j in range(L - 1):
+            rows = [b for b in range(B) if j >= (L - 1) - (b % L)]
+            if not rows:
+                continue
+            idx = torch.tensor(rows, dtype=torch.long, device="cuda")
+            slot = idx.to(torch.int32)
+            pick = lambda key: d[key][j].index_select(0, idx).contiguous()  # noqa: E731
+            beta = None if self.rwkv6 else pick("beta")
+            o = torch.empty(len(rows), self.w.H, self.w.d_v, device="cuda")
+            g.dl_pool_step(self.pool, slot, pick("q"), pick("k"), pick("v"), beta, pick("a"), o, self.stream)
+
     def run(self, events=None):
         g, d, S, o, st = self.g, self.d, self.S, self.o_all, self.stream
+        if self.schedule == "pool":
+            slots = self.pool_slots
+            for t in range(self.w.T):
+                if events is not None:
+                    events.append(self._ev())
+                beta = None if self.rwkv6 else d["beta"][t]
+                g.dl_pool_step(self.pool, slots, d["q"][t], d["k"][t], d["v"][t], beta, d["a"][t], o[t], st)
+            if events is not None:
+                events.append(self._ev())
+            return
         t = 0
         for kind, n in self.plan():
             if events is not None:
                 events.append(self._ev())
+            beta = None if self.rwkv6 else d["beta"][t]
             if kind == "eager":
-                fn = g.dl_kda_decode_step if self.chan else g.dl_gdn_decode_step
-                fn(S, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                if self.rwkv6:
+                    g.dl_rwkv6_decode_step(S, d["q"][t], d["k"][t], d["v"][t], d["a"][t], o[t], st)
+                else:
+                    fn = g.dl_kda_decode_step if self.chan else g.dl_gdn_decode_step
+                    fn(S, d["q"][t], d["k"][t], d["v"][t], beta, d["a"][t], o[t], st)
                 t += 1
             elif kind == "append_read":
-                g.dl_log_append_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                g.dl_log_append_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], beta, d["a"][t], o[t], st)
                 t += 1
             elif kind == "merge_read":
-                g.dl_log_merge_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o[t], st)
+                g.dl_log_merge_read(S, self.log, n, d["q"][t], d["k"][t], d["v"][t], beta, d["a"][t], o[t], st)
                 t += 1
             else:
                 g.dl_log_merge(S, self.log, n, st)
@@ -340,7 +394,7 @@ def timed(launcher, steps, warmup):
         for i, (kind, n) in enumerate(plan):
             per_kind.setdefault(kind, []).append((n, ev[i].elapsed_time(ev[i + 1])))
     ms = reduce_max(total_ms / steps)
-    return ms, per_kind, steps * len(plan)
+    return ms, per_kind, steps * sum(KERNELS_PER_CALL[kind] for kind, _ in plan)
 
 
 def roofline_for(w, per_kind, kind, peak, peak_note, traffic):
@@ -364,12 +418,13 @@ def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
     import torch
 
     dev = torch.device("cuda")
-    chan = w.decay == W.CHANNEL
+    chan = w.decay != W.HEAD
+    rw = w.decay == W.RWKV6
     tdt = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
     B, H = w.B, w.H
     S = torch.empty(B, H, w.d_v, w.d_k, dtype=host["S0"].dtype, device=dev)
-    log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=dev)
-    names = ("q", "k", "v", "beta", "a")
+    log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=dev, rwkv6=rw)
+    names = ("q", "k", "v", "a") if rw else ("q", "k", "v", "beta", "a")
     nslot = 3
     slots = [{n: torch.empty_like(host[n][0], device=dev) for n in names} for _ in range(nslot)]
     o_dev = [torch.empty(B, H, w.d_v, dtype=torch.float32, device=dev) for _ in range(nslot)]
@@ -402,7 +457,7 @@ def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
             if ev_out[j] is not None:
                 stream.wait_event(ev_out[j])  # o slot drained
             sl = slots[j]
-            dec.step(sl["q"], sl["k"], sl["v"], sl["beta"], sl["a"], o_dev[j], stream)
+            dec.step(sl["q"], sl["k"], sl["v"], sl.get("beta"), sl["a"], o_dev[j], stream)
             ev_used[j] = torch.cuda.Event()
             ev_used[j].record(stream)
             with torch.cuda.stream(d2h):
@@ -452,7 +507,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--L", type=int, default=0, help="log capacity (default: the workload's)")
-    ap.add_argument("--schedule", choices=["fused", "unfused"], default="fused")
+    ap.add_argument("--schedule", choices=["fused", "unfused", "pool"], default="fused",
+                    help="pool: the slot-pool step over the whole batch at staggered log fills")
     ap.add_argument("--workers", type=int, default=0, help="input-generation processes (0: auto)")
     ap.add_argument("--cpu-seconds-per-step", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -496,17 +552,27 @@ def main(argv=None):
     g.load()
     d = W.device_inputs(w, x)
     stream = torch.cuda.current_stream()
-    chan = w.decay == W.CHANNEL
+    chan = w.decay != W.HEAD
     tdt = d["q"].dtype
     o_all = torch.empty(w.T, w.B, w.H, w.d_v, dtype=torch.float32, device="cuda")
     peak, peak_note = measured_peaks()
-    traffic = profiled_traffic()
+    # the committed DRAM-traffic figure is for the KDA workload's append_read at L = 16
+    traffic = profiled_traffic() if (w.name == DEFAULT_WORKLOAD and L == 16) else None
 
     sampler = ClockSampler(local_rank)
     with sampler:
-        S_def = d["S0"].clone()
-        log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, tdt, chan)
-        lau = Launcher(g, w, d, S_def, log, o_all, args.schedule, stream)
+        rw = w.decay == W.RWKV6
+        if args.schedule == "pool":
+            pool = g.Pool.allocate(w.B, w.H, w.d_k, w.d_v, L, d["S0"].dtype, tdt, chan, rwkv6=rw)
+            pool.S.copy_(d["S0"])
+            S_def, log = pool.S, pool.log
+            lau = Launcher(g, w, d, S_def, log, o_all, "pool", stream, pool=pool)
+            lau.pool_slots = torch.arange(w.B, dtype=torch.int32, device="cuda")
+            lau.pool_join()
+        else:
+            S_def = d["S0"].clone()
+            log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, tdt, chan, rwkv6=rw)
+            lau = Launcher(g, w, d, S_def, log, o_all, args.schedule, stream)
         ms_def, kinds_def, launches = timed(lau, args.steps, args.warmup)
         eager = None
         if not args.no_eager:
@@ -520,14 +586,17 @@ def main(argv=None):
     clocks = sampler.summary()
 
     value = w.B * w.T / (ms_def / 1000.0) * ws
-    rf = roofline_for(w, kinds_def, "append_read", peak, peak_note, traffic)
-    other = {k: roofline_for(w, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != "append_read"}
+    main_kind = "pool" if args.schedule == "pool" else "append_read"
+    rf = roofline_for(w, kinds_def, main_kind, peak, peak_note, traffic if main_kind == "append_read" else None)
+    other = {k: roofline_for(w, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != main_kind}
     step_time = {k: round(sum(ms for _, ms in v) / args.steps, 3) for k, v in kinds_def.items()}
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.schedule != "pool":
         host = {}
         for n in ("S0", "q", "k", "v", "beta", "a"):
+            if n == "beta" and w.decay == W.RWKV6:
+                continue
             host[n] = d[n].cpu().pin_memory()
         ms_e2e, h2d_b, d2h_b = run_e2e(g, w, host, L, args.schedule, max(2, args.steps // 4), args.warmup, stream)
         e2e = {"value": w.B * w.T / (ms_e2e / 1000.0) * ws, "unit": UNIT, "ms_per_step": round(ms_e2e, 3),

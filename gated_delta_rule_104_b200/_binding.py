@@ -16,12 +16,13 @@ LIB_PATH = os.path.join(HERE, "libdeltalog.so")
 
 DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = range(5)
 DL_F32, DL_BF16 = 0, 1
-DL_DECAY_HEAD, DL_DECAY_CHANNEL = 0, 1
+DL_DECAY_HEAD, DL_DECAY_CHANNEL, DL_RWKV6 = 0, 1, 2
 DL_MAX_LOG = 64
-ABI_VERSION = 4
+ABI_VERSION = 6
 
-EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
-           "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_status_string",
+EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read", "dl_log_merge",
+           "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_pool_step",
+           "dl_pool_flush", "dl_status_string",
            "dl_last_error", "dl_abi_version")
 DL_NOALLOC_WORK_BYTES = 16 << 20
 
@@ -36,6 +37,11 @@ class dl_log(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("beta", ctypes.c_void_p),
                 ("a", ctypes.c_void_p), ("x", ctypes.c_void_p), ("dtype", ctypes.c_int), ("L", ctypes.c_int),
                 ("work", ctypes.c_void_p), ("work_bytes", ctypes.c_size_t)]
+
+
+class dl_pool(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_void_p), ("s_dtype", ctypes.c_int), ("P", ctypes.c_int), ("n", ctypes.c_void_p),
+                ("status", ctypes.c_void_p), ("log", dl_log)]
 
 
 _lib = None
@@ -55,12 +61,18 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     step = [vp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
     lib.dl_gdn_decode_step.argtypes = step
     lib.dl_kda_decode_step.argtypes = step
+    lib.dl_rwkv6_decode_step.argtypes = [vp, i, vp, vp, vp, vp, i, f, i, i, i, i, vp]
     lp = ctypes.POINTER(dl_log)
     lib.dl_log_append_read.argtypes = [vp, i, i, lp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
     lib.dl_log_merge_read.argtypes = [vp, i, i, lp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    lib.dl_log_append_read_noalloc.argtypes = [vp, i, i, lp, i, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    pp = ctypes.POINTER(dl_pool)
+    lib.dl_pool_step.argtypes = [pp, i, vp, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
+    lib.dl_pool_flush.argtypes = [pp, i, vp, i, i, i, i, vp]
     lib.dl_log_merge.argtypes = [vp, i, i, lp, i, i, i, i, i, vp]
-    for name in ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_log_append_read", "dl_log_merge",
-                 "dl_log_merge_read"):
+    for name in ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read",
+                 "dl_log_merge", "dl_log_merge_read", "dl_log_append_read_noalloc", "dl_pool_step",
+                 "dl_pool_flush"):
         getattr(lib, name).restype = ctypes.c_int
     lib.dl_status_string.argtypes = [ctypes.c_int]
     lib.dl_status_string.restype = ctypes.c_char_p
@@ -105,8 +117,10 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
 
 
-def _ptr(t, name: str) -> int:
+def _ptr(t, name: str, optional: bool = False) -> Optional[int]:
     if t is None:
+        if optional:
+            return None
         raise ValueError(f"{name} is required")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -131,7 +145,7 @@ def _dims(S):
 
 
 def _in_dtype(*ts) -> int:
-    codes = {_dtype_code(t) for t in ts}
+    codes = {_dtype_code(t) for t in ts if t is not None}
     if len(codes) != 1:
         raise TypeError("q, k, v, beta and a must share one dtype")
     return codes.pop()
@@ -141,6 +155,8 @@ def _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, chan):
     exp = {"q": (q, B * H * dk), "k": (k, B * H * dk), "v": (v, B * H * dv), "beta": (beta, B * H),
            "a": (a, B * H * (dk if chan else 1)), "o": (o, B * H * dv)}
     for name, (t, n) in exp.items():
+        if t is None and name == "beta":
+            continue
         if t.numel() != n:
             raise ValueError(f"{name} has {t.numel()} elements, expected {n}")
     if o.dtype != _torch().float32:
@@ -157,6 +173,16 @@ def dl_kda_decode_step(S, q, k, v, beta, a, o, stream=None) -> None:
     _eager("dl_kda_decode_step", S, q, k, v, beta, a, o, stream, chan=True)
 
 
+def dl_rwkv6_decode_step(S, q, k, v, a, o, stream=None) -> None:
+    """Eager RWKV6 step (a [B,H,d_k]; raw-value update, no beta) in place on S."""
+    B, H, dk, dv = _dims(S)
+    _check_shapes(B, H, dk, dv, q, k, v, None, a, o, True)
+    st = _stream(stream)
+    status = load().dl_rwkv6_decode_step(_ptr(S, "S"), _dtype_code(S), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                         _ptr(a, "a"), _in_dtype(q, k, v, a), _ptr(o, "o"), B, H, dk, dv, st)
+    check("dl_rwkv6_decode_step", status)
+
+
 def _eager(fn, S, q, k, v, beta, a, o, stream, chan):
     B, H, dk, dv = _dims(S)
     _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, chan)
@@ -170,32 +196,39 @@ def _eager(fn, S, q, k, v, beta, a, o, stream, chan):
 class Log:
     """Caller-owned bounded log buffers of a deferred state (device tensors):
     k [B,H,L,d_k], v [B,H,L,d_v], beta [B,H,L], a [B,H,L] or [B,H,L,d_k],
-    x [B,H,L,L] float32 (the log's triangular solve matrix), work (fp32 workspace)."""
+    x [B,H,L,L] float32 (the log's triangular solve matrix), work (fp32 workspace).
+    An RWKV6 log (``rwkv6=True``: channel decay, no delta correction) has no
+    beta and no x (None)."""
 
-    def __init__(self, k, v, beta, a, x, L: int, channel_decay: bool, work=None):
+    def __init__(self, k, v, beta, a, x, L: int, channel_decay: bool, work=None, rwkv6: bool = False):
         self.k, self.v, self.beta, self.a, self.x = k, v, beta, a, x
         self.L = int(L)
-        self.channel_decay = bool(channel_decay)
+        self.rwkv6 = bool(rwkv6)
+        self.channel_decay = bool(channel_decay) or self.rwkv6
         self.dtype = _in_dtype(k, v, beta, a)
         self.work = work
 
     @classmethod
-    def allocate(cls, B, H, d_k, d_v, L, dtype, channel_decay, device="cuda"):
+    def allocate(cls, B, H, d_k, d_v, L, dtype, channel_decay, device="cuda", rwkv6: bool = False):
         torch = _torch()
         z = lambda *s: torch.zeros(*s, dtype=dtype, device=device)  # noqa: E731
-        a = z(B, H, L, d_k) if channel_decay else z(B, H, L)
+        chan = channel_decay or rwkv6
+        a = z(B, H, L, d_k) if chan else z(B, H, L)
         work = torch.empty(B * H * (d_k + d_v), dtype=torch.float32, device=device)
-        x = torch.zeros(B, H, L, L, dtype=torch.float32, device=device)
-        return cls(z(B, H, L, d_k), z(B, H, L, d_v), z(B, H, L), a, x, L, channel_decay, work)
+        x = None if rwkv6 else torch.zeros(B, H, L, L, dtype=torch.float32, device=device)
+        beta = None if rwkv6 else z(B, H, L)
+        return cls(z(B, H, L, d_k), z(B, H, L, d_v), beta, a, x, L, chan, work, rwkv6)
 
     def struct(self) -> dl_log:
         wp = _ptr(self.work, "log.work") if self.work is not None else None
         wb = self.work.numel() * self.work.element_size() if self.work is not None else 0
-        return dl_log(_ptr(self.k, "log.k"), _ptr(self.v, "log.v"), _ptr(self.beta, "log.beta"),
-                      _ptr(self.a, "log.a"), _ptr(self.x, "log.x"), self.dtype, self.L, wp, wb)
+        return dl_log(_ptr(self.k, "log.k"), _ptr(self.v, "log.v"), _ptr(self.beta, "log.beta", self.rwkv6),
+                      _ptr(self.a, "log.a"), _ptr(self.x, "log.x", self.rwkv6), self.dtype, self.L, wp, wb)
 
     @property
     def kind(self) -> int:
+        if self.rwkv6:
+            return DL_RWKV6
         return DL_DECAY_CHANNEL if self.channel_decay else DL_DECAY_HEAD
 
 
@@ -215,7 +248,8 @@ def _log_step(fn, S, log, n, q, k, v, beta, a, o, stream):
     st = _stream(stream)
     ls = log.struct()
     status = getattr(load(), fn)(_ptr(S, "S_base"), _dtype_code(S), log.kind, ctypes.byref(ls), int(n),
-                                 _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(beta, "beta"), _ptr(a, "a"),
+                                 _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(beta, "beta", log.rwkv6),
+                                 _ptr(a, "a"),
                                  _in_dtype(q, k, v, beta, a), _ptr(o, "o"), B, H, dk, dv, st)
     check(fn, status)
 
@@ -238,10 +272,67 @@ def dl_log_append_read_noalloc(S_base, log: Log, n: int, q, k, v, beta, a, o, st
     """As dl_log_append_read, with the scratch in the library's fixed device
     array instead of ``log.work``: for callers that cannot allocate device
     memory. Calls that overlap on the GPU race on that array."""
-    lib = load()
-    fn = lib.dl_log_append_read_noalloc
-    if fn.argtypes is None:
-        vp, i = ctypes.c_void_p, ctypes.c_int
-        fn.argtypes = [vp, i, i, ctypes.POINTER(dl_log), i, vp, vp, vp, vp, vp, i, vp, i, i, i, i, vp]
-        fn.restype = ctypes.c_int
     _log_step("dl_log_append_read_noalloc", S_base, log, n, q, k, v, beta, a, o, stream)
+
+
+# ------------------------------------------------------------------ slot pool
+
+class Pool:
+    """A pool of P per-sequence deferred states (device tensors): S [P,H,d_v,d_k],
+    ``log`` a Log over the P slots (its workspace covers a batch of up to P
+    rows), n [P] int32 log counts, status [1] int32 error word. A new sequence
+    taking slot s needs S[s] = its initial state and n[s] = 0 (``reset``)."""
+
+    def __init__(self, S, log: Log, n, status=None):
+        self.S, self.log, self.n, self.status = S, log, n, status
+        self.P = int(S.shape[0])
+
+    @classmethod
+    def allocate(cls, P, H, d_k, d_v, L, s_dtype, in_dtype, channel_decay, rwkv6: bool = False, device="cuda"):
+        torch = _torch()
+        S = torch.zeros(P, H, d_v, d_k, dtype=s_dtype, device=device)
+        log = Log.allocate(P, H, d_k, d_v, L, in_dtype, channel_decay, device=device, rwkv6=rwkv6)
+        n = torch.zeros(P, dtype=torch.int32, device=device)
+        status = torch.zeros(1, dtype=torch.int32, device=device)
+        return cls(S, log, n, status)
+
+    def reset(self, slot: int, S0) -> None:
+        """Start a new sequence in ``slot`` from state S0 [H, d_v, d_k] (stream-ordered copies)."""
+        self.S[slot].copy_(S0)
+        self.n[slot] = 0
+
+    def struct(self) -> dl_pool:
+        if self.n.dtype != _torch().int32:
+            raise TypeError("pool.n must be int32")
+        return dl_pool(_ptr(self.S, "pool.S"), _dtype_code(self.S), self.P, _ptr(self.n, "pool.n"),
+                       _ptr(self.status, "pool.status", True), self.log.struct())
+
+
+def _slots(slot, B: int) -> int:
+    torch = _torch()
+    if slot.dtype != torch.int32 or slot.numel() != B:
+        raise ValueError(f"slot must be int32 with {B} entries")
+    return _ptr(slot, "slot")
+
+
+def dl_pool_step(pool: Pool, slot, q, k, v, beta, a, o, stream=None) -> None:
+    """One decode step of the batch rows ``slot`` [B] int32 of the pool
+    (inputs and o are [B,H,...]); each row appends or, on its L-th entry,
+    merges, following its own log count."""
+    B, H, dk = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
+    dv = int(pool.S.shape[2])
+    _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, pool.log.channel_decay)
+    ps = pool.struct()
+    status = load().dl_pool_step(ctypes.byref(ps), pool.log.kind, _slots(slot, B), _ptr(q, "q"), _ptr(k, "k"),
+                                 _ptr(v, "v"), _ptr(beta, "beta", pool.log.rwkv6), _ptr(a, "a"),
+                                 _in_dtype(q, k, v, beta, a), _ptr(o, "o"), B, H, dk, dv, _stream(stream))
+    check("dl_pool_step", status)
+
+
+def dl_pool_flush(pool: Pool, slot, stream=None) -> None:
+    """Merge the listed slots' logs into their bases and zero their counts."""
+    B = int(slot.numel())
+    _, H, dv, dk = (int(x) for x in pool.S.shape)
+    ps = pool.struct()
+    status = load().dl_pool_flush(ctypes.byref(ps), pool.log.kind, _slots(slot, B), B, H, dk, dv, _stream(stream))
+    check("dl_pool_flush", status)

@@ -26,23 +26,25 @@ dl_status ok() {
 
 size_t elem_size(dl_dtype t) { return t == DL_BF16 ? 2 : 4; }
 bool valid_dtype(int t) { return t == DL_F32 || t == DL_BF16; }
-bool valid_decay(int t) { return t == DL_DECAY_HEAD || t == DL_DECAY_CHANNEL; }
+bool valid_decay(int t) { return t == DL_DECAY_HEAD || t == DL_DECAY_CHANNEL || t == DL_RWKV6; }
 
 struct Buf {
     const char *name;
     const void *p;
     size_t bytes;
     size_t align;
+    bool unused = false;  // not read by this kind (may be null)
 };
 
 bool overlaps(const Buf &a, const Buf &b) {
-    if (!a.p || !b.p || !a.bytes || !b.bytes) return false;
+    if (a.unused || b.unused || !a.p || !b.p || !a.bytes || !b.bytes) return false;
     const uintptr_t a0 = (uintptr_t)a.p, b0 = (uintptr_t)b.p;
     return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
 }
 
 dl_status check_bufs(const Buf *bufs, int nb) {
     for (int i = 0; i < nb; ++i) {
+        if (bufs[i].unused) continue;
         if (!bufs[i].p) return fail(DL_ERR_INVALID_ARG, "%s is a null pointer", bufs[i].name);
         if ((uintptr_t)bufs[i].p % bufs[i].align)
             return fail(DL_ERR_INVALID_ARG, "%s is not %zu-byte aligned", bufs[i].name, bufs[i].align);
@@ -74,19 +76,21 @@ dl_status check_dims(int B, int H, int dk, int dv, int s_dt, int in_dt) {
 // Step operands: S, q, k, v, beta, a, o (indices fixed for the callers).
 int step_bufs(Buf *out, const void *S, const char *sname, dl_dtype s_dt, const void *q, const void *k,
               const void *v, const void *beta, const void *a, dl_dtype in_dt, const float *o, int B,
-              int H, int dk, int dv, bool chan) {
+              int H, int dk, int dv, int kind) {
     const size_t bh = (size_t)B * H, is = elem_size(in_dt);
+    const bool chan = kind != DL_DECAY_HEAD;
     out[0] = {sname, S, bh * dv * dk * elem_size(s_dt), 16};
     out[1] = {"q", q, bh * dk * is, 16};
     out[2] = {"k", k, bh * dk * is, 16};
     out[3] = {"v", v, bh * dv * is, 16};
-    out[4] = {"beta", beta, bh * is, is};
+    out[4] = {"beta", beta, bh * is, is, kind == DL_RWKV6};
     out[5] = chan ? Buf{"a", a, bh * dk * is, 16} : Buf{"a", a, bh * is, is};
     out[6] = {"o", o, bh * dv * sizeof(float), 16};
     return 7;
 }
 
-dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, int dk, int dv, bool chan) {
+dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, int dk, int dv, int kind) {
+    const bool chan = kind != DL_DECAY_HEAD;
     if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
     if (!valid_dtype(log->dtype)) return fail(DL_ERR_INVALID_ARG, "unknown log dtype %d", (int)log->dtype);
     if (log->L < 1 || log->L > DL_MAX_LOG)
@@ -95,9 +99,9 @@ dl_status check_log(const dl_log *log, Buf *out, dl_dtype in_dt, int B, int H, i
     const size_t bhl = (size_t)B * H * log->L, is = elem_size(in_dt);
     out[0] = {"log.k", log->k, bhl * dk * is, 16};
     out[1] = {"log.v", log->v, bhl * dv * is, 16};
-    out[2] = {"log.beta", log->beta, bhl * is, is};
+    out[2] = {"log.beta", log->beta, bhl * is, is, kind == DL_RWKV6};
     out[3] = chan ? Buf{"log.a", log->a, bhl * dk * is, 16} : Buf{"log.a", log->a, bhl * is, is};
-    out[4] = {"log.x", log->x, bhl * log->L * sizeof(float), 16};
+    out[4] = {"log.x", log->x, bhl * log->L * sizeof(float), 16, kind == DL_RWKV6};
     return DL_OK;
 }
 
@@ -108,15 +112,15 @@ dl_status cuda_status(cudaError_t e, const char *what) {
 
 dl_status eager_step(void *S, dl_dtype s_dt, const void *q, const void *k, const void *v, const void *beta,
                      const void *a, dl_dtype in_dt, float *o, int B, int H, int dk, int dv,
-                     cudaStream_t stream, bool chan) {
+                     cudaStream_t stream, int kind) {
     dl_status s = check_dims(B, H, dk, dv, s_dt, in_dt);
     if (s != DL_OK) return s;
     Buf b[7];
-    int nb = step_bufs(b, S, "S", s_dt, q, k, v, beta, a, in_dt, o, B, H, dk, dv, chan);
+    int nb = step_bufs(b, S, "S", s_dt, q, k, v, beta, a, in_dt, o, B, H, dk, dv, kind);
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     const Buf writers[2] = {b[0], b[6]};  // S and o are written
     if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
-    dl::StepParams p{S, q, k, v, beta, a, o, B, H, dk, dv, chan, s_dt, in_dt};
+    dl::StepParams p{S, q, k, v, beta, a, o, B, H, dk, dv, kind, s_dt, in_dt};
     return cuda_status(dl::launch_eager(p, stream), "eager step launch");
 }
 
@@ -127,13 +131,19 @@ extern "C" {
 dl_status dl_gdn_decode_step(void *S, dl_dtype s_dtype, const void *q, const void *k, const void *v,
                              const void *beta, const void *a, dl_dtype in_dtype, float *o, int B, int H,
                              int d_k, int d_v, cudaStream_t stream) {
-    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, false);
+    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, DL_DECAY_HEAD);
 }
 
 dl_status dl_kda_decode_step(void *S, dl_dtype s_dtype, const void *q, const void *k, const void *v,
                              const void *beta, const void *a, dl_dtype in_dtype, float *o, int B, int H,
                              int d_k, int d_v, cudaStream_t stream) {
-    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, true);
+    return eager_step(S, s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, stream, DL_DECAY_CHANNEL);
+}
+
+dl_status dl_rwkv6_decode_step(void *S, dl_dtype s_dtype, const void *q, const void *k, const void *v,
+                               const void *a, dl_dtype in_dtype, float *o, int B, int H, int d_k, int d_v,
+                               cudaStream_t stream) {
+    return eager_step(S, s_dtype, q, k, v, nullptr, a, in_dtype, o, B, H, d_k, d_v, stream, DL_RWKV6);
 }
 
 dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_log *log, int n,
@@ -143,10 +153,9 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
-    const bool chan = kind == DL_DECAY_CHANNEL;
     Buf b[13];
-    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
-    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, kind);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, kind)) != DL_OK) return s;
     nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
@@ -160,7 +169,7 @@ dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind
     // written: o, the log (slot n, metadata row n) and its workspace; the base is only read.
     const Buf writers[7] = {b[6], b[7], b[8], b[9], b[10], b[11], b[12]};
     if ((s = check_overlap(writers, 7, b, nb)) != DL_OK) return s;
-    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, kind, s_dtype, in_dtype};
     dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_append_read(p, lg, n, static_cast<float *>(log->work), stream),
                        "append-read launch");
@@ -171,18 +180,17 @@ dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_l
     dl_status s = check_dims(B, H, d_k, d_v, s_dtype, log ? (int)log->dtype : (int)DL_F32);
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
-    const bool chan = kind == DL_DECAY_CHANNEL;
     if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
     Buf b[6];
     b[0] = {"S_base", S_base, (size_t)B * H * d_v * d_k * elem_size(s_dtype), 16};
-    if ((s = check_log(log, b + 1, log->dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    if ((s = check_log(log, b + 1, log->dtype, B, H, d_k, d_v, kind)) != DL_OK) return s;
     if ((s = check_bufs(b, 6)) != DL_OK) return s;
     if (n < 1 || n > log->L) return fail(DL_ERR_INVALID_ARG, "merge needs 1 <= n <= L (n=%d, L=%d)", n, log->L);
     const Buf writers[1] = {b[0]};
     if ((s = check_overlap(writers, 1, b, 6)) != DL_OK) return s;
     const Buf logw[5] = {b[1], b[2], b[3], b[4], b[5]};
     if ((s = check_overlap(logw, 5, b + 1, 5)) != DL_OK) return s;
-    dl::StepParams p{S_base, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, chan,
+    dl::StepParams p{S_base, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, kind,
                      s_dtype, log->dtype};
     dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, false, stream), "merge launch");
@@ -195,17 +203,16 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind, const
     dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
-    const bool chan = kind == DL_DECAY_CHANNEL;
     Buf b[12];
-    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
-    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, kind);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, kind)) != DL_OK) return s;
     nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
     if (n >= log->L) return fail(DL_ERR_LOG_FULL, "log holds n=%d of L=%d entries: merge first", n, log->L);
     const Buf writers[2] = {b[0], b[6]};  // the base and o
     if ((s = check_overlap(writers, 2, b, nb)) != DL_OK) return s;
-    dl::StepParams p{S_base, q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::StepParams p{S_base, q, k, v, beta, a, o, B, H, d_k, d_v, kind, s_dtype, in_dtype};
     dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_merge(p, lg, n, true, stream), "merge-read launch");
 }
@@ -217,10 +224,9 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
     dl_status s = check_dims(B, H, d_k, d_v, s_dtype, in_dtype);
     if (s != DL_OK) return s;
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
-    const bool chan = kind == DL_DECAY_CHANNEL;
     Buf b[12];
-    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, chan);
-    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, chan)) != DL_OK) return s;
+    int nb = step_bufs(b, S_base, "S_base", s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, kind);
+    if ((s = check_log(log, b + nb, in_dtype, B, H, d_k, d_v, kind)) != DL_OK) return s;
     nb += 5;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
     if (n < 0) return fail(DL_ERR_INVALID_ARG, "n=%d is negative", n);
@@ -233,9 +239,89 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
                     need, (size_t)DL_NOALLOC_WORK_BYTES);
     const Buf writers[6] = {b[6], b[7], b[8], b[9], b[10], b[11]};  // o and the log
     if ((s = check_overlap(writers, 6, b, nb)) != DL_OK) return s;
-    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, chan, s_dtype, in_dtype};
+    dl::StepParams p{const_cast<void *>(S_base), q, k, v, beta, a, o, B, H, d_k, d_v, kind, s_dtype, in_dtype};
     dl::LogParams lg{log->k, log->v, log->beta, log->a, log->x, log->L};
     return cuda_status(dl::launch_append_read_noalloc(p, lg, n, stream), "no-alloc append-read launch");
+}
+
+// ------------------------------------------------------------------ slot pool
+
+static dl_status pool_checks(const dl_pool *pool, dl_decay kind, const int *slot, dl_dtype in_dt, int B, int H,
+                             int d_k, int d_v, Buf *b, int &nb) {
+    if (!pool) return fail(DL_ERR_INVALID_ARG, "pool is a null pointer");
+    dl_status s = check_dims(B, H, d_k, d_v, pool->s_dtype, in_dt);
+    if (s != DL_OK) return s;
+    if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
+    if (pool->P < 1) return fail(DL_ERR_INVALID_ARG, "pool.P=%d must be >= 1", pool->P);
+    if (B > pool->P) return fail(DL_ERR_INVALID_ARG, "B=%d rows need distinct slots but P=%d", B, pool->P);
+    if ((long long)pool->P * H > (1LL << 26)) return fail(DL_ERR_UNSUPPORTED, "P*H exceeds 2^26");
+    if ((s = check_log(&pool->log, b + nb, in_dt, pool->P, H, d_k, d_v, kind)) != DL_OK) return s;
+    nb += 5;
+    b[nb++] = {"pool.n", pool->n, (size_t)pool->P * sizeof(int), 4};
+    b[nb++] = {"slot", slot, (size_t)B * sizeof(int), 4};
+    b[nb++] = {"pool.status", pool->status, sizeof(int), 4, pool->status == nullptr};
+    return DL_OK;
+}
+
+dl_status dl_pool_step(const dl_pool *pool, dl_decay kind, const int *slot, const void *q, const void *k,
+                       const void *v, const void *beta, const void *a, dl_dtype in_dtype, float *o, int B, int H,
+                       int d_k, int d_v, cudaStream_t stream) {
+    Buf b[17];
+    int nb = 7;
+    if (pool) step_bufs(b, pool->S, "pool.S", pool->s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, kind);
+    dl_status s = pool_checks(pool, kind, slot, in_dtype, B, H, d_k, d_v, b, nb);
+    if (s != DL_OK) return s;
+    b[0].bytes = (size_t)pool->P * H * d_v * d_k * elem_size(pool->s_dtype);  // the whole pool
+    const size_t need = dl::read_work_bytes(B, H, d_k, d_v);
+    b[nb++] = {"log.work", pool->log.work, need, 16};
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    if (pool->log.work_bytes < need)
+        return fail(DL_ERR_INVALID_ARG, "log.work holds %zu bytes, needs %zu", pool->log.work_bytes, need);
+    // written: the pool's bases (merging slots), o, the logs, counts, status, workspace
+    const Buf writers[10] = {b[0], b[6], b[7], b[8], b[9], b[10], b[11], b[12], b[14], b[15]};
+    if ((s = check_overlap(writers, 10, b, nb)) != DL_OK) return s;
+    dl::StepParams p{pool->S, q, k, v, beta, a, o, B, H, d_k, d_v, kind, pool->s_dtype, in_dtype};
+    const dl_log *lg0 = &pool->log;
+    dl::LogParams lg{lg0->k, lg0->v, lg0->beta, lg0->a, lg0->x, lg0->L};
+    dl::PoolIdx pi;
+    pi.slot = slot;
+    pi.counts = pool->n;
+    pi.status = pool->status;
+    pi.P = pool->P;
+    pi.H = H;
+    pi.L = lg0->L;
+    // the merge part (rows on their L-th entry) first; the append part of the
+    // other rows runs beside it (programmatic dependent launch), then the counts
+    cudaError_t e = dl::launch_merge(p, lg, lg0->L - 1, true, stream, pi, dl::POOL_MERGE_FULL);
+    if (e == cudaSuccess) e = dl::launch_append_read(p, lg, 0, static_cast<float *>(lg0->work), stream, pi);
+    if (e == cudaSuccess) e = dl::launch_pool_counts(pi, B, true, stream);
+    return cuda_status(e, "pool step launch");
+}
+
+dl_status dl_pool_flush(const dl_pool *pool, dl_decay kind, const int *slot, int B, int H, int d_k, int d_v,
+                        cudaStream_t stream) {
+    Buf b[10];
+    int nb = 1;
+    if (pool) b[0] = {"pool.S", pool->S, (size_t)pool->P * H * d_v * d_k * elem_size(pool->s_dtype), 16};
+    dl_status s = pool_checks(pool, kind, slot, pool ? pool->log.dtype : DL_F32, B, H, d_k, d_v, b, nb);
+    if (s != DL_OK) return s;
+    if ((s = check_bufs(b, nb)) != DL_OK) return s;
+    const Buf writers[3] = {b[0], b[6], b[8]};  // bases, counts, status
+    if ((s = check_overlap(writers, 3, b, nb)) != DL_OK) return s;
+    dl::StepParams p{pool->S, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, d_k, d_v, kind,
+                     pool->s_dtype, pool->log.dtype};
+    const dl_log *lg0 = &pool->log;
+    dl::LogParams lg{lg0->k, lg0->v, lg0->beta, lg0->a, lg0->x, lg0->L};
+    dl::PoolIdx pi;
+    pi.slot = slot;
+    pi.counts = pool->n;
+    pi.status = pool->status;
+    pi.P = pool->P;
+    pi.H = H;
+    pi.L = lg0->L;
+    cudaError_t e = dl::launch_merge(p, lg, lg0->L - 1, false, stream, pi, dl::POOL_FLUSH);
+    if (e == cudaSuccess) e = dl::launch_pool_counts(pi, B, false, stream);
+    return cuda_status(e, "pool flush launch");
 }
 
 const char *dl_status_string(dl_status s) {

@@ -25,6 +25,8 @@
 // row (the same kind of dots as d_e), extends X by one row and stores it. A
 // read is then two parallel dot passes with no serial solve, and the merge
 // uses the same X.
+// RWKV6 (no delta correction: A_e = Diag(a_e), value added raw) is the case
+// X = I: s_e = d_e and x_0 = gamma_n o q.
 //
 // Two kernels, chained with programmatic dependent launch:
 //   replay_prep   one warp per head: stages the head's log keys and decays
@@ -56,13 +58,15 @@ struct PrepSmem {  // one warp's staging area
     static constexpr int BYTES = F_OFF + FLOATS * 4;
 };
 
-template <class IT, int DK, int DV, bool CHAN, int EMAX>
+template <class IT, int DK, int DV, int KIND, int EMAX>
 __global__ void __launch_bounds__(128)
 replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                    const IT *__restrict__ beta, const IT *__restrict__ a, IT *__restrict__ log_k,
                    IT *__restrict__ log_v, IT *__restrict__ log_b, IT *__restrict__ log_a,
-                   float *__restrict__ log_x, int L, int n, float *__restrict__ work, long long heads) {
+                   float *__restrict__ log_x, int L, int n, float *__restrict__ work, long long heads,
+                   PoolIdx pool) {
     pdl_launch_dependents();
+    constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
     using P = PrepSmem<IT, DK, EMAX, CHAN>;
     constexpr int CW = DK / 32;            // key columns per lane (contiguous)
     constexpr int RV = DV / 32;            // value rows per lane
@@ -76,9 +80,17 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     float *fas = reinterpret_cast<float *>(base + P::F_OFF);
     float *fbeta = fas + EMAX, *fd = fbeta + EMAX, *fcn = fd + EMAX, *fs = fcn + EMAX, *xrow = fs + EMAX;
 
-    const long long head = (long long)blockIdx.x * (blockDim.x / 32) + warp;
-    if (head >= heads) return;
-    const long long lrow = head * L;
+    // A pool step launches this kernel as a programmatic dependent of its merge
+    // part (which works on other slots), so the two overlap; every warp waits
+    // for that grid before it exits, so that this grid's completion implies the
+    // merge's for the kernels after it. (A no-op for an ordinary launch.)
+    const long long head = (long long)blockIdx.x * (blockDim.x / 32) + warp;  // batch head (inputs, work)
+    long long shead;  // state / log head (a pool slot's, or the batch head itself)
+    if (head >= heads || !pool_head(pool, POOL_APPEND, head, shead, n)) {
+        pdl_wait();
+        return;
+    }
+    const long long lrow = shead * L;
     const int c0 = lane * CW, r0 = lane * RV;
     // The log stays L2-resident between steps: its reads and writes carry an
     // evict-last policy (the base streams through with evict-first).
@@ -97,10 +109,12 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     }
     cp_async_commit();
     for (int e = lane; e <= n; e += 32) {
-        float bx[1];
-        if (e < n) load_vec_hint<1>(log_b + lrow + e, bx, keep);
-        else bx[0] = to_f(beta[head]);
-        fbeta[e] = bx[0];
+        if constexpr (DELTA) {
+            float bx[1];
+            if (e < n) load_vec_hint<1>(log_b + lrow + e, bx, keep);
+            else bx[0] = to_f(beta[head]);
+            fbeta[e] = bx[0];
+        }
         if constexpr (!CHAN) {
             float ax[1];
             if (e < n) load_vec_hint<1>(log_a + lrow + e, ax, keep);
@@ -109,7 +123,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         }
     }
     // X rows of the logged entries (rows j < n, columns e <= j).
-    for (int u = lane; u < n * EMAX; u += 32) {
+    for (int u = lane; DELTA && u < n * EMAX; u += 32) {
         const int j = u / EMAX, e = u % EMAX;
         if (e <= j) {
             float xx[1];
@@ -125,7 +139,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     } else if (lane == 0) {
         copy_hint<1>(log_a + lrow + n, a + head, keep);
     }
-    if (lane == 0) copy_hint<1>(log_b + lrow + n, beta + head, keep);
+    if (DELTA && lane == 0) copy_hint<1>(log_b + lrow + n, beta + head, keep);
     float qv[CW];
     load_vec<CW>(q + head * DK + c0, qv);
     cp_async_wait_all();
@@ -159,14 +173,16 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll
                 for (int c = 0; c < CW; ++c) {
                     pd[jj] = fmaf(ke[c], z[c], pd[jj]);
-                    pc[jj] = fmaf(ke[c], y[c], pc[jj]);
                     z[c] *= ae[c];
-                    y[c] *= ae[c];
+                    if constexpr (DELTA) {
+                        pc[jj] = fmaf(ke[c], y[c], pc[jj]);
+                        y[c] *= ae[c];
+                    }
                 }
             }
         }
         multi_sum<CH>(pd, lane);
-        multi_sum<CH>(pc, lane);
+        if constexpr (DELTA) multi_sum<CH>(pc, lane);
         constexpr int shift = CH == 32 ? 0 : CH == 16 ? 1 : CH == 8 ? 2 : 3;
         const int e = top - (lane >> shift);
         if ((lane & ((1 << shift) - 1)) == 0 && e >= 0) {
@@ -176,8 +192,8 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     }
     __syncwarp();
     // X row n: X(n, n) = beta_n, X(n, j) = -beta_n sum_{m=j..n-1} C(n, m) X(m, j).
-    const float bn = fbeta[n];
-    for (int j = lane; j <= n; j += 32) {
+    const float bn = DELTA ? fbeta[n] : 0.f;
+    for (int j = lane; DELTA && j <= n; j += 32) {
         float acc = 0.f;
         for (int m = j; m < n; ++m) acc = fmaf(fcn[m], xrow[m * EMAX + j], acc);
         const float xnj = j == n ? bn : -bn * acc;
@@ -188,7 +204,11 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     // s_e = sum_{i=e..n} X(i, e) d_i (the back-substitution, as one dot per entry).
     for (int e = lane; e <= n; e += 32) {
         float acc = 0.f;
-        for (int i = e; i <= n; ++i) acc = fmaf(xrow[i * EMAX + e], fd[i], acc);
+        if constexpr (DELTA) {
+            for (int i = e; i <= n; ++i) acc = fmaf(xrow[i * EMAX + e], fd[i], acc);
+        } else {
+            acc = fd[e];
+        }
         fs[e] = acc;
     }
     __syncwarp();
@@ -208,7 +228,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
             g[c] *= ae[c];
-            xs[c] = fmaf(se * g[c], ke[c], xs[c]);
+            if constexpr (DELTA) xs[c] = fmaf(se * g[c], ke[c], xs[c]);
         }
     }
     float w[RV];
@@ -229,6 +249,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     for (int c = 0; c < CW; ++c) wk[c0 + c] = fmaf(g[c], qv[c], -xs[c]);
 #pragma unroll
     for (int r = 0; r < RV; ++r) wk[DK + r0 + r] = w[r];
+    pdl_wait();
 }
 
 // ------------------------------------------------------------------ decode
@@ -246,24 +267,26 @@ struct DecodeShape {
 template <class ST, int DK, int DV>
 __global__ void __launch_bounds__(256)
 append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work, float *__restrict__ o,
-                     long long num_units) {
+                     long long num_units, PoolIdx pool) {
     using C = DecodeShape<ST, DK>;
     constexpr int VEC = C::VEC;
     static_assert(DV % C::UNIT == 0, "unit divides d_v");
     const int lane = threadIdx.x & 31;
     const long long unit = (long long)blockIdx.x * C::WARPS + (threadIdx.x >> 5);
-    const bool active = unit < num_units;
     const long long row0 = unit * C::UNIT;
-    const long long head = row0 / DV;
+    const long long head = row0 / DV;  // batch head (work, o)
     const int rin0 = (int)(row0 - head * DV);
     const int sub = lane / C::G;
     const int col = (lane % C::G) * VEC;
+    long long shead = head;  // state head
+    int n_unused = 0;
+    const bool active = unit < num_units && pool_head(pool, POOL_APPEND, head, shead, n_unused);
 
     // D3 operands: the base rows first (read only, streamed).
     uint4 raw[C::R];
     if (active) {
         const uint64_t stream = l2_policy_stream();
-        const ST *src = Sbar + (row0 + sub) * DK + col;
+        const ST *src = Sbar + (shead * DV + rin0 + sub) * DK + col;
 #pragma unroll
         for (int r = 0; r < C::R; ++r) raw[r] = ld_ro_hint(src + (long long)r * C::RPW * DK, stream);
     }
@@ -288,7 +311,7 @@ append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work
 size_t read_work_bytes(int B, int H, int dk, int dv) { return (size_t)B * H * (dk + dv) * sizeof(float); }
 
 template <class ST, int DK, int DV>
-static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStream_t st) {
+static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStream_t st, const PoolIdx &pool) {
     using C = DecodeShape<ST, DK>;
     const long long units = (long long)p.B * p.H * DV / C::UNIT;
     const long long blocks = (units + C::WARPS - 1) / C::WARPS;
@@ -303,14 +326,15 @@ static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStr
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, append_decode_kernel<ST, DK, DV>, static_cast<const ST *>(p.S), work, p.o,
-                              units);
+                              units, pool);
 }
 
-template <class IT, int DK, int DV, bool CH, int EMAX>
-static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st) {
-    using P = PrepSmem<IT, DK, EMAX, CH>;
+template <class IT, int DK, int DV, int KD, int EMAX>
+static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
+                               const PoolIdx &pool) {
+    using P = PrepSmem<IT, DK, EMAX, Rule<KD>::CHAN>;
     constexpr int WARPS = EMAX <= 32 ? 4 : 2;
-    auto kern = replay_prep_kernel<IT, DK, DV, CH, EMAX>;
+    auto kern = replay_prep_kernel<IT, DK, DV, KD, EMAX>;
     const size_t smem = (size_t)WARPS * P::BYTES;
     static bool configured = false;
     if (!configured && smem > 48 * 1024) {
@@ -319,26 +343,36 @@ static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, 
         configured = true;
     }
     const long long heads = (long long)p.B * p.H;
-    kern<<<(unsigned)((heads + WARPS - 1) / WARPS), WARPS * 32, smem, st>>>(
-        static_cast<const IT *>(p.q), static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
-        static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
-        static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.x, lg.L, n, work, heads);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((heads + WARPS - 1) / WARPS));
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pool.slot ? 1 : 0;  // a pool step overlaps it with its merge part
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
+                              static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta),
+                              static_cast<const IT *>(p.a), static_cast<IT *>(lg.k), static_cast<IT *>(lg.v),
+                              static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.x, lg.L, n, work, heads, pool);
 }
 
-cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st) {
+cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
+                               const PoolIdx &pool) {
     return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
         using ST = decltype(st_t);
         using IT = decltype(it_t);
         constexpr int DK = decltype(dk_c)::value;
         constexpr int DV = decltype(dv_c)::value;
-        constexpr bool CH = decltype(ch_c)::value;
+        constexpr int KD = decltype(ch_c)::value;
         cudaError_t e;
-        if (lg.L <= 16) e = launch_prep<IT, DK, DV, CH, 16>(p, lg, n, work, st);
-        else if (lg.L <= 32) e = launch_prep<IT, DK, DV, CH, 32>(p, lg, n, work, st);
-        else e = launch_prep<IT, DK, DV, CH, 64>(p, lg, n, work, st);
+        if (lg.L <= 16) e = launch_prep<IT, DK, DV, KD, 16>(p, lg, n, work, st, pool);
+        else if (lg.L <= 32) e = launch_prep<IT, DK, DV, KD, 32>(p, lg, n, work, st, pool);
+        else e = launch_prep<IT, DK, DV, KD, 64>(p, lg, n, work, st, pool);
         if (e != cudaSuccess) return e;
-        e = launch_decode<ST, DK, DV>(p, work, st);
+        e = launch_decode<ST, DK, DV>(p, work, st, pool);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     });

@@ -5,6 +5,8 @@
 // Per (b, h), with S' = S Diag(a):
 //   u = S' k,  p = S' q,  S <- S' + beta (v - u) k^T,  o = p + beta (v - u) (k . q)
 // which is S_t = S_{t-1} Diag(a)(I - beta k k^T) + beta v k^T and o = S_t q.
+// RWKV6 (raw-value update, no delta correction) takes d = v in place of
+// beta (v - u): S <- S' + v k^T, o = p + v (k . q).
 //
 // HBM-bound streaming kernel (about 1 FLOP per state byte). Layout: one state
 // row (d_k contiguous elements, 128-512 bytes) is spread over a group of G
@@ -30,13 +32,14 @@ struct EagerShape {
     static_assert(G >= 1 && G <= 32 && 32 % G == 0, "row group");
 };
 
-template <class ST, class IT, int DK, int DV, bool CHAN>
+template <class ST, class IT, int DK, int DV, int KIND>
 __global__ void __launch_bounds__(256)
 eager_step_kernel(ST *__restrict__ S, const IT *__restrict__ q, const IT *__restrict__ k,
                   const IT *__restrict__ v, const IT *__restrict__ beta, const IT *__restrict__ a,
                   float *__restrict__ o, long long num_units) {
     using C = EagerShape<ST, DK>;
     constexpr int VEC = C::VEC;
+    constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
     const int lane = threadIdx.x & 31;
     const long long unit = (long long)blockIdx.x * C::WARPS + (threadIdx.x >> 5);
     if (unit >= num_units) return;  // whole warps leave together
@@ -64,7 +67,7 @@ eager_step_kernel(ST *__restrict__ S, const IT *__restrict__ q, const IT *__rest
 #pragma unroll
         for (int e = 0; e < VEC; ++e) aa[e] = as;
     }
-    const float b = to_f(beta[head]);
+    const float b = DELTA ? to_f(beta[head]) : 1.f;
     float vr[C::R];
 #pragma unroll
     for (int r = 0; r < C::R; ++r) vr[r] = to_f(v[head * DV + rin0 + r * C::RPW + sub]);
@@ -81,13 +84,13 @@ eager_step_kernel(ST *__restrict__ S, const IT *__restrict__ q, const IT *__rest
         float u = 0.f, pq = 0.f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            s[e] *= aa[e];                 // E2: decay
-            u = fmaf(s[e], kk[e], u);      // E3: S'k
-            pq = fmaf(s[e], qq[e], pq);    //     S'q
+            s[e] *= aa[e];                           // E2: decay
+            if constexpr (DELTA) u = fmaf(s[e], kk[e], u);  // E3: S'k
+            pq = fmaf(s[e], qq[e], pq);              //     S'q
         }
-        u = group_sum<C::G>(u);
+        if constexpr (DELTA) u = group_sum<C::G>(u);
         pq = group_sum<C::G>(pq);
-        const float d = b * (vr[r] - u);   // E4: beta (v - S'k)
+        const float d = DELTA ? b * (vr[r] - u) : vr[r];  // E4: beta (v - S'k), or v
 #pragma unroll
         for (int e = 0; e < VEC; ++e) s[e] = fmaf(d, kk[e], s[e]);
         st_stream(srow + (long long)r * C::RPW * DK, StateVec<ST>::pack(s));
@@ -102,13 +105,13 @@ cudaError_t launch_eager(const StepParams &p, cudaStream_t st) {
         using IT = decltype(it_t);
         constexpr int DK = decltype(dk_c)::value;
         constexpr int DV = decltype(dv_c)::value;
-        constexpr bool CH = decltype(ch_c)::value;
+        constexpr int KD = decltype(ch_c)::value;
         using C = EagerShape<ST, DK>;
         static_assert(DV % C::UNIT == 0, "unit divides d_v");
         const long long rows = (long long)p.B * p.H * DV;
         const long long units = rows / C::UNIT;
         const long long blocks = (units + C::WARPS - 1) / C::WARPS;
-        eager_step_kernel<ST, IT, DK, DV, CH><<<(unsigned)blocks, C::WARPS * 32, 0, st>>>(
+        eager_step_kernel<ST, IT, DK, DV, KD><<<(unsigned)blocks, C::WARPS * 32, 0, st>>>(
             static_cast<ST *>(p.S), static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
             static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a),
             p.o, units);

@@ -14,8 +14,16 @@ struct StepParams {
     const void *q, *k, *v, *beta, *a;  // this step's inputs (may be null for a plain merge)
     float *o;            // [B, H, d_v] output (may be null for a plain merge)
     int B, H, dk, dv;
-    bool chan;           // channel-wise decay (KDA) vs head-wise (GDN)
+    int kind;            // dl_decay: GDN (head decay), KDA (channel decay), RWKV6 (channel decay, no delta)
     dl_dtype s_dt, in_dt;
+    bool chan() const { return kind != DL_DECAY_HEAD; }
+};
+
+// Compile-time rule of a kernel instantiation (the dl_decay value).
+template <int KIND>
+struct Rule {
+    static constexpr bool CHAN = KIND != DL_DECAY_HEAD;  // a decay value per key channel
+    static constexpr bool DELTA = KIND != DL_RWKV6;      // delta-rule correction (beta, S'k)
 };
 
 struct LogParams {
@@ -24,24 +32,68 @@ struct LogParams {
     int L;
 };
 
+// Slot indirection of the pool entry points. With slot == nullptr (the plain
+// entry points) batch head i is state/log head i and the log count is the
+// launch's scalar n. Otherwise batch row b works on state and log slot
+// slot[b] with counts[slot[b]] entries; a launch only takes the rows its part
+// of the step owns (PoolPart), and rows whose slot or count is out of range
+// are skipped (and flagged in *status, when given).
+enum PoolPart { POOL_APPEND = 0, POOL_MERGE_FULL = 1, POOL_FLUSH = 2 };
+struct PoolIdx {
+    const int *slot = nullptr;  // [B] slot of each batch row
+    int *counts = nullptr;        // [P] log entries held per slot
+    int *status = nullptr;        // optional error word (bit 0: a slot or count out of range)
+    int P = 0, H = 1, L = 0;
+};
+
+// Batch head -> (state head, count) for one part of a pool step; false if the
+// head is not this launch's to process.
+__device__ __forceinline__ bool pool_head(const PoolIdx &pi, int part, long long head, long long &shead, int &n) {
+    if (pi.slot == nullptr) {
+        shead = head;
+        return true;
+    }
+    const long long b = head / pi.H;
+    const int h = (int)(head - b * pi.H);
+    const int s = pi.slot[b];
+    const int c = (s >= 0 && s < pi.P) ? pi.counts[s] : -1;
+    if (c < 0 || c >= pi.L) {
+        if (pi.status && h == 0) atomicOr(pi.status, 1);
+        return false;
+    }
+    shead = (long long)s * pi.H + h;
+    n = c;
+    if (part == POOL_APPEND) return c < pi.L - 1;
+    if (part == POOL_MERGE_FULL) return c == pi.L - 1;
+    return c > 0;  // POOL_FLUSH
+}
+
 cudaError_t launch_eager(const StepParams &p, cudaStream_t st);
 // Deferred read: needs read_work_bytes() of fp32 workspace (x_0 and w per head).
-cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st);
+cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
+                               const PoolIdx &pool = PoolIdx{});
 size_t read_work_bytes(int B, int H, int dk, int dv);
 // The same with the scratch in a fixed module array (DL_NOALLOC_WORK_BYTES).
 cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg, int n, cudaStream_t st);
 // Merge n_log log entries (plus, if with_cur, this step's inputs as one more
 // entry, and then o = S_new q) into the base.
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,
-                         cudaStream_t st);
+                         cudaStream_t st, const PoolIdx &pool = PoolIdx{}, int part = POOL_MERGE_FULL);
+// Pool bookkeeping after a step (advance = true: count + 1, or 0 after the L-th
+// entry merged) or a flush (advance = false: count = 0), for each batch row's slot.
+cudaError_t launch_pool_counts(const PoolIdx &pool, int B, bool advance, cudaStream_t st);
 
-// Calls f(ST{}, IT{}, DK_constant, DV_constant, CHAN_constant) with the
+// Calls f(ST{}, IT{}, DK_constant, DV_constant, KIND_constant) with the
 // compile-time types/sizes matching the runtime description.
 template <class F>
 cudaError_t dispatch(const StepParams &p, F &&f) {
     auto with_chan = [&](auto st, auto it, auto dk, auto dv) -> cudaError_t {
-        if (p.chan) return f(st, it, dk, dv, std::true_type{});
-        return f(st, it, dk, dv, std::false_type{});
+        switch (p.kind) {
+            case DL_DECAY_HEAD: return f(st, it, dk, dv, std::integral_constant<int, DL_DECAY_HEAD>{});
+            case DL_DECAY_CHANNEL: return f(st, it, dk, dv, std::integral_constant<int, DL_DECAY_CHANNEL>{});
+            case DL_RWKV6: return f(st, it, dk, dv, std::integral_constant<int, DL_RWKV6>{});
+        }
+        return cudaErrorInvalidValue;
     };
     auto with_dv = [&](auto st, auto it, auto dk) -> cudaError_t {
         switch (p.dv) {

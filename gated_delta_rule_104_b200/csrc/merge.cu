@@ -25,6 +25,8 @@
 // state, so every operand is split as x = hi + lo (two TF32 values) and each
 // product is formed as hi*hi + hi*lo + lo*hi, which recovers ~fp32 accuracy.
 //
+// RWKV6 (no delta correction) is the case X = I and no G: delta = V.
+//
 // Kernel: one block per (head, tile of up to 128 rows); warp w owns rows
 // 16w..16w+15 of the tile. The entries are merged in blocks of NB = 8 or 16
 // (a longer log is a chain of sub-merges; short blocks are padded with
@@ -75,16 +77,6 @@ __device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ah)[4], con
 
 __device__ __forceinline__ float ld_state(const float *p) { return *p; }
 __device__ __forceinline__ float ld_state(const bf16 *p) { return to_f(*p); }
-__device__ __forceinline__ void ld_state2(const float *p, float &x, float &y) {
-    const float2 v = *reinterpret_cast<const float2 *>(p);
-    x = v.x;
-    y = v.y;
-}
-__device__ __forceinline__ void ld_state2(const bf16 *p, float &x, float &y) {
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
-    x = bf_lo(w);
-    y = bf_hi(w);
-}
 __device__ __forceinline__ void st_state2(float *p, float x, float y) {
     __stcs(reinterpret_cast<float2 *>(p), make_float2(x, y));
 }
@@ -96,77 +88,130 @@ __device__ __forceinline__ void st_state2(bf16 *p, float x, float y) {
 
 __host__ __device__ constexpr size_t round4(size_t x) { return (x + 3) & ~(size_t)3; }
 
-template <int DK>
+template <int DK, int NB>
 struct MergeShape {
+    static constexpr int ROWS = 64;     // base rows per block: 4 warps of 16
     static constexpr int KH = DK + 4;   // Khat row stride (conflict-free B-fragment reads)
-    static constexpr int WS = DK + 8;   // W row stride (conflict-free B-fragment reads)
+    static constexpr int WS = DK + 8;   // F row stride (conflict-free B-fragment reads)
+    static constexpr int XS = NB + 4;   // X row stride (conflict-free B-fragment reads)
+    static constexpr int VS = ROWS + 4; // value row stride (conflict-free accumulator-layout reads)
     static constexpr int CW = DK / 32;  // key channels per lane (warp-wide dots)
-    __host__ __device__ static constexpr int rows(int dv) { return 64; }  // 4 warps per block
 };
 
-// Shared memory for one block of NB entries (all float):
-//   fk [NB][DK] keys   fa: channel decay [NB][DK] or head decay [NB] (padded to 4)
-//   ff [NB][DK] F      kh [NB][KH] Khat   sw [NB][WS] W
-//   gn [DK] gamma      sq [DK] q          cm [NB] C row   sx [NB][NB] X   sb [NB] beta
-//   sv [NB][rows] the tile's values
-template <int DK, bool CHAN, int NB>
-__host__ __device__ constexpr size_t merge_smem_bytes(int rows) {
-    using C = MergeShape<DK>;
-    const size_t floats = (size_t)NB * DK + (CHAN ? (size_t)NB * DK : round4(NB)) + (size_t)NB * DK +
-                          (size_t)NB * C::KH + (size_t)NB * C::WS + DK + DK + round4(NB) + (size_t)NB * NB + round4(NB) +
-                          (size_t)NB * rows;
-    return floats * sizeof(float);
+// The block's base rows in shared memory: ROWS x DK elements of the state
+// type, row-major with the 16-byte chunks of row r XOR-swizzled by (r mod 8),
+// so that an 8-row x 4-column fragment read touches 32 distinct banks
+// without padding.
+template <class ST, int DK>
+struct BaseTile {
+    static constexpr int CE = 16 / (int)sizeof(ST);  // elements per 16-byte chunk
+    static_assert(DK / CE >= 8, "swizzle spans 8 chunks");
+    __device__ static __forceinline__ int off(int r, int c) {
+        return r * DK + (((c / CE) ^ (r & 7)) * CE) + (c % CE);
+    }
+};
+
+// Shared memory (bytes) of one block for NB-entry sub-merges:
+//   tile [ROWS][DK] of ST (swizzled base rows), then floats:
+//   kh [NB][KH] keys, turned into Khat in place
+//   ff [NB][WS] F (channel decay: holds the decays until F replaces them)
+//   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
+//   cm [NB] C row   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
+template <class ST, int DK, int NB>
+__host__ __device__ constexpr size_t merge_smem_bytes() {
+    using C = MergeShape<DK, NB>;
+    const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK + round4(NB) +
+                          (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS;
+    return (size_t)C::ROWS * DK * sizeof(ST) + floats * sizeof(float);
+}
+
+__device__ __forceinline__ float2 ld_tile2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+__device__ __forceinline__ float2 ld_tile2(const bf16 *p) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+    return make_float2(bf_lo(w), bf_hi(w));
+}
+__device__ __forceinline__ void st_tile2(float *p, float x, float y) {
+    *reinterpret_cast<float2 *>(p) = make_float2(x, y);
+}
+__device__ __forceinline__ void st_tile2(bf16 *p, float x, float y) {
+    *reinterpret_cast<uint32_t *>(p) = pack_bf2(x, y);
+}
+
+// Accumulator layout (rows g, g + 8; columns 8i + 2t, 8i + 2t + 1) to A-operand
+// layout (columns 8i + t, 8i + t + 4) of a 16 x 8NT tile, split into TF32 hi + lo.
+template <int NT>
+__device__ __forceinline__ void acc_to_operand(const float (&x)[NT][4], uint32_t (&hi)[NT][4],
+                                               uint32_t (&lo)[NT][4], int lane) {
+    const int t = lane & 3;
+    const int s0 = (lane & ~3) | (t >> 1), s1 = s0 + 2;  // quad lanes holding columns t, t + 4
+    const bool odd = t & 1;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        const float x00 = __shfl_sync(0xffffffffu, x[i][0], s0), x01 = __shfl_sync(0xffffffffu, x[i][1], s0);
+        const float x10 = __shfl_sync(0xffffffffu, x[i][2], s0), x11 = __shfl_sync(0xffffffffu, x[i][3], s0);
+        const float y00 = __shfl_sync(0xffffffffu, x[i][0], s1), y01 = __shfl_sync(0xffffffffu, x[i][1], s1);
+        const float y10 = __shfl_sync(0xffffffffu, x[i][2], s1), y11 = __shfl_sync(0xffffffffu, x[i][3], s1);
+        split_tf32(odd ? x01 : x00, hi[i][0], lo[i][0]);  // [g][8i + t]
+        split_tf32(odd ? x11 : x10, hi[i][1], lo[i][1]);  // [g + 8][8i + t]
+        split_tf32(odd ? y01 : y00, hi[i][2], lo[i][2]);  // [g][8i + t + 4]
+        split_tf32(odd ? y11 : y10, hi[i][3], lo[i][3]);  // [g + 8][8i + t + 4]
+    }
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <class ST, int DK, bool CHAN, bool WITH_CUR, int NB>
-__global__ void __launch_bounds__(256, 2)
+template <class ST, int DK, int KIND, bool WITH_CUR, int NB>
+__global__ void __launch_bounds__(128, 4)
 merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__restrict__ log_v,
              const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_x,
              int L, int n_log, const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
-             const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV, bool bf) {
-    using C = MergeShape<DK>;
+             const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV, bool bf,
+             PoolIdx pool, int part) {
+    using C = MergeShape<DK, NB>;
+    using TL = BaseTile<ST, DK>;
+    constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
     constexpr int KS = DK / 8;   // k-steps of the first product / column tiles of the second
     constexpr int NT = NB / 8;   // entry tiles
-    const int ROWS = blockDim.x / 2;  // 16 rows per warp
-    const int nthr = blockDim.x;
-    const int NTOT = n_log + (WITH_CUR ? 1 : 0);
+    constexpr int ROWS = C::ROWS;
+    constexpr int nthr = 2 * ROWS;  // 4 warps, 16 rows each
 
     extern __shared__ float4 smem_raw[];
-    float *fk = reinterpret_cast<float *>(smem_raw);
-    float *fa = fk + NB * DK;
-    float *ff = fa + (CHAN ? NB * DK : (int)round4(NB));
-    float *kh = ff + NB * DK;
-    float *sw = kh + NB * C::KH;
-    float *gn = sw + NB * C::WS;
+    ST *tile = reinterpret_cast<ST *>(smem_raw);
+    float *kh = reinterpret_cast<float *>(tile + ROWS * DK);
+    float *ff = kh + NB * C::KH;
+    float *fa = ff + NB * C::WS;
+    float *gn = fa + round4(NB);
     float *sq = gn + DK;
     float *cm = sq + DK;
     float *sx = cm + round4(NB);
-    float *sb = sx + NB * NB;
+    float *sb = sx + NB * C::XS;
     float *sv = sb + round4(NB);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;  // fragment coordinates
     const int tiles = DV / ROWS;
-    const long long head = blockIdx.x / tiles;
+    const long long head = blockIdx.x / tiles;  // batch head (this step's inputs, o)
     const int row0 = (blockIdx.x % tiles) * ROWS;
-    const long long lrow = head * L;
-    ST *Sw = S + (head * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
+    long long shead;                            // state / log head
+    pdl_launch_dependents();  // a pool step's append part (other slots) may start beside this grid
+    if (!pool_head(pool, part, head, shead, n_log)) return;  // the whole block: no barrier passed yet
+    const int NTOT = n_log + (WITH_CUR ? 1 : 0);
+    const long long lrow = shead * L;
+    ST *Sw = S + (shead * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
+    const int tr = 16 * warp;                           // and their first row in the tile
 
-    // First-product operand fragments of the warp's rows, fetched before anything
-    // else (they land while the key side is prepared): a0 = S[g][8s + t],
-    // a1 = S[g + 8][8s + t], a2 = S[g][8s + t + 4], a3 = S[g + 8][8s + t + 4].
-    float afr[KS][4];
-    auto load_afr = [&]() {
-#pragma unroll
-        for (int s = 0; s < KS; ++s) {
-            afr[s][0] = ld_state(Sw + g * DK + 8 * s + t);
-            afr[s][1] = ld_state(Sw + (g + 8) * DK + 8 * s + t);
-            afr[s][2] = ld_state(Sw + g * DK + 8 * s + t + 4);
-            afr[s][3] = ld_state(Sw + (g + 8) * DK + 8 * s + t + 4);
+    // The block's base rows, fetched first (they land while the log is staged).
+    {
+        constexpr int CPR = DK / TL::CE;  // chunks per row
+        const ST *src = S + (shead * DV + row0) * DK;
+#pragma unroll 4
+        for (int u = tid; u < ROWS * CPR; u += nthr) {
+            const int r = u / CPR, ch = u % CPR;
+            cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
         }
-    };
+        cp_async_commit();
+    }
+
     if constexpr (WITH_CUR) {
         if (bf) stage_block(sq, DK, static_cast<const bf16 *>(q) + head * DK, DK, 1, DK, tid, nthr);
         else stage_block(sq, DK, static_cast<const float *>(q) + head * DK, DK, 1, DK, tid, nthr);
@@ -214,8 +259,9 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             float bsc = 0.f, asc = 1.f;
             (void)asc;
             if (tid < nb) {
-                bsc = tid < nl ? to_f(static_cast<const IT *>(log_b)[lrow + b0 + tid])
-                               : to_f(static_cast<const IT *>(beta)[head]);
+                if constexpr (DELTA)
+                    bsc = tid < nl ? to_f(static_cast<const IT *>(log_b)[lrow + b0 + tid])
+                                   : to_f(static_cast<const IT *>(beta)[head]);
                 if constexpr (!CHAN)
                     asc = tid < nl ? to_f(static_cast<const IT *>(log_a)[lrow + b0 + tid])
                                    : to_f(static_cast<const IT *>(a)[head]);
@@ -227,27 +273,27 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 #pragma unroll
             for (int u = 0; u < CN; ++u) {
                 const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
-                cval[u] = (idx < NB * NB && cj <= ci && ci < nl) ? log_x[(lrow + b0 + ci) * L + b0 + cj] : 0.f;
+                cval[u] = (DELTA && idx < NB * NB && cj <= ci && ci < nl) ? log_x[(lrow + b0 + ci) * L + b0 + cj]
+                                                                            : 0.f;
             }
+            auto put = [](float *dst, const float *x, bool real, float pad) {
+#pragma unroll
+                for (int e = 0; e < E; e += 4)
+                    *reinterpret_cast<float4 *>(dst + e) =
+                        real ? make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]) : make_float4(pad, pad, pad, pad);
+            };
 #pragma unroll
             for (int u = 0; u < KN; ++u) {
                 const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
-                if (c < NB * KC) {
-                    const bool real = r < nb;  // padded entries: k = 0, a = 1
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        fk[r * DK + col + e] = real ? kx[u][e] : 0.f;
-                        if constexpr (CHAN) fa[r * DK + col + e] = real ? ax[u][e] : 1.f;
-                    }
+                if (c < NB * KC) {  // padded entries: k = 0, a = 1
+                    put(kh + r * C::KH + col, kx[u], r < nb, 0.f);
+                    if constexpr (CHAN) put(ff + r * C::WS + col, ax[u], r < nb, 1.f);
                 }
             }
 #pragma unroll
             for (int u = 0; u < VN; ++u) {
                 const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
-                if (c < NB * VC) {
-#pragma unroll
-                    for (int e = 0; e < E; ++e) sv[r * ROWS + col + e] = r < nb ? vx[u][e] : 0.f;
-                }
+                if (c < NB * VC) put(sv + r * C::VS + col, vx[u], r < nb, 0.f);
             }
             if (tid < NB) {
                 sb[tid] = bsc;  // 0 for padded entries
@@ -255,43 +301,49 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             }
 #pragma unroll
             for (int u = 0; u < CN; ++u) {
-                const int idx = tid + u * nthr, ci = idx / NB;
-                if (idx < NB * NB && !(cur_here && ci == nl)) sx[idx] = cval[u];
+                const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
+                if (idx < NB * NB && !(cur_here && ci == nl)) sx[ci * C::XS + cj] = cval[u];
             }
         };
         if (bf) stage(bf16{});
         else stage(float{});
         __syncthreads();
 
-        // 2. per key channel: Khat_i = gamma_i o k_i, gamma, F_j = k_j o D(nb-1, j).
+        // 2. per key channel, in place: Khat_i = gamma_i o k_i, gamma,
+        // F_j = k_j o D(NB-1, j) (padded entries have a = 1, so D(NB-1, j) = D(nb-1, j)).
         for (int c = tid; c < DK; c += nthr) {
-            float ac[NB];
+            float ac[NB], kc[NB];
 #pragma unroll
-            for (int i = 0; i < NB; ++i) ac[i] = CHAN ? fa[i * DK + c] : fa[i];
+            for (int i = 0; i < NB; ++i) {
+                ac[i] = CHAN ? ff[i * C::WS + c] : fa[i];
+                kc[i] = kh[i * C::KH + c];
+            }
             float gm = 1.f;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 gm *= ac[i];
-                kh[i * C::KH + c] = gm * fk[i * DK + c];
+                kh[i * C::KH + c] = gm * kc[i];
             }
             gn[c] = gm;
             float f = 1.f;
 #pragma unroll
             for (int j = NB - 1; j >= 0; --j) {
-                ff[j * DK + c] = fk[j * DK + c] * f;
+                ff[j * C::WS + c] = kc[j] * f;
                 f *= ac[j];
             }
         }
+        cp_async_wait_all();  // this thread's share of the base tile has landed
         __syncthreads();
-        // The fused read's current entry is the block's last real one, so
-        // D(nl, j) is F_j's suffix product: C(nl, j) = k_nl . F_j.
-        if (cur_here) {
+        // The fused read's current entry is the block's last real one: F_nl = k_nl
+        // exactly (every later factor is a padded 1) and D(nl, j) is F_j's suffix
+        // product, so C(nl, j) = F_nl . F_j.
+        if (DELTA && cur_here) {
             for (int j = warp; j < nl; j += nthr / 32) {
                 float pj = 0.f;
 #pragma unroll
                 for (int e = 0; e < C::CW; ++e) {
                     const int c = e * 32 + lane;
-                    pj = fmaf(fk[nl * DK + c], ff[j * DK + c], pj);
+                    pj = fmaf(ff[nl * C::WS + c], ff[j * C::WS + c], pj);
                 }
                 pj = group_sum<32>(pj);
                 if (lane == 0) cm[j] = pj;
@@ -301,77 +353,87 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             if (tid < NB) {
                 const int j = tid;
                 float acc = 0.f;
-                for (int m = j; m < nl; ++m) acc = fmaf(cm[m], sx[m * NB + j], acc);
-                sx[nl * NB + j] = j < nl ? -sb[nl] * acc : (j == nl ? sb[nl] : 0.f);
+                for (int m = j; m < nl; ++m) acc = fmaf(cm[m], sx[m * C::XS + j], acc);
+                sx[nl * C::XS + j] = j < nl ? -sb[nl] * acc : (j == nl ? sb[nl] : 0.f);
             }
             __syncthreads();
         }
 
-        // 3. W = X^T F: W[j][c] = sum_{i>=j} X(i, j) F[i][c].
-        for (int u = tid; u < NB * DK; u += nthr) {
-            const int j = u / DK, c = u % DK;
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < NB; ++i) acc = fmaf(sx[i * NB + j], ff[i * DK + c], acc);
-            sw[j * C::WS + c] = acc;
-        }
-        __syncthreads();
-
-        // 4. this warp's 16 rows. G = S Khat^T.
+        // 3. this warp's 16 rows: delta in the A-operand layout (split hi + lo).
         __syncwarp();  // a previous block's rows, written by this warp, are visible
-        load_afr();
-        float acc1[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) acc1[nt][x] = 0.f;
-#pragma unroll
-        for (int s = 0; s < KS; ++s) {
-            uint32_t ah[4], al[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) split_tf32(afr[s][x], ah[x], al[x]);
+        const int rg = 16 * warp + g;
+        uint32_t xh[NT][4], xl[NT][4];
+        if constexpr (!DELTA) {
+            // delta = V, read straight into the operand layout (entries 8nt + t, + 4).
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float *kp = kh + (8 * nt + g) * C::KH + 8 * s + t;
-                mma3(acc1[nt], ah, al, kp[0], kp[4]);
+                const int i0 = 8 * nt + t;
+                split_tf32(sv[i0 * C::VS + rg], xh[nt][0], xl[nt][0]);
+                split_tf32(sv[i0 * C::VS + rg + 8], xh[nt][1], xl[nt][1]);
+                split_tf32(sv[(i0 + 4) * C::VS + rg], xh[nt][2], xl[nt][2]);
+                split_tf32(sv[(i0 + 4) * C::VS + rg + 8], xh[nt][3], xl[nt][3]);
             }
-        }
-        // E = V - G (accumulator layout: rows g, g + 8; entries 8nt + 2t, 8nt + 2t + 1),
-        // then moved to operand layout (entries 8nt + t, 8nt + t + 4) within each quad.
-        const int rg = 16 * warp + g;
-        uint32_t eh[NT][4], el[NT][4];
+        } else {
+            // G = S Khat^T, the A fragments from the base tile: a0 = S[g][8s + t],
+            // a1 = S[g + 8][8s + t], a2 = S[g][8s + t + 4], a3 = S[g + 8][8s + t + 4].
+            float acc1[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int i0 = 8 * nt + 2 * t;
-            const float e0 = sv[i0 * ROWS + rg] - acc1[nt][0];
-            const float e1 = sv[(i0 + 1) * ROWS + rg] - acc1[nt][1];
-            const float e2 = sv[i0 * ROWS + rg + 8] - acc1[nt][2];
-            const float e3 = sv[(i0 + 1) * ROWS + rg + 8] - acc1[nt][3];
-            const int s0 = (lane & ~3) | (t >> 1), s1 = s0 + 2;  // quad lanes holding entries t, t + 4
-            const float x00 = __shfl_sync(0xffffffffu, e0, s0), x01 = __shfl_sync(0xffffffffu, e1, s0);
-            const float x10 = __shfl_sync(0xffffffffu, e2, s0), x11 = __shfl_sync(0xffffffffu, e3, s0);
-            const float y00 = __shfl_sync(0xffffffffu, e0, s1), y01 = __shfl_sync(0xffffffffu, e1, s1);
-            const float y10 = __shfl_sync(0xffffffffu, e2, s1), y11 = __shfl_sync(0xffffffffu, e3, s1);
-            const bool odd = t & 1;
-            split_tf32(odd ? x01 : x00, eh[nt][0], el[nt][0]);  // E[g][8nt + t]
-            split_tf32(odd ? x11 : x10, eh[nt][1], el[nt][1]);  // E[g + 8][8nt + t]
-            split_tf32(odd ? y01 : y00, eh[nt][2], el[nt][2]);  // E[g][8nt + t + 4]
-            split_tf32(odd ? y11 : y10, eh[nt][3], el[nt][3]);  // E[g + 8][8nt + t + 4]
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) acc1[nt][x] = 0.f;
+#pragma unroll
+            for (int s = 0; s < KS; ++s) {
+                uint32_t ah[4], al[4];
+                split_tf32(ld_state(tile + TL::off(tr + g, 8 * s + t)), ah[0], al[0]);
+                split_tf32(ld_state(tile + TL::off(tr + g + 8, 8 * s + t)), ah[1], al[1]);
+                split_tf32(ld_state(tile + TL::off(tr + g, 8 * s + t + 4)), ah[2], al[2]);
+                split_tf32(ld_state(tile + TL::off(tr + g + 8, 8 * s + t + 4)), ah[3], al[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float *kp = kh + (8 * nt + g) * C::KH + 8 * s + t;
+                    mma3(acc1[nt], ah, al, kp[0], kp[4]);
+                }
+            }
+            // E = V - G in the accumulator layout (rows g, g + 8; entries 8nt + 2t, +1).
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int i0 = 8 * nt + 2 * t;
+                acc1[nt][0] = sv[i0 * C::VS + rg] - acc1[nt][0];
+                acc1[nt][1] = sv[(i0 + 1) * C::VS + rg] - acc1[nt][1];
+                acc1[nt][2] = sv[i0 * C::VS + rg + 8] - acc1[nt][2];
+                acc1[nt][3] = sv[(i0 + 1) * C::VS + rg + 8] - acc1[nt][3];
+            }
+            // delta = E X^T (the triangular solve, one small product per warp; X is
+            // lower triangular, so tiles above the diagonal are skipped).
+            acc_to_operand<NT>(acc1, xh, xl, lane);
+            float dl[NT][4];
+#pragma unroll
+            for (int mt = 0; mt < NT; ++mt) {
+#pragma unroll
+                for (int x = 0; x < 4; ++x) dl[mt][x] = 0.f;
+#pragma unroll
+                for (int kt = 0; kt <= mt; ++kt) {
+                    const float *xp = sx + (8 * mt + g) * C::XS + 8 * kt + t;
+                    mma3(dl[mt], xh[kt], xl[kt], xp[0], xp[4]);
+                }
+            }
+            acc_to_operand<NT>(dl, xh, xl, lane);
         }
-        // S <- S o gamma + E W, one 16 x 8 column tile at a time, written straight
-        // from the accumulator layout (rows g, g + 8; columns 8c + 2t, 8c + 2t + 1).
+        // S <- S o gamma + delta F, one 16 x 8 column tile at a time (rows g, g + 8;
+        // columns 8c + 2t, 8c + 2t + 1 of the accumulator layout): from the tile,
+        // back to the tile for a following sub-merge, else straight to HBM.
 #pragma unroll 4
         for (int cb = 0; cb < KS; ++cb) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float *wp = sw + (8 * nt + t) * C::WS + 8 * cb + g;
-                mma3(d, eh[nt], el[nt], wp[0], wp[4 * C::WS]);
+                const float *fp = ff + (8 * nt + t) * C::WS + 8 * cb + g;
+                mma3(d, xh[nt], xl[nt], fp[0], fp[4 * C::WS]);
             }
             const int col = 8 * cb + 2 * t;
-            float s00, s01, s10, s11;
-            ld_state2(Sw + g * DK + col, s00, s01);
-            ld_state2(Sw + (g + 8) * DK + col, s10, s11);
+            ST *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
+            const float2 r0 = ld_tile2(p0), r1 = ld_tile2(p1);
+            float s00 = r0.x, s01 = r0.y, s10 = r1.x, s11 = r1.y;
             const float2 gv = *reinterpret_cast<const float2 *>(gn + col);
             s00 = fmaf(s00, gv.x, d[0]);
             s01 = fmaf(s01, gv.y, d[1]);
@@ -382,8 +444,13 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 oacc[0] = fmaf(s00, qv.x, fmaf(s01, qv.y, oacc[0]));
                 oacc[1] = fmaf(s10, qv.x, fmaf(s11, qv.y, oacc[1]));
             }
-            st_state2(Sw + g * DK + col, s00, s01);
-            st_state2(Sw + (g + 8) * DK + col, s10, s11);
+            if (last) {
+                st_state2(Sw + g * DK + col, s00, s01);
+                st_state2(Sw + (g + 8) * DK + col, s10, s11);
+            } else {
+                st_tile2(p0, s00, s01);
+                st_tile2(p1, s10, s11);
+            }
         }
         __syncthreads();  // the next entry block reuses the shared buffers
     }
@@ -400,15 +467,16 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 
 // ------------------------------------------------------------------ launch
 
-template <class ST, int DK, bool CHAN, bool WC, int NB>
-static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
-    using C = MergeShape<DK>;
-    auto kern = merge_kernel<ST, DK, CHAN, WC, NB>;
-    const int rows = C::rows(p.dv);
-    const size_t smem = merge_smem_bytes<DK, CHAN, NB>(rows);
+template <class ST, int DK, int KD, bool WC, int NB>
+static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st,
+                                  const PoolIdx &pool, int part) {
+    using C = MergeShape<DK, NB>;
+    auto kern = merge_kernel<ST, DK, KD, WC, NB>;
+    constexpr int rows = C::ROWS;
+    const size_t smem = merge_smem_bytes<ST, DK, NB>();
     static bool configured = false;
     if (!configured) {
-        const size_t want = merge_smem_bytes<DK, CHAN, NB>(rows);
+        const size_t want = smem;
         if (want > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
             if (e != cudaSuccess) return e;
@@ -418,31 +486,36 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
     const long long blocks = (long long)p.B * p.H * (p.dv / rows);
     kern<<<(unsigned)blocks, rows * 2, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.x, lg.L,
                                                    n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
-                                                   p.in_dt == DL_BF16);
+                                                   p.in_dt == DL_BF16, pool, part);
     return cudaGetLastError();
 }
 
 // Entry-block size: 8 when all entries fit, else 16 (a longer log runs as a
-// chain of 16-entry sub-merges, the last one padded).
-template <class ST, int DK, bool CHAN, bool WC>
-static cudaError_t launch_merge_nb(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
-    const int nt = n_log + (WC ? 1 : 0);
-    if (nt <= 8) return launch_merge_t<ST, DK, CHAN, WC, 8>(p, lg, n_log, st);
-    return launch_merge_t<ST, DK, CHAN, WC, 16>(p, lg, n_log, st);
+// chain of 16-entry sub-merges, the last one padded). A pool launch sizes it
+// for the largest count a slot can hold.
+template <class ST, int DK, int KD, bool WC>
+static cudaError_t launch_merge_nb(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st,
+                                   const PoolIdx &pool, int part) {
+    const int nt = (pool.slot ? lg.L - 1 : n_log) + (WC ? 1 : 0);
+    if (nt <= 8) return launch_merge_t<ST, DK, KD, WC, 8>(p, lg, n_log, st, pool, part);
+    return launch_merge_t<ST, DK, KD, WC, 16>(p, lg, n_log, st, pool, part);
 }
 
-cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st) {
+cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st,
+                         const PoolIdx &pool, int part) {
     // The input dtype and d_v are run-time arguments of the merge kernel (they
     // only change staging and the grid), which keeps instantiations few.
     auto go = [&](auto st_t, auto dk_c) -> cudaError_t {
         using ST = decltype(st_t);
         constexpr int DK = decltype(dk_c)::value;
-        if (p.chan) {
-            if (with_cur) return launch_merge_nb<ST, DK, true, true>(p, lg, n_log, st);
-            return launch_merge_nb<ST, DK, true, false>(p, lg, n_log, st);
-        }
-        if (with_cur) return launch_merge_nb<ST, DK, false, true>(p, lg, n_log, st);
-        return launch_merge_nb<ST, DK, false, false>(p, lg, n_log, st);
+        auto with_kind = [&](auto kd_c) -> cudaError_t {
+            constexpr int KD = decltype(kd_c)::value;
+            if (with_cur) return launch_merge_nb<ST, DK, KD, true>(p, lg, n_log, st, pool, part);
+            return launch_merge_nb<ST, DK, KD, false>(p, lg, n_log, st, pool, part);
+        };
+        if (p.kind == DL_RWKV6) return with_kind(std::integral_constant<int, DL_RWKV6>{});
+        if (p.kind == DL_DECAY_CHANNEL) return with_kind(std::integral_constant<int, DL_DECAY_CHANNEL>{});
+        return with_kind(std::integral_constant<int, DL_DECAY_HEAD>{});
     };
     auto with_dk = [&](auto st_t) -> cudaError_t {
         if (p.dk == 64) return go(st_t, std::integral_constant<int, 64>{});
@@ -450,6 +523,26 @@ cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bo
     };
     if (p.s_dt == DL_BF16) return with_dk(bf16{});
     return with_dk(float{});
+}
+
+// ------------------------------------------------------------------ pool counts
+
+// After a pool step every listed slot holds one more entry, or none if this
+// step was its L-th (merged); after a flush it holds none.
+__global__ void pool_counts_kernel(const int *__restrict__ slot, int *__restrict__ counts, int B, int P, int L,
+                                   bool advance) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    const int s = slot[b];
+    if (s < 0 || s >= P) return;  // flagged by the step's kernels
+    const int c = counts[s];
+    if (c < 0 || c >= L) return;
+    counts[s] = (advance && c < L - 1) ? c + 1 : 0;
+}
+
+cudaError_t launch_pool_counts(const PoolIdx &pool, int B, bool advance, cudaStream_t st) {
+    pool_counts_kernel<<<(B + 127) / 128, 128, 0, st>>>(pool.slot, pool.counts, B, pool.P, pool.L, advance);
+    return cudaGetLastError();
 }
 
 }  // namespace dl

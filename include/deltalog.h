@@ -11,7 +11,14 @@
  *     o_t = S_t q_t,
  *
  * where the decay is one scalar per head for Gated DeltaNet (GDN) and one
- * value per key channel for Kimi Delta Attention (KDA).
+ * value per key channel for Kimi Delta Attention (KDA). The third model of
+ * the page's operator list, RWKV6 (per-key decay, raw-value update with no
+ * delta-rule correction, "Kernel Implementation"), is
+ *
+ *     S_t = S_{t-1} Diag(a_t) + v_t k_t^T,    o_t = S_t q_t
+ *
+ * (beta is not used; RWKV6's per-channel "bonus" on the current token is not
+ * defined on the page and is not computed).
  *
  * Two schedules:
  *   eager     -- dl_gdn_decode_step / dl_kda_decode_step read S, apply the
@@ -55,7 +62,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 4
+#define DL_ABI_VERSION 6
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -68,9 +75,12 @@ typedef enum {
 
 typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
 
+/* The model's update rule: its decay shape and whether the delta-rule
+ * correction applies. */
 typedef enum {
     DL_DECAY_HEAD = 0,    /* a is one scalar per (b, h, step): GDN */
-    DL_DECAY_CHANNEL = 1  /* a is one value per key channel: KDA  */
+    DL_DECAY_CHANNEL = 1, /* a is one value per key channel: KDA  */
+    DL_RWKV6 = 2          /* a per key channel, raw-value update, no beta: RWKV6 */
 } dl_decay;
 
 /* Caller-owned bounded log of a deferred state: per (b, h) up to L entries of
@@ -78,12 +88,13 @@ typedef enum {
  * log-decay metadata, and a small fp32 workspace the deferred read uses to
  * hand its per-head key-side results to the value tiles.
  * (The page's log keeps "compact update factors" plus log-decay metadata,
- * Technical Summary, "Core Mechanism: Base + Log"; here the metadata is
- * recomputed from the stored decays where it is needed.)
+ * Technical Summary, "Core Mechanism: Base + Log"; here the decay products
+ * are recomputed from the stored decays where they are needed, and the
+ * triangular solve they lead to is kept as x below.)
  *   k     [B, H, L, d_k]
  *   v     [B, H, L, d_v]
  *   beta  [B, H, L]
- *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL)
+ *   a     [B, H, L] (DL_DECAY_HEAD) or [B, H, L, d_k] (DL_DECAY_CHANNEL, DL_RWKV6)
  *   x     [B, H, L, L] float: the log's metadata, row j holding X(j, e) for
  *         e <= j, where X = (I + Diag(beta) C)^{-1} Diag(beta) and
  *         C(j, e) = sum_c k_e[c] k_j[c] prod_{m=e+1..j} a_m[c] for e < j (the
@@ -93,6 +104,8 @@ typedef enum {
  *         append, so dl_log_append_read writes row n for the entry it appends;
  *         the deferred read and the merge read it. Log entries must therefore
  *         be written by dl_log_append_read. 16-byte aligned.
+ *         DL_RWKV6 has no correction (X is the identity): beta and x are not
+ *         used and may be null.
  *   work  at least dl_log_work_bytes(B, H, d_k, d_v) bytes, 16-byte aligned,
  *         contents irrelevant between calls (only dl_log_append_read uses it)
  * The number of valid entries n (the same for every head) is tracked by the
@@ -129,6 +142,15 @@ dl_status dl_kda_decode_step(void *S, dl_dtype s_dtype,
                              float *o, int B, int H, int d_k, int d_v,
                              cudaStream_t stream);
 
+/* Eager RWKV6 step (channel-wise decay, raw-value update), in place:
+ *   S_t = S_{t-1} Diag(a) + v k^T,  o = S_t q.
+ * Arguments as dl_kda_decode_step without beta. */
+dl_status dl_rwkv6_decode_step(void *S, dl_dtype s_dtype,
+                               const void *q, const void *k, const void *v,
+                               const void *a, dl_dtype in_dtype,
+                               float *o, int B, int H, int d_k, int d_v,
+                               cudaStream_t stream);
+
 /* Bytes of log workspace (dl_log.work) the deferred read needs:
  * B * H * (d_k + d_v) * 4. */
 size_t dl_log_work_bytes(int B, int H, int d_k, int d_v);
@@ -142,7 +164,8 @@ size_t dl_log_work_bytes(int B, int H, int d_k, int d_v);
  *   log    entries 0..n-1 read, entry n written; log->work is overwritten
  *          (missing or smaller than dl_log_work_bytes -> DL_ERR_INVALID_ARG)
  *   n      entries already in the log, 0 <= n < L; n >= L -> DL_ERR_LOG_FULL
- *   q, k, v, beta, a, o: as the eager step of the same decay kind. */
+ *   q, k, v, beta, a, o: as the eager step of the same kind (DL_RWKV6: beta
+ *          is not used and may be null). */
 dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind,
                              const dl_log *log, int n,
                              const void *q, const void *k, const void *v,
@@ -199,6 +222,56 @@ dl_status dl_log_append_read_noalloc(const void *S_base, dl_dtype s_dtype, dl_de
                                      const void *beta, const void *a, dl_dtype in_dtype,
                                      float *o, int B, int H, int d_k, int d_v,
                                      cudaStream_t stream);
+
+/* A pool of per-sequence deferred states for continuous batching: the
+ * sequences of a decode batch own slots of a preallocated pool, and each slot
+ * keeps its own log fill (the page's per-"slot-head" state, Technical
+ * Summary, "Kernel Implementation"; its vLLM-based serving stack, "System
+ * Implementation and Evaluation").
+ *   S       [P, H, d_v, d_k] s_dtype: the base of every slot
+ *   P       slots, >= 1
+ *   n       [P] int32, device: the log entries each slot holds, 0 <= n[s] < L.
+ *           dl_pool_step and dl_pool_flush update it. When a new sequence
+ *           takes slot s, the caller writes its initial state into S[s] and
+ *           sets n[s] = 0.
+ *   status  optional (may be null) int32, device: a step or flush ORs in 1
+ *           when a batch row's slot is outside [0, P) or that slot's count
+ *           outside [0, L); such a row is skipped (o not written).
+ *   log     the slots' logs: k [P, H, L, d_k], v [P, H, L, d_v], beta [P, H, L],
+ *           a [P, H, L] or [P, H, L, d_k], x [P, H, L, L] (as dl_log with B = P);
+ *           log.work must hold dl_log_work_bytes(B, H, d_k, d_v) for the batch.
+ * Alignment and aliasing rules as for the other entry points; n, status and
+ * slot need 4-byte alignment. */
+typedef struct {
+    void *S;
+    dl_dtype s_dtype;
+    int P;
+    int *n;
+    int *status;
+    dl_log log;
+} dl_pool;
+
+/* One decode step of B sequences of a pool. Batch row b works on slot slot[b]
+ * (int32 [B], device; the slots of one call must be distinct). With
+ * c = n[slot[b]] before the call:
+ *   c < L - 1   append this step's factors as the slot's entry c and read
+ *               o = S_c q from base + log (dl_log_append_read); n <- c + 1
+ *   c = L - 1   merge the slot's c entries and this step into its base and
+ *               read o from the new base (dl_log_merge_read); n <- 0
+ * so every sequence follows its own deferred schedule whatever the fills of
+ * the others. q, k, v, beta, a and o are batch tensors [B, H, ...] as for
+ * dl_log_append_read; B <= P. */
+dl_status dl_pool_step(const dl_pool *pool, dl_decay kind, const int *slot,
+                       const void *q, const void *k, const void *v,
+                       const void *beta, const void *a, dl_dtype in_dtype,
+                       float *o, int B, int H, int d_k, int d_v,
+                       cudaStream_t stream);
+
+/* Merge the log of every listed slot into its base (slots holding n[s] > 0
+ * entries) and set n[s] = 0: afterwards S[slot[b]] is the dense state of
+ * that sequence (for a sequence that ends, or a state handed elsewhere). */
+dl_status dl_pool_flush(const dl_pool *pool, dl_decay kind, const int *slot,
+                        int B, int H, int d_k, int d_v, cudaStream_t stream);
 
 /* Static text for a status code. */
 const char *dl_status_string(dl_status s);

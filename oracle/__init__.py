@@ -10,7 +10,9 @@ States for Linear Attention Decoding", Technical Summary):
   * ``eager``       -- the recurrence step by step (C, deltalog_oracle.c);
   * ``deferred``    -- base + bounded log with merges every L steps (C);
   * ``brute_force`` -- dense d_k x d_k factor matrices multiplied with numpy,
-                       for tiny shapes only.
+                       for tiny shapes only;
+  * ``pool_eager``  -- a pool of per-sequence states, each listed slot
+                       advanced one eager step (the slot-pool entry points).
 
 Definition used (the pages describe the update only in words -- decay, then a
 delta-rule correction that subtracts the current read before writing, with a
@@ -19,6 +21,11 @@ Attention, "Kernel Implementation"): per head, S is d_v x d_k and
 
     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
     o_t = S_t q_t.
+
+RWKV6 (``rwkv6=True``), the page's third model ("per-key decay; raw-value
+updates, no delta-rule correction", "Kernel Implementation"), is read as
+S_t = S_{t-1} Diag(a_t) + v_t k_t^T, o_t = S_t q_t: no beta, and no "bonus"
+term (the pages do not define one).
 
 Every function's parity with the pages is pinned by tests/test_oracle_pins.py
 (invariants, closed forms, hand-worked exact examples, brute force).
@@ -68,25 +75,31 @@ class CLib:
         self.lib = lib
         self.path = path
 
-    def eager(self, S0, q, k, v, beta, a, channel_decay: bool):
+    def eager(self, S0, q, k, v, beta, a, channel_decay: bool, rwkv6: bool = False):
         """Eager recurrence over T steps. Shapes: S0 [NH,d_v,d_k]; q,k [T,NH,d_k];
-        v [T,NH,d_v]; beta [T,NH]; a [T,NH] or [T,NH,d_k]. Returns (o [T,NH,d_v], S_T)."""
-        S, q, k, v, beta, a, NH, T, dk, dv = _prep(S0, q, k, v, beta, a, channel_decay)
+        v [T,NH,d_v]; beta [T,NH] (unused, may be None, for RWKV6); a [T,NH] or
+        [T,NH,d_k]. Returns (o [T,NH,d_v], S_T)."""
+        S, q, k, v, beta, a, NH, T, dk, dv = _prep(S0, q, k, v, beta, a, channel_decay or rwkv6)
         o = np.zeros((T, NH, dv), dtype=np.float64)
-        self.lib.oracle_eager(NH, T, dk, dv, int(bool(channel_decay)),
+        self.lib.oracle_eager(NH, T, dk, dv, _kind(channel_decay, rwkv6),
                               _c(S), _c(q), _c(k), _c(v), _c(beta), _c(a), _c(o))
         return o, S
 
-    def deferred(self, S0, q, k, v, beta, a, channel_decay: bool, L: int):
+    def deferred(self, S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False):
         """DeltaLog schedule with log capacity L (merge when full and at the end).
         Returns (o [T,NH,d_v], S_T)."""
         if L < 1:
             raise ValueError("log capacity L must be >= 1")
-        S, q, k, v, beta, a, NH, T, dk, dv = _prep(S0, q, k, v, beta, a, channel_decay)
+        S, q, k, v, beta, a, NH, T, dk, dv = _prep(S0, q, k, v, beta, a, channel_decay or rwkv6)
         o = np.zeros((T, NH, dv), dtype=np.float64)
-        self.lib.oracle_deferred(NH, T, dk, dv, int(bool(channel_decay)), int(L),
+        self.lib.oracle_deferred(NH, T, dk, dv, _kind(channel_decay, rwkv6), int(L),
                                  _c(S), _c(q), _c(k), _c(v), _c(beta), _c(a), _c(o))
         return o, S
+
+
+def _kind(channel_decay: bool, rwkv6: bool) -> int:
+    """The C oracle's rule code: 0 head-wise decay, 1 channel-wise, 2 RWKV6."""
+    return 2 if rwkv6 else int(bool(channel_decay))
 
 
 def _load() -> CLib:
@@ -106,6 +119,8 @@ def _prep(S0, q, k, v, beta, a, channel_decay):
     q = np.ascontiguousarray(q, dtype=np.float64)
     k = np.ascontiguousarray(k, dtype=np.float64)
     v = np.ascontiguousarray(v, dtype=np.float64)
+    if beta is None:  # RWKV6 has no beta; the C side does not read it
+        beta = np.zeros(q.shape[:2], dtype=np.float64)
     beta = np.ascontiguousarray(beta, dtype=np.float64)
     a = np.ascontiguousarray(a, dtype=np.float64)
     NH, dv, dk = S.shape
@@ -116,20 +131,21 @@ def _prep(S0, q, k, v, beta, a, channel_decay):
     return S, q, k, v, beta, a, NH, T, dk, dv
 
 
-def eager(S0, q, k, v, beta, a, channel_decay: bool):
+def eager(S0, q, k, v, beta, a, channel_decay: bool, rwkv6: bool = False):
     """Eager recurrence (see ``CLib.eager``) with the default build."""
-    return _load().eager(S0, q, k, v, beta, a, channel_decay)
+    return _load().eager(S0, q, k, v, beta, a, channel_decay, rwkv6)
 
 
-def deferred(S0, q, k, v, beta, a, channel_decay: bool, L: int):
+def deferred(S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False):
     """DeltaLog schedule (see ``CLib.deferred``) with the default build."""
-    return _load().deferred(S0, q, k, v, beta, a, channel_decay, L)
+    return _load().deferred(S0, q, k, v, beta, a, channel_decay, L, rwkv6)
 
 
-def brute_force(S0, q, k, v, beta, a, channel_decay: bool):
+def brute_force(S0, q, k, v, beta, a, channel_decay: bool, rwkv6: bool = False):
     """Tiny shapes only: build A_t = Diag(a_t)(I - beta_t k_t k_t^T) as dense
     matrices and apply S_t = S_{t-1} A_t + beta_t v_t k_t^T, o_t = S_t q_t with
-    numpy matrix products. Returns (o [T,NH,d_v], S_T)."""
+    numpy matrix products (RWKV6: A_t = Diag(a_t), S_t = S_{t-1} A_t + v_t k_t^T).
+    Returns (o [T,NH,d_v], S_T)."""
     S = np.array(S0, dtype=np.float64, copy=True)
     NH, dv, dk = S.shape
     T = q.shape[0]
@@ -141,11 +157,43 @@ def brute_force(S0, q, k, v, beta, a, channel_decay: bool):
             kt = np.asarray(k[t, h], dtype=np.float64).reshape(dk, 1)
             vt = np.asarray(v[t, h], dtype=np.float64).reshape(dv, 1)
             at = np.asarray(a[t, h], dtype=np.float64)
-            Da = np.diag(at if channel_decay else np.full(dk, float(at)))
-            A = Da @ (eye - float(beta[t, h]) * (kt @ kt.T))
-            S[h] = S[h] @ A + float(beta[t, h]) * (vt @ kt.T)
+            Da = np.diag(at if (channel_decay or rwkv6) else np.full(dk, float(at)))
+            if rwkv6:
+                S[h] = S[h] @ Da + vt @ kt.T
+            else:
+                A = Da @ (eye - float(beta[t, h]) * (kt @ kt.T))
+                S[h] = S[h] @ A + float(beta[t, h]) * (vt @ kt.T)
             o[t, h] = S[h] @ np.asarray(q[t, h], dtype=np.float64)
     return o, S
+
+
+def pool_eager(S_pool0, steps, channel_decay: bool, rwkv6: bool = False, resets=None):
+    """A pool of per-sequence states advanced by the recurrence, for the slot
+    pool entry points: ``S_pool0`` [P, H, d_v, d_k]; ``steps`` a list of
+    (slot [B], q [B,H,d_k], k, v [B,H,d_v], beta [B,H], a [B,H] or [B,H,d_k]) in
+    which every listed slot takes one eager step with its row's inputs;
+    ``resets`` maps a step index to {slot: new state [H, d_v, d_k]} applied
+    before that step (a new sequence taking the slot). Returns (list of o
+    [B,H,d_v] per step, final S_pool)."""
+    S = np.array(S_pool0, dtype=np.float64, copy=True)
+    P, H, dv, dk = S.shape
+    flat = S.reshape(P * H, dv, dk)
+    outs = []
+    for t, (slot, q, k, v, beta, a) in enumerate(steps):
+        for s_, S0 in (resets or {}).get(t, {}).items():
+            flat[s_ * H:(s_ + 1) * H] = np.asarray(S0, dtype=np.float64)
+        slot = np.asarray(slot, dtype=np.int64)
+        B = slot.size
+        heads = (slot[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+        chan = channel_decay or rwkv6
+        a_ = np.asarray(a, np.float64).reshape((1, B * H, dk) if chan else (1, B * H))
+        beta_ = None if beta is None else np.asarray(beta, np.float64).reshape(1, B * H)
+        o, Snew = eager(flat[heads], np.asarray(q, np.float64).reshape(1, B * H, dk),
+                        np.asarray(k, np.float64).reshape(1, B * H, dk), np.asarray(v, np.float64).reshape(1, B * H, dv),
+                        beta_, a_, channel_decay, rwkv6)
+        flat[heads] = Snew
+        outs.append(o[0].reshape(B, H, dv))
+    return outs, flat.reshape(P, H, dv, dk)
 
 
 def brute_force_window(Sbar, ks, vs, betas, As_diag):
@@ -179,10 +227,11 @@ def run_workload_heads(w, inputs: Dict[str, np.ndarray], path: str = "eager", L:
     import workloads  # the shared seeded-input module, no method arithmetic
 
     f = workloads.as_f64(w, inputs)
-    chan = w.decay == workloads.CHANNEL
+    chan = w.decay != workloads.HEAD
+    rw = w.decay == workloads.RWKV6
     if path == "eager":
-        return eager(f["S0"], f["q"], f["k"], f["v"], f["beta"], f["a"], chan)
-    return deferred(f["S0"], f["q"], f["k"], f["v"], f["beta"], f["a"], chan, int(L))
+        return eager(f["S0"], f["q"], f["k"], f["v"], f["beta"], f["a"], chan, rw)
+    return deferred(f["S0"], f["q"], f["k"], f["v"], f["beta"], f["a"], chan, int(L), rw)
 
 
 def omp_threads() -> int:

@@ -20,6 +20,15 @@
  *   i.e. decay, then the delta-rule correction that subtracts the current
  *   read S k before writing the new value v.
  *
+ *   RWKV6, the page's third model (per-key decay, "raw-value updates" with
+ *   no delta-rule correction, "Kernel Implementation"), is read as
+ *
+ *       S_t = S_{t-1} Diag(a_t) + v_t k_t^T,    o_t = S_t q_t
+ *
+ *   (no beta; RWKV6's "bonus" term is not given by the pages and is left out).
+ *   `kind` selects the rule: 0 head-wise decay (GDN), 1 channel-wise decay
+ *   (KDA), 2 RWKV6.
+ *
  * Three forms:
  *   oracle_eager     -- the definition, one step at a time (the "eager"
  *                       schedule of section "Problem: The State-Update Tax").
@@ -39,17 +48,18 @@
  *   q, k  [T, NH, d_k]
  *   v     [T, NH, d_v]
  *   beta  [T, NH]
- *   a     [T, NH]  (head-wise decay)  or  [T, NH, d_k]  (channel-wise decay)
+ *   a     [T, NH]  (head-wise decay)  or  [T, NH, d_k]  (channel-wise decay, RWKV6)
+ *   beta  is not read for RWKV6
  *   o     [T, NH, d_v]             out
  */
 #include <stdlib.h>
 #include <string.h>
 
 /* decay value of channel j at step t for head h */
-static double decay_at(const double *a, int channel_decay, long NH, int dk,
+static double decay_at(const double *a, int kind, long NH, int dk,
                        int t, long h, int j)
 {
-    if (channel_decay)
+    if (kind != 0)
         return a[((long)t * NH + h) * dk + j];
     return a[(long)t * NH + h];
 }
@@ -61,8 +71,9 @@ static double decay_at(const double *a, int channel_decay, long NH, int dk,
  *   2. u_i      = sum_j S'[i][j] k_j                   (S' k)
  *   3. S[i][j]  = S'[i][j] + beta (v_i - u_i) k_j      (S'(I - beta k k^T) + beta v k^T)
  *   4. o_i      = sum_j S[i][j] q_j                    (S_t q), from the updated S
+ * RWKV6 (delta = 0) replaces step 3 by S[i][j] = S'[i][j] + v_i k_j.
  */
-static void eager_head_step(double *S, int dk, int dv,
+static void eager_head_step(double *S, int dk, int dv, int delta,
                             const double *q, const double *k, const double *v,
                             double beta, const double *avec, double *o)
 {
@@ -73,7 +84,7 @@ static void eager_head_step(double *S, int dk, int dv,
         double u = 0.0;
         for (int j = 0; j < dk; ++j)
             u += row[j] * k[j];
-        double coef = beta * (v[i] - u);
+        double coef = delta ? beta * (v[i] - u) : v[i];
         for (int j = 0; j < dk; ++j)
             row[j] = row[j] + coef * k[j];
         double acc = 0.0;
@@ -83,22 +94,23 @@ static void eager_head_step(double *S, int dk, int dv,
     }
 }
 
-void oracle_eager(long NH, int T, int dk, int dv, int channel_decay,
+void oracle_eager(long NH, int T, int dk, int dv, int kind,
                   double *S, const double *q, const double *k, const double *v,
                   const double *beta, const double *a, double *o)
 {
+    const int delta = kind != 2;
 #pragma omp parallel for schedule(dynamic, 1)
     for (long h = 0; h < NH; ++h) {
         double *Sh = S + h * (long)dv * dk;
         double *avec = (double *)malloc(sizeof(double) * (size_t)dk);
         for (int t = 0; t < T; ++t) {
             for (int j = 0; j < dk; ++j)
-                avec[j] = decay_at(a, channel_decay, NH, dk, t, h, j);
-            eager_head_step(Sh, dk, dv,
+                avec[j] = decay_at(a, kind, NH, dk, t, h, j);
+            eager_head_step(Sh, dk, dv, delta,
                             q + ((long)t * NH + h) * dk,
                             k + ((long)t * NH + h) * dk,
                             v + ((long)t * NH + h) * dv,
-                            beta[(long)t * NH + h], avec,
+                            delta ? beta[(long)t * NH + h] : 0.0, avec,
                             o + ((long)t * NH + h) * dv);
         }
         free(avec);
@@ -111,6 +123,7 @@ void oracle_eager(long NH, int T, int dk, int dv, int channel_decay,
  * the decay always held as a d_k vector (a head-wise decay is repeated). */
 typedef struct {
     int cap, n, dk, dv;
+    int delta;    /* 1: delta rule (GDN, KDA); 0: RWKV6 */
     double *k;    /* [cap, dk] */
     double *v;    /* [cap, dv] */
     double *beta; /* [cap]     */
@@ -125,6 +138,8 @@ typedef struct {
  * so  o = S_bar x_0 + sum_i s_i v_i  where x_n = q and, for i = n..1,
  *   c_i = k_i . x_i,  s_i = beta_i c_i,  x_{i-1} = A_i x_i = a_i o (x_i - s_i k_i).
  * (A product of Householder-like factors applied to q from the right end.)
+ * RWKV6 has A_i = Diag(a_i) and adds v_i k_i^T unscaled: s_i = c_i and
+ * x_{i-1} = a_i o x_i.
  */
 static void deferred_read(const double *Sbar, const head_log *lg,
                           const double *q, double *o, double *x, double *s)
@@ -138,9 +153,15 @@ static void deferred_read(const double *Sbar, const head_log *lg,
         double c = 0.0;
         for (int j = 0; j < dk; ++j)
             c += ki[j] * x[j];
-        s[i] = lg->beta[i] * c;
-        for (int j = 0; j < dk; ++j)
-            x[j] = ai[j] * (x[j] - s[i] * ki[j]);
+        if (lg->delta) {
+            s[i] = lg->beta[i] * c;
+            for (int j = 0; j < dk; ++j)
+                x[j] = ai[j] * (x[j] - s[i] * ki[j]);
+        } else {
+            s[i] = c;
+            for (int j = 0; j < dk; ++j)
+                x[j] = ai[j] * x[j];
+        }
     }
     for (int r = 0; r < dv; ++r) {
         const double *row = Sbar + (long)r * dk;
@@ -166,6 +187,7 @@ static void deferred_read(const double *Sbar, const head_log *lg,
  *   G_i = s_bar . (gamma_i o k_i),  C(i, j) = sum_c k_j[c] D(i, j)[c] k_i[c],
  *
  * found by forward substitution in i; then s_bar <- s_n. The log empties.
+ * RWKV6 adds each value unscaled and uncorrected: delta_i = v_i[r].
  */
 static void deferred_merge(double *Sbar, head_log *lg)
 {
@@ -204,6 +226,10 @@ static void deferred_merge(double *Sbar, head_log *lg)
     for (int r = 0; r < dv; ++r) {
         double *row = Sbar + (long)r * dk;
         for (int i = 1; i <= n; ++i) {
+            if (!lg->delta) {
+                delta[i] = lg->v[(long)(i - 1) * dv + r];
+                continue;
+            }
             const double *gi = DV(i, 0), *ki = KE(i);
             double G = 0.0;
             for (int c = 0; c < dk; ++c)
@@ -236,7 +262,7 @@ static void deferred_merge(double *Sbar, head_log *lg)
  * as entry n+1 (the base is not written), read o from base + log; when the
  * log holds L entries, merge it into the base and empty it. After the last
  * step any remaining entries are merged, so S returns S_T. */
-void oracle_deferred(long NH, int T, int dk, int dv, int channel_decay, int L,
+void oracle_deferred(long NH, int T, int dk, int dv, int kind, int L,
                      double *S, const double *q, const double *k, const double *v,
                      const double *beta, const double *a, double *o)
 {
@@ -244,7 +270,7 @@ void oracle_deferred(long NH, int T, int dk, int dv, int channel_decay, int L,
     for (long h = 0; h < NH; ++h) {
         double *Sbar = S + h * (long)dv * dk;
         head_log lg;
-        lg.cap = L; lg.n = 0; lg.dk = dk; lg.dv = dv;
+        lg.cap = L; lg.n = 0; lg.dk = dk; lg.dv = dv; lg.delta = kind != 2;
         lg.k = (double *)malloc(sizeof(double) * (size_t)L * dk);
         lg.v = (double *)malloc(sizeof(double) * (size_t)L * dv);
         lg.beta = (double *)malloc(sizeof(double) * (size_t)L);
@@ -255,9 +281,9 @@ void oracle_deferred(long NH, int T, int dk, int dv, int channel_decay, int L,
             int e = lg.n;
             memcpy(lg.k + (long)e * dk, k + ((long)t * NH + h) * dk, sizeof(double) * (size_t)dk);
             memcpy(lg.v + (long)e * dv, v + ((long)t * NH + h) * dv, sizeof(double) * (size_t)dv);
-            lg.beta[e] = beta[(long)t * NH + h];
+            lg.beta[e] = lg.delta ? beta[(long)t * NH + h] : 0.0;
             for (int j = 0; j < dk; ++j)
-                lg.a[(long)e * dk + j] = decay_at(a, channel_decay, NH, dk, t, h, j);
+                lg.a[(long)e * dk + j] = decay_at(a, kind, NH, dk, t, h, j);
             lg.n = e + 1;
             deferred_read(Sbar, &lg, q + ((long)t * NH + h) * dk,
                           o + ((long)t * NH + h) * dv, x, s);
@@ -271,4 +297,4 @@ void oracle_deferred(long NH, int T, int dk, int dv, int channel_decay, int L,
 }
 
 /* Version tag so the Python side can tell a stale build. */
-int oracle_abi_version(void) { return 1; }
+int oracle_abi_version(void) { return 2; }

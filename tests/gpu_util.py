@@ -28,21 +28,26 @@ def run_cuda(w: W.Workload, d, path: str, L: int = 0, fused: bool = True, keep_o
     S = d["S0"].clone()
     B, H = S.shape[0], S.shape[1]
     T = w.T
-    chan = w.decay == W.CHANNEL
+    chan = w.decay != W.HEAD
+    rw = w.decay == W.RWKV6
     o_step = torch.empty(B, H, w.d_v, dtype=torch.float32, device=S.device)
     keep = []
     if path == "eager":
         fn = g.dl_kda_decode_step if chan else g.dl_gdn_decode_step
         for t in range(T):
-            fn(S, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o_step)
+            if rw:
+                g.dl_rwkv6_decode_step(S, d["q"][t], d["k"][t], d["v"][t], d["a"][t], o_step)
+            else:
+                fn(S, d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o_step)
             if keep_o:
                 keep.append(_pick(o_step, o_heads))
     else:
         tdt = d["q"].dtype
-        log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=S.device)
+        log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=S.device, rwkv6=rw)
         dec = g.DeferredDecoder(S, log, fused_merge=fused)
         for t in range(T):
-            dec.step(d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["a"][t], o_step)
+            beta_t = None if rw else d["beta"][t]
+            dec.step(d["q"][t], d["k"][t], d["v"][t], beta_t, d["a"][t], o_step)
             if keep_o:
                 keep.append(_pick(o_step, o_heads))
         dec.flush()

@@ -87,6 +87,15 @@ def test_byte_model_matches_the_state_sizes():
     assert bench.alg_bytes(w, "append_read", 3) - w.state_bytes() == w.heads * (5 * 770 + 256 + 512 + 4 * 3 + 4 * 3)
     w4 = W.WORKLOADS["gdn_b1024_h32_dk128_dv256_t256"]
     assert w4.state_bytes() == 2 << 30 and bench.entry_bytes(w4) == (128 + 256 + 2) * 2
+    # a pool step at staggered fills: 1/L of the rows at each count, the last one merging
+    assert bench.alg_bytes(w, "pool", 16) == (sum(bench.alg_bytes(w, "append_read", c) for c in range(15))
+                                              + bench.alg_bytes(w, "merge_read", 15)) // 16
+    lau = bench.Launcher(None, w, None, None, type("FakeLog", (), {"L": 16})(), None, "pool", None)
+    assert lau.plan() == [("pool", 16)] * w.T
+    # RWKV6: no beta in an entry and no triangular-solve rows in the log
+    w6 = W.WORKLOADS["rwkv6_b256_h32_d128_t512"]
+    assert bench.entry_bytes(w6) == (128 + 128 + 128) * 2
+    assert bench.alg_bytes(w6, "append_read", 3) - w6.state_bytes() == w6.heads * (5 * 768 + 256 + 512)
 
 
 def test_reduce_max_without_process_group():

@@ -117,6 +117,35 @@ def test_log_step_argument_checks(lib, fn):
     assert "log.x is a null pointer" in lib.dl_last_error().decode()
 
 
+def test_rwkv6_needs_no_beta_or_metadata(lib):
+    # RWKV6 reads neither beta nor log.x, so null is accepted for both; each call
+    # then stops at a later check that fails on purpose (n = L), launching nothing.
+    lg = make_log()
+    lg.beta = None
+    lg.x = None
+    args = (addr(1), addr(2), addr(3), None, addr(5), b.DL_BF16, addr(6), 2, 3, 128, 128, None)
+    for fn in ("dl_log_append_read", "dl_log_merge_read", "dl_log_append_read_noalloc"):
+        assert getattr(lib, fn)(addr(0), b.DL_F32, b.DL_RWKV6, ctypes.byref(lg), 8, *args) == b.DL_ERR_LOG_FULL
+        assert getattr(lib, fn)(addr(0), b.DL_F32, b.DL_DECAY_CHANNEL, ctypes.byref(lg), 8, *args) \
+            == b.DL_ERR_INVALID_ARG
+        assert "is a null pointer" in lib.dl_last_error().decode()
+    assert lib.dl_log_merge(addr(0), b.DL_F32, b.DL_RWKV6, ctypes.byref(lg), 0, 2, 3, 128, 128, None) \
+        == b.DL_ERR_INVALID_ARG                                           # n = 0: nothing to merge
+    assert "1 <= n <= L" in lib.dl_last_error().decode()
+
+
+def test_rwkv6_eager_argument_checks(lib):
+    def rw(S=None, a=None, o=None, dk=128, dv=128):
+        S = None if S == -1 else (S or addr(0))
+        return lib.dl_rwkv6_decode_step(S, b.DL_F32, addr(1), addr(2), addr(3), a or addr(5), b.DL_BF16,
+                                        o or addr(6), 2, 3, dk, dv, None)
+
+    assert rw(S=-1) == b.DL_ERR_INVALID_ARG and "S is a null pointer" in lib.dl_last_error().decode()
+    assert rw(a=addr(5) + 2) == b.DL_ERR_INVALID_ARG                        # a is a per-channel vector
+    assert rw(dk=96) == b.DL_ERR_UNSUPPORTED
+    assert rw(o=addr(0) + 4096) == b.DL_ERR_INVALID_ARG                     # o inside S
+
+
 def test_append_read_workspace_checks(lib):
     assert lib.dl_log_work_bytes(2, 3, 128, 128) == 2 * 3 * 256 * 4
     lg = make_log()
@@ -139,7 +168,7 @@ def test_merge_argument_checks(lib):
 
     assert merge(0) == b.DL_ERR_INVALID_ARG
     assert merge(9) == b.DL_ERR_INVALID_ARG
-    assert merge(3, kind=2) == b.DL_ERR_INVALID_ARG
+    assert merge(3, kind=5) == b.DL_ERR_INVALID_ARG
     assert merge(3, dk=32) == b.DL_ERR_UNSUPPORTED
     assert merge(3, S=addr(0) + 4) == b.DL_ERR_INVALID_ARG
     assert lib.dl_log_merge(addr(0), b.DL_F32, 0, None, 1, 2, 3, 128, 128, None) == b.DL_ERR_INVALID_ARG

@@ -18,7 +18,7 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "deltalog_oracle.c")
 MUTATIONS = {
     # eager step
     "eager_drops_decay": ("row[j] = row[j] * avec[j];", "row[j] = row[j];"),
-    "eager_wrong_sign": ("double coef = beta * (v[i] - u);", "double coef = beta * (v[i] + u);"),
+    "eager_wrong_sign": ("beta * (v[i] - u) : v[i];", "beta * (v[i] + u) : v[i];"),
     "eager_writes_q": ("row[j] = row[j] + coef * k[j];", "row[j] = row[j] + coef * q[j];"),
     "eager_output_reads_k": ("acc += row[j] * q[j];", "acc += row[j] * k[j];"),
     "head_decay_wrong_head": ("return a[(long)t * NH + h];", "return a[(long)t * NH];"),
@@ -36,6 +36,13 @@ MUTATIONS = {
     "merge_write_undecayed": ("newrow[c] += delta[j] * kj[c] * dnj[c];", "newrow[c] += delta[j] * kj[c];"),
     "merge_decay_product": ("cur[c] = prev[c] * ai[c];", "cur[c] = prev[c];"),
     "no_final_flush": ("        deferred_merge(Sbar, &lg);\n        free(s);", "        free(s);"),
+    # RWKV6
+    "rwkv6_scales_value_by_beta": ("beta * (v[i] - u) : v[i];", "beta * (v[i] - u) : beta * v[i];"),
+    "rwkv6_eager_corrects": ("double coef = delta ?", "double coef = 1 ?"),
+    "rwkv6_read_subtracts": ("x[j] = ai[j] * x[j];", "x[j] = ai[j] * (x[j] - s[i] * ki[j]);"),
+    "rwkv6_read_drops_decay": ("x[j] = ai[j] * x[j];", "x[j] = x[j];"),
+    "rwkv6_merge_decays_own_value": ("delta[i] = lg->v[(long)(i - 1) * dv + r];",
+                                     "delta[i] = lg->v[(long)(i - 1) * dv + r] * lg->a[(long)(i - 1) * dk];"),
 }
 
 CHECKS = {
@@ -47,6 +54,8 @@ CHECKS = {
     "p5": pins.check_p5,
     "p6": pins.check_p6,
     "p7": pins.check_p7,
+    "p9": pins.check_p9,
+    "p10": pins.check_p10,
 }
 
 

@@ -18,7 +18,14 @@ Pins:
   P5 channel decay with all channels equal = head-wise decay;
   P6 deferred schedule = eager for every log capacity (merge cadence, flush);
   P7 dense brute-force matrix products = eager = deferred on tiny shapes;
-  P8 the deferred window identity S_n = S_bar A_1..A_n + sum beta v k^T A_{i+1}..A_n.
+  P8 the deferred window identity S_n = S_bar A_1..A_n + sum beta v k^T A_{i+1}..A_n;
+  P9 RWKV6 (per-key decay, raw-value update, no correction: S_t = S_{t-1} Diag(a_t)
+     + v_t k_t^T) -- dense brute force = eager = deferred at every log capacity;
+  P10 RWKV6 closed form S_T = S_0 Diag(prod_t a_t) + sum_t v_t (k_t o prod_{m>t} a_m)^T,
+     with its special cases a = 1 (plain linear attention) and a = 0;
+  P11 the slot pool (per-sequence states in slots, ragged batches): a
+     sequence's outputs and state are those of its own recurrence, whatever
+     the other slots do; slots not listed in a step are left unchanged.
 The mutation test builds copies of the C oracle with planted mistakes and
 checks that these pins reject each of them.
 """
@@ -68,7 +75,8 @@ def test_p0_hand_worked_examples(form, oracle_mod):
 def run_golden(form, impl):
     g = json.load(open(GOLDEN))
     for case in g["cases"]:
-        chan = case["decay"] == "channel"
+        rw = case["decay"] == "rwkv6"
+        chan = case["decay"] in ("channel", "rwkv6")
         S0 = np.array([[[_frac(x) for x in r] for r in case["S0"]]])
         steps = case["steps"]
         T = len(steps)
@@ -84,18 +92,18 @@ def run_golden(form, impl):
         o_exp = np.array([[[_frac(x) for x in s["o"]]] for s in steps])
         S_exp = np.array([[[_frac(x) for x in r] for r in steps[-1]["S"]]])
         if form == "eager":
-            o, S = impl.eager(S0, q, k, v, beta, a, chan)
+            o, S = impl.eager(S0, q, k, v, beta, a, chan, rw)
         elif form.startswith("deferred"):
-            o, S = impl.deferred(S0, q, k, v, beta, a, chan, int(form[-1]))
+            o, S = impl.deferred(S0, q, k, v, beta, a, chan, int(form[-1]), rw)
         else:
-            o, S = oracle.brute_force(S0, q, k, v, beta, a, chan)
+            o, S = oracle.brute_force(S0, q, k, v, beta, a, chan, rw)
         assert np.allclose(o, o_exp, rtol=0, atol=1e-14), (case["name"], form, o, o_exp)
         assert np.allclose(S, S_exp, rtol=0, atol=1e-14), (case["name"], form, S, S_exp)
         # every intermediate state as well (eager, one step at a time)
         if form == "eager":
             Sc = S0
             for t, s in enumerate(steps):
-                _, Sc = impl.eager(Sc, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1], a[t:t + 1], chan)
+                _, Sc = impl.eager(Sc, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1], a[t:t + 1], chan, rw)
                 exp = np.array([[[_frac(x) for x in r] for r in s["S"]]])
                 assert np.allclose(Sc, exp, rtol=0, atol=1e-14), (case["name"], t)
 
@@ -289,6 +297,102 @@ def test_p8_window_identity():
     for i in range(n):
         S = S @ np.diag(As[i]) @ (np.eye(dk) - betas[i] * np.outer(ks[i], ks[i])) + betas[i] * np.outer(vs[i], ks[i])
     assert rel(oracle.brute_force_window(Sbar, ks, vs, betas, As), S) < 1e-13
+
+
+# ------------------------------------------------------------------ P9, P10 (RWKV6)
+
+def check_p9(impl):
+    rng = np.random.default_rng(20)
+    for (dk, dv) in ((4, 4), (5, 3), (3, 7), (8, 8)):
+        NH, T = 2, 7
+        S0, q, k, v, _, a = rand_case(rng, NH, T, dk, dv, True, unit_k=False)
+        o_b, S_b = oracle.brute_force(S0, q, k, v, None, a, True, rwkv6=True)
+        o_e, S_e = impl.eager(S0, q, k, v, None, a, True, rwkv6=True)
+        assert rel(o_e, o_b) < 1e-13 and rel(S_e, S_b) < 1e-13, (dk, dv)
+        for L in (1, 2, 3, 7, 9):
+            o_d, S_d = impl.deferred(S0, q, k, v, None, a, True, L, rwkv6=True)
+            assert rel(o_d, o_b) < 1e-12 and rel(S_d, S_b) < 1e-12, (dk, dv, L)
+
+
+def test_p9_rwkv6_brute_force(oracle_mod):
+    check_p9(oracle_mod)
+
+
+def rwkv6_closed_form(S0, q, k, v, a):
+    """o_t and S_T from the unrolled sum (no step recursion):
+    S_t = S_0 Diag(prod_{m<=t} a_m) + sum_{i<=t} v_i (k_i o prod_{i<m<=t} a_m)^T."""
+    T = q.shape[0]
+    o = np.zeros(v.shape)
+    for t in range(T):
+        cum = np.prod(a[:t + 1], axis=0)  # [NH, dk]
+        S = S0 * cum[:, None, :]
+        for i in range(t + 1):
+            tail = np.prod(a[i + 1:t + 1], axis=0) if i < t else np.ones_like(cum)
+            S = S + np.einsum("hv,hk->hvk", v[i], k[i] * tail)
+        o[t] = np.einsum("hvk,hk->hv", S, q[t])
+    return o, S
+
+
+def check_p10(impl):
+    rng = np.random.default_rng(21)
+    NH, T, dk, dv = 2, 8, 6, 5
+    S0, q, k, v, _, a = rand_case(rng, NH, T, dk, dv, True, unit_k=False)
+    for aa in (a, np.ones_like(a), np.zeros_like(a)):
+        o_c, S_c = rwkv6_closed_form(S0, q, k, v, aa)
+        if aa is not a and aa.max() == 1.0:  # a = 1: plain linear attention
+            assert rel(S_c, S0 + np.einsum("thv,thk->hvk", v, k)) < 1e-14
+        if aa.max() == 0.0:  # a = 0: only the last outer product survives
+            assert rel(S_c, np.einsum("hv,hk->hvk", v[-1], k[-1])) < 1e-14
+        for form in ("eager", 1, 3, 8):
+            o, S = (impl.eager(S0, q, k, v, None, aa, True, rwkv6=True) if form == "eager"
+                    else impl.deferred(S0, q, k, v, None, aa, True, form, rwkv6=True))
+            assert rel(o, o_c) < 1e-13 and rel(S, S_c) < 1e-13, form
+
+
+def test_p10_rwkv6_closed_form(oracle_mod):
+    check_p10(oracle_mod)
+
+
+# ------------------------------------------------------------------ P11 (slot pool)
+
+def check_p11():
+    rng = np.random.default_rng(22)
+    P, H, dk, dv, T = 4, 2, 6, 5, 9
+    for chan, rw in ((False, False), (True, False), (True, True)):
+        S_pool0 = rng.standard_normal((P, H, dv, dk))
+        # two sequences: A lives in slot 2 for all steps; B in slot 0 for steps
+        # 0..3, then a new sequence C takes slot 0 from its own initial state.
+        S_C = rng.standard_normal((H, dv, dk))
+        per_seq = {name: rand_case(rng, H, T, dk, dv, chan or rw) for name in "ABC"}
+        steps, resets, rows = [], {5: {0: S_C}}, []
+        for t in range(T):
+            listed = [(2, "A")] + ([(0, "B")] if t < 4 else [(0, "C")] if t >= 5 else [])
+            if t % 2:
+                listed = listed[::-1]
+            slot = np.array([s_ for s_, _ in listed])
+            idx = {"q": 1, "k": 2, "v": 3, "beta": 4, "a": 5}
+            steps.append((slot, *(np.stack([per_seq[n_][idx[key]][t] for _, n_ in listed])
+                                  for key in ("q", "k", "v", "beta", "a"))))
+            rows.append([n_ for _, n_ in listed])
+        outs, S_fin = oracle.pool_eager(S_pool0, steps, chan, rw, resets)
+        # each sequence alone
+        def alone(S0, name, t0, t1):
+            c = per_seq[name]
+            sl = slice(t0, t1)
+            return oracle.eager(S0, c[1][sl], c[2][sl], c[3][sl], c[4][sl], c[5][sl], chan, rw)
+        oA, SA = alone(S_pool0[2], "A", 0, T)
+        oB, SB = alone(S_pool0[0], "B", 0, 4)
+        oC, SC = alone(S_C, "C", 5, T)
+        for t in range(T):
+            for j, name in enumerate(rows[t]):
+                ref = {"A": lambda: oA[t], "B": lambda: oB[t], "C": lambda: oC[t - 5]}[name]()
+                assert np.array_equal(outs[t][j], ref), (chan, rw, t, name)
+        assert np.array_equal(S_fin[2], SA) and np.array_equal(S_fin[0], SC)
+        assert np.array_equal(S_fin[1], S_pool0[1]) and np.array_equal(S_fin[3], S_pool0[3])  # never listed
+
+
+def test_p11_slot_pool_is_per_sequence_recurrence(oracle_mod):
+    check_p11()
 
 
 # ------------------------------------------------------------------ inputs

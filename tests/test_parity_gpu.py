@@ -48,12 +48,19 @@ def test_gdn_small_fp32(path, L, fused):
     check(W.WORKLOADS["gdn_b1_h2_d64_t16"], path, L, fused)
 
 
+@pytest.mark.parametrize("path,L,fused", [("eager", 0, True), ("deferred", 4, True), ("deferred", 4, False),
+                                          ("deferred", 16, True), ("deferred", 1, True), ("deferred", 5, False)])
+def test_rwkv6_small_fp32(path, L, fused):
+    check(W.scaled(W.WORKLOADS["gdn_b1_h2_d64_t16"], name="rwkv6_b1_h2_d64_t16", decay=W.RWKV6), path, L, fused)
+
+
 # --------------------------------------------------------------- reduced sizes of each workload
 
 REDUCED = [
     (W.scaled(W.WORKLOADS["gdn_b64_h16_d128_t1024"], B=3, H=4, T=45), 8),
     (W.scaled(W.WORKLOADS["kda_b256_h32_d128_t512"], B=3, H=5, T=40), 16),
     (W.scaled(W.WORKLOADS["gdn_b1024_h32_dk128_dv256_t256"], B=2, H=3, T=29), 8),
+    (W.scaled(W.WORKLOADS["rwkv6_b256_h32_d128_t512"], B=3, H=5, T=40), 16),
 ]
 
 
@@ -81,7 +88,7 @@ _SWEEP_INPUTS = {}
 # --------------------------------------------------------------- every supported shape and dtype
 
 COMBOS = [(dk, dv, sd, idt, dec) for dk in (64, 128) for dv in (64, 128, 256) for sd in ("f32", "bf16")
-          for idt in ("f32", "bf16") for dec in (W.HEAD, W.CHANNEL)]
+          for idt in ("f32", "bf16") for dec in (W.HEAD, W.CHANNEL, W.RWKV6)]
 
 
 @pytest.mark.parametrize("dk,dv,sd,idt,dec", COMBOS)
@@ -108,6 +115,16 @@ def test_zero_decay_resets_state():
     x = _custom(w, a=lambda a: np.zeros_like(a))
     for path, L, fused in (("eager", 0, True), ("deferred", 4, True), ("deferred", 4, False)):
         check(w, path, L, fused, x=x)
+
+
+def test_rwkv6_zero_decay_keeps_last_outer_product():
+    """RWKV6 with a = 0: S_t = v_t k_t^T each step; with a = 1 it is plain
+    linear attention, S_t = S_0 + sum v k^T (both against the oracle)."""
+    w = W.Workload("rwkv6_decays", W.RWKV6, 2, 3, 128, 64, 9, "f32", "f32", 0.1, (4,))
+    for fill in (np.zeros_like, np.ones_like):
+        x = _custom(w, a=lambda a: fill(a))
+        for path, L, fused in (("eager", 0, True), ("deferred", 4, True), ("deferred", 4, False)):
+            check(w, path, L, fused, x=x)
 
 
 def test_beta_zero_and_unit_decay_keep_state():
@@ -160,3 +177,26 @@ def test_append_leaves_base_unwritten_and_logs_inputs():
         assert torch.equal(log.beta[:, :, t], d["beta"][t]) and torch.equal(log.a[:, :, t], d["a"][t])
     with pytest.raises(g.DeltaLogError):
         g.dl_log_append_read(S, log, 4, d["q"][0], d["k"][0], d["v"][0], d["beta"][0], d["a"][0], o)
+
+
+def test_rwkv6_log_has_no_beta_or_metadata():
+    """An RWKV6 log is allocated without beta and x (null pointers through the
+    ABI); appends store k, v, a unchanged and leave the base unwritten."""
+    import torch
+
+    import gated_delta_rule_104_b200 as g
+
+    w = W.Workload("append_rwkv6", W.RWKV6, 2, 3, 128, 128, 3, "bf16", "f32", 0.1, (4,))
+    d = device_inputs(w, W.generate(w))
+    S = d["S0"].clone()
+    before = S.clone()
+    log = g.Log.allocate(2, 3, 128, 128, 4, torch.bfloat16, True, rwkv6=True)
+    assert log.beta is None and log.x is None and log.kind == g.DL_RWKV6
+    o = torch.empty(2, 3, 128, device="cuda")
+    for t in range(3):
+        g.dl_log_append_read(S, log, t, d["q"][t], d["k"][t], d["v"][t], None, d["a"][t], o)
+    torch.cuda.synchronize()
+    assert torch.equal(S, before)
+    for t in range(3):
+        assert torch.equal(log.k[:, :, t], d["k"][t]) and torch.equal(log.v[:, :, t], d["v"][t])
+        assert torch.equal(log.a[:, :, t], d["a"][t])

@@ -46,12 +46,13 @@ import numpy as np
 
 HEAD = "head"        # one scalar decay per head and step (Gated DeltaNet)
 CHANNEL = "channel"  # one decay per key channel and step (Kimi Delta Attention)
+RWKV6 = "rwkv6"      # one decay per key channel, raw-value update, no beta (RWKV6)
 
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    decay: str           # HEAD or CHANNEL
+    decay: str           # HEAD, CHANNEL or RWKV6
     B: int
     H: int
     d_k: int
@@ -85,6 +86,8 @@ WORKLOADS: Dict[str, Workload] = {
                  (1, 4, 8, 16, 32, 64), note="KDA log-length sweep"),
         Workload("gdn_b1024_h32_dk128_dv256_t256", HEAD, 1024, 32, 128, 256, 256, "bf16", "bf16", 1.0,
                  (8,), note="large-batch GDN, bf16 state, strong decay, deferred L=8"),
+        Workload("rwkv6_b256_h32_d128_t512", RWKV6, 256, 32, 128, 128, 512, "bf16", "f32", 0.1, (16,),
+                 note="RWKV6 at the KDA target's shapes: channel decay, raw-value update"),
     ]
 }
 WORKLOAD_ORDER: List[str] = list(WORKLOADS)
