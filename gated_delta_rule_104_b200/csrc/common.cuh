@@ -187,6 +187,33 @@ __device__ __forceinline__ void copy_hint(T *dst, const T *src, uint64_t pol) {
         st_hint(reinterpret_cast<unsigned char *>(dst) + i * W,
                 *reinterpret_cast<const Word *>(reinterpret_cast<const unsigned char *>(src) + i * W), pol);
 }
+// The same copy split in two, so that several copies' loads can be in flight
+// before the first store: load() reads the words, store() writes them.
+template <int N, class T>
+struct RawCopy {
+    static constexpr int BYTES = N * (int)sizeof(T), W = BYTES < 16 ? BYTES : 16, K = BYTES / W;
+    using Word = typename HintWord<W>::T;
+    Word w[K];
+    __device__ __forceinline__ void load(const T *src) {
+#pragma unroll
+        for (int i = 0; i < K; ++i)
+            w[i] = *reinterpret_cast<const Word *>(reinterpret_cast<const unsigned char *>(src) + i * W);
+    }
+    __device__ __forceinline__ void load_hint(const T *src, uint64_t pol) {
+#pragma unroll
+        for (int i = 0; i < K; ++i) ld_hint(reinterpret_cast<const unsigned char *>(src) + i * W, w[i], pol);
+    }
+    __device__ __forceinline__ void store(T *dst, uint64_t pol) const {
+#pragma unroll
+        for (int i = 0; i < K; ++i) st_hint(reinterpret_cast<unsigned char *>(dst) + i * W, w[i], pol);
+    }
+    // the N elements widened to float
+    __device__ __forceinline__ void widen(float (&x)[N]) const {
+        const T *e = reinterpret_cast<const T *>(w);
+#pragma unroll
+        for (int i = 0; i < N; ++i) x[i] = to_f(e[i]);
+    }
+};
 // N elements of T (as load_vec) read under an L2 policy, widened to float.
 template <int N, class T>
 __device__ __forceinline__ void load_vec_hint(const T *p, float (&x)[N], uint64_t pol) {
@@ -274,11 +301,6 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
     asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(s), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async16_hint(void *smem_dst, const void *gmem_src, uint64_t pol) {
-    uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem_src), "l"(pol)
-                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }

@@ -92,56 +92,102 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     }
     const long long lrow = shead * L;
     const int c0 = lane * CW, r0 = lane * RV;
-    // The log stays L2-resident between steps: its reads and writes carry an
-    // evict-last policy (the base streams through with evict-first).
+    // The log stays L2-resident between steps: its loads and stores carry an
+    // evict-last policy (the base streams through with evict-first); the
+    // cp.async staging copies carry none.
     const uint64_t keep = l2_policy_keep();
 
     // Stage keys and decays of entries 0..n-1 (log) and n (this step), raw.
     for (int u = lane; u < (n + 1) * (DK / E); u += 32) {
         const int e = u / (DK / E), col = (u % (DK / E)) * E;
         if (e < n) {
-            cp_async16_hint(sk + e * DK + col, log_k + (lrow + e) * DK + col, keep);
-            if constexpr (CHAN) cp_async16_hint(sa + e * DK + col, log_a + (lrow + e) * DK + col, keep);
+            cp_async16(sk + e * DK + col, log_k + (lrow + e) * DK + col);
+            if constexpr (CHAN) cp_async16(sa + e * DK + col, log_a + (lrow + e) * DK + col);
         } else {
             cp_async16(sk + e * DK + col, k + head * DK + col);
             if constexpr (CHAN) cp_async16(sa + e * DK + col, a + head * DK + col);
         }
     }
     cp_async_commit();
-    for (int e = lane; e <= n; e += 32) {
-        if constexpr (DELTA) {
-            float bx[1];
-            if (e < n) load_vec_hint<1>(log_b + lrow + e, bx, keep);
-            else bx[0] = to_f(beta[head]);
-            fbeta[e] = bx[0];
-        }
-        if constexpr (!CHAN) {
-            float ax[1];
-            if (e < n) load_vec_hint<1>(log_a + lrow + e, ax, keep);
-            else ax[0] = to_f(a[head]);
-            fas[e] = ax[0];
-        }
-    }
-    // X rows of the logged entries (rows j < n, columns e <= j).
-    for (int u = lane; DELTA && u < n * EMAX; u += 32) {
-        const int j = u / EMAX, e = u % EMAX;
-        if (e <= j) {
-            float xx[1];
-            load_vec_hint<1>(log_x + (lrow + j) * L + e, xx, keep);
-            xrow[j * EMAX + e] = xx[0];
+    // Everything else the head needs is loaded next, all loads before the first
+    // store that consumes one (a warp issues in order: a store waiting on its
+    // load would hold back every load behind it).
+    constexpr int SB = (EMAX + 31) / 32;
+    RawCopy<1, IT> bx[SB], ax[SB];  // beta and a head-wise decay of entries lane, lane + 32 (<= n), raw
+#pragma unroll
+    for (int i = 0; i < SB; ++i) {
+        const int e = lane + 32 * i;
+        if (e <= n) {
+            if constexpr (DELTA) {
+                if (e < n) bx[i].load_hint(log_b + lrow + e, keep);
+                else bx[i].load(beta + head);
+            }
+            if constexpr (!CHAN) {
+                if (e < n) ax[i].load_hint(log_a + lrow + e, keep);
+                else ax[i].load(a + head);
+            }
         }
     }
+    // X rows of the logged entries (rows j < n, columns e <= j), XB per lane a batch.
+    constexpr int XB = 8;
+    float xx[XB];
+    auto x_load = [&](int base) {
+#pragma unroll
+        for (int i = 0; i < XB; ++i) {
+            const int u = base + i * 32 + lane, j = u / EMAX, e = u % EMAX;
+            xx[i] = 0.f;
+            if (DELTA && u < n * EMAX && e <= j) {
+                float t1[1];
+                load_vec_hint<1>(log_x + (lrow + j) * L + e, t1, keep);
+                xx[i] = t1[0];
+            }
+        }
+    };
+    auto x_store = [&](int base) {
+#pragma unroll
+        for (int i = 0; i < XB; ++i) {
+            const int u = base + i * 32 + lane, j = u / EMAX, e = u % EMAX;
+            if (DELTA && u < n * EMAX && e <= j) xrow[j * EMAX + e] = xx[i];
+        }
+    };
+    x_load(0);
     // D1: the entry is appended unchanged (raw input elements).
-    copy_hint<CW>(log_k + (lrow + n) * DK + c0, k + head * DK + c0, keep);
-    copy_hint<RV>(log_v + (lrow + n) * DV + r0, v + head * DV + r0, keep);
+    RawCopy<CW, IT> ck, ca;
+    RawCopy<RV, IT> cv;
+    ck.load(k + head * DK + c0);
+    cv.load(v + head * DV + r0);
+    if constexpr (CHAN) ca.load(a + head * DK + c0);
+    float qv[CW];
+    load_vec<CW>(q + head * DK + c0, qv);
+    // the stores
+#pragma unroll
+    for (int i = 0; i < SB; ++i) {
+        const int e = lane + 32 * i;
+        if (e <= n) {
+            float t1[1];
+            if constexpr (DELTA) {
+                bx[i].widen(t1);
+                fbeta[e] = t1[0];
+            }
+            if constexpr (!CHAN) {
+                ax[i].widen(t1);
+                fas[e] = t1[0];
+            }
+        }
+    }
+    x_store(0);
+    for (int base = 32 * XB; DELTA && base < n * EMAX; base += 32 * XB) {  // longer logs only
+        x_load(base);
+        x_store(base);
+    }
+    ck.store(log_k + (lrow + n) * DK + c0, keep);
+    cv.store(log_v + (lrow + n) * DV + r0, keep);
     if constexpr (CHAN) {
-        copy_hint<CW>(log_a + (lrow + n) * DK + c0, a + head * DK + c0, keep);
+        ca.store(log_a + (lrow + n) * DK + c0, keep);
     } else if (lane == 0) {
         copy_hint<1>(log_a + lrow + n, a + head, keep);
     }
     if (DELTA && lane == 0) copy_hint<1>(log_b + lrow + n, beta + head, keep);
-    float qv[CW];
-    load_vec<CW>(q + head * DK + c0, qv);
     cp_async_wait_all();
     __syncwarp();
 
@@ -195,6 +241,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     const float bn = DELTA ? fbeta[n] : 0.f;
     for (int j = lane; DELTA && j <= n; j += 32) {
         float acc = 0.f;
+#pragma unroll 4
         for (int m = j; m < n; ++m) acc = fmaf(fcn[m], xrow[m * EMAX + j], acc);
         const float xnj = j == n ? bn : -bn * acc;
         xrow[n * EMAX + j] = xnj;
@@ -205,6 +252,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     for (int e = lane; e <= n; e += 32) {
         float acc = 0.f;
         if constexpr (DELTA) {
+#pragma unroll 4
             for (int i = e; i <= n; ++i) acc = fmaf(xrow[i * EMAX + e], fd[i], acc);
         } else {
             acc = fd[e];
@@ -220,6 +268,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         g[c] = 1.f;
         xs[c] = 0.f;
     }
+#pragma unroll 4
     for (int e = 0; e <= n; ++e) {
         float ke[CW], ae[CW];
         load_vec<CW>(sk + e * DK + c0, ke);
@@ -234,14 +283,29 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     float w[RV];
 #pragma unroll
     for (int r = 0; r < RV; ++r) w[r] = 0.f;
-#pragma unroll 4
-    for (int e = 0; e <= n; ++e) {
-        float ve[RV];
-        if (e < n) load_vec_hint<RV>(log_v + (lrow + e) * DV + r0, ve, keep);
-        else load_vec<RV>(v + head * DV + r0, ve);
-        const float se = fs[e];
+    // Entries in batches of VB: a batch's raw words are all loaded before any is
+    // widened (a widening right after its load would stall the loads behind it).
+    constexpr int VB = 8;
+    using VC = RawCopy<RV, IT>;
+    for (int e0 = 0; e0 <= n; e0 += VB) {
+        VC raw[VB];
 #pragma unroll
-        for (int r = 0; r < RV; ++r) w[r] = fmaf(se, ve[r], w[r]);
+        for (int i = 0; i < VB; ++i) {
+            const int e = e0 + i;
+            if (e < n) raw[i].load_hint(log_v + (lrow + e) * DV + r0, keep);
+            else if (e == n) raw[i].load(v + head * DV + r0);
+        }
+#pragma unroll
+        for (int i = 0; i < VB; ++i) {
+            const int e = e0 + i;
+            if (e <= n) {
+                const float se = fs[e];
+                float ve[RV];
+                raw[i].widen(ve);
+#pragma unroll
+                for (int r = 0; r < RV; ++r) w[r] = fmaf(se, ve[r], w[r]);
+            }
+        }
     }
 
     float *wk = work + head * (DK + DV);

@@ -99,15 +99,19 @@ struct MergeShape {
 };
 
 // The block's base rows in shared memory: ROWS x DK elements of the state
-// type, row-major with the 16-byte chunks of row r XOR-swizzled by (r mod 8),
-// so that an 8-row x 4-column fragment read touches 32 distinct banks
-// without padding.
+// type, row-major with the 16-byte chunks of row r XOR-swizzled by
+// f(r) = 2 (r mod 4) + (r / 4 mod 2), a permutation of 0..7. Over the 8 rows
+// of a fragment f takes every value, so an 8-row x 4-column operand read hits
+// 32 distinct banks; over each 4-row half it takes distinct pairs f / 2, so
+// the accumulator-layout accesses (4 rows x 8 consecutive fp32 per half warp)
+// do too. No padding.
 template <class ST, int DK>
 struct BaseTile {
     static constexpr int CE = 16 / (int)sizeof(ST);  // elements per 16-byte chunk
     static_assert(DK / CE >= 8, "swizzle spans 8 chunks");
     __device__ static __forceinline__ int off(int r, int c) {
-        return r * DK + (((c / CE) ^ (r & 7)) * CE) + (c % CE);
+        const int f = ((r & 3) << 1) | ((r >> 2) & 1);
+        return r * DK + (((c / CE) ^ f) * CE) + (c % CE);
     }
 };
 
@@ -116,12 +120,13 @@ struct BaseTile {
 //   kh [NB][KH] keys, turned into Khat in place
 //   ff [NB][WS] F (channel decay: holds the decays until F replaces them)
 //   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
-//   cm [NB] C row   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
+//   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
+//   sxw [4][XS] each warp's copy of the fused entry's X row
 template <class ST, int DK, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
     using C = MergeShape<DK, NB>;
-    const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK + round4(NB) +
-                          (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS;
+    const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK +
+                          (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS + 4 * (size_t)C::XS;
     return (size_t)C::ROWS * DK * sizeof(ST) + floats * sizeof(float);
 }
 
@@ -182,10 +187,10 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     float *fa = ff + NB * C::WS;
     float *gn = fa + round4(NB);
     float *sq = gn + DK;
-    float *cm = sq + DK;
-    float *sx = cm + round4(NB);
+    float *sx = sq + DK;
     float *sb = sx + NB * C::XS;
     float *sv = sb + round4(NB);
+    float *sxw = sv + NB * C::VS;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;  // fragment coordinates
@@ -200,8 +205,10 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     ST *Sw = S + (shead * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
     const int tr = 16 * warp;                           // and their first row in the tile
 
-    // The block's base rows, fetched first (they land while the log is staged).
-    {
+    // The block's base rows, fetched by cp.async right after the first entry
+    // block's loads are issued (those come first, so that they do not queue
+    // behind the tile); the tile lands while the key side is worked out.
+    auto fetch_tile = [&]() {
         constexpr int CPR = DK / TL::CE;  // chunks per row
         const ST *src = S + (shead * DV + row0) * DK;
 #pragma unroll 4
@@ -210,12 +217,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
         }
         cp_async_commit();
-    }
-
-    if constexpr (WITH_CUR) {
-        if (bf) stage_block(sq, DK, static_cast<const bf16 *>(q) + head * DK, DK, 1, DK, tid, nthr);
-        else stage_block(sq, DK, static_cast<const float *>(q) + head * DK, DK, 1, DK, tid, nthr);
-    }
+    };
 
     float oacc[2] = {0.f, 0.f};  // o for rows g and g + 8 (fused read), partial over this lane's columns
     for (int b0 = 0; b0 < NTOT; b0 += NB) {
@@ -233,8 +235,11 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             constexpr int KN = (NB * KC + 127) / 128;       // >= 128 threads per block
             constexpr int VN = (NB * 128 / E + 127) / 128;  // rows <= 128
             const int VC = ROWS / E;
-            float kx[KN][E], ax[KN][E], vx[VN][E];
+            float kx[KN][E], ax[KN][E], vx[VN][E], qx[E];
             (void)ax;
+            (void)qx;
+            const bool qload = WITH_CUR && b0 == 0 && tid < KC;  // this step's q, with the first block
+            if (qload) load_vec<E>(static_cast<const IT *>(q) + head * DK + tid * E, qx);
             auto key_src = [&](const void *logp, const void *cur, int r) -> const IT * {
                 return r < nl ? static_cast<const IT *>(logp) + (lrow + b0 + r) * DK
                               : static_cast<const IT *>(cur) + head * DK;
@@ -276,6 +281,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 cval[u] = (DELTA && idx < NB * NB && cj <= ci && ci < nl) ? log_x[(lrow + b0 + ci) * L + b0 + cj]
                                                                             : 0.f;
             }
+            if (b0 == 0) fetch_tile();
             auto put = [](float *dst, const float *x, bool real, float pad) {
 #pragma unroll
                 for (int e = 0; e < E; e += 4)
@@ -299,6 +305,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 sb[tid] = bsc;  // 0 for padded entries
                 if constexpr (!CHAN) fa[tid] = asc;
             }
+            if (qload) put(sq + tid * E, qx, true, 0.f);
 #pragma unroll
             for (int u = 0; u < CN; ++u) {
                 const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
@@ -336,27 +343,32 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         __syncthreads();
         // The fused read's current entry is the block's last real one: F_nl = k_nl
         // exactly (every later factor is a padded 1) and D(nl, j) is F_j's suffix
-        // product, so C(nl, j) = F_nl . F_j.
+        // product, so C(nl, j) = F_nl . F_j. Every warp forms that C row and the
+        // entry's X row itself, with no block barrier: lane-partial dots over its
+        // key channels, one transposing butterfly (lane l ends with C(nl, l >> SH)),
+        // then on lane j: X(nl, j) = -beta sum_{m=j..nl-1} C(nl, m) X(m, j),
+        // X(nl, nl) = beta, kept in the warp's own row sxw.
         if (DELTA && cur_here) {
-            for (int j = warp; j < nl; j += nthr / 32) {
-                float pj = 0.f;
+            constexpr int SH = NB == 16 ? 1 : 2;
+            float fn[C::CW], pc[NB];
 #pragma unroll
-                for (int e = 0; e < C::CW; ++e) {
-                    const int c = e * 32 + lane;
-                    pj = fmaf(ff[nl * C::WS + c], ff[j * C::WS + c], pj);
-                }
-                pj = group_sum<32>(pj);
-                if (lane == 0) cm[j] = pj;
+            for (int e = 0; e < C::CW; ++e) fn[e] = ff[nl * C::WS + e * 32 + lane];
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+                pc[j] = 0.f;
+#pragma unroll
+                for (int e = 0; e < C::CW; ++e) pc[j] = fmaf(fn[e], ff[j * C::WS + e * 32 + lane], pc[j]);
             }
-            __syncthreads();
-            // its X row: X(nl, nl) = beta, X(nl, j) = -beta sum_{m=j..nl-1} C(nl, m) X(m, j)
-            if (tid < NB) {
-                const int j = tid;
-                float acc = 0.f;
-                for (int m = j; m < nl; ++m) acc = fmaf(cm[m], sx[m * C::XS + j], acc);
-                sx[nl * C::XS + j] = j < nl ? -sb[nl] * acc : (j == nl ? sb[nl] : 0.f);
+            multi_sum<NB>(pc, lane);
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < NB; ++m) {
+                const float cnm = __shfl_sync(0xffffffffu, pc[0], m << SH);
+                if (lane <= m && m < nl) acc = fmaf(cnm, sx[m * C::XS + lane], acc);
             }
-            __syncthreads();
+            const float bn = sb[nl];
+            if (lane < NB) sxw[warp * C::XS + lane] = lane < nl ? -bn * acc : (lane == nl ? bn : 0.f);
+            __syncwarp();
         }
 
         // 3. this warp's 16 rows: delta in the A-operand layout (split hi + lo).
@@ -411,9 +423,11 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             for (int mt = 0; mt < NT; ++mt) {
 #pragma unroll
                 for (int x = 0; x < 4; ++x) dl[mt][x] = 0.f;
+                const int xr = 8 * mt + g;  // the fused entry's row is the warp's own copy
+                const float *xrow = (cur_here && xr == nl) ? sxw + warp * C::XS : sx + xr * C::XS;
 #pragma unroll
                 for (int kt = 0; kt <= mt; ++kt) {
-                    const float *xp = sx + (8 * mt + g) * C::XS + 8 * kt + t;
+                    const float *xp = xrow + 8 * kt + t;
                     mma3(dl[mt], xh[kt], xl[kt], xp[0], xp[4]);
                 }
             }
