@@ -388,11 +388,12 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         } else {
             // G = S Khat^T, the A fragments from the base tile: a0 = S[g][8s + t],
             // a1 = S[g + 8][8s + t], a2 = S[g][8s + t + 4], a3 = S[g + 8][8s + t + 4].
-            float acc1[NT][4];
+            // (two accumulator sets, even and odd k-steps, halve the dependent chains)
+            float acc1[NT][4], acc2[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int x = 0; x < 4; ++x) acc1[nt][x] = 0.f;
+                for (int x = 0; x < 4; ++x) acc1[nt][x] = acc2[nt][x] = 0.f;
 #pragma unroll
             for (int s = 0; s < KS; ++s) {
                 uint32_t ah[4], al[4];
@@ -403,9 +404,13 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const float *kp = kh + (8 * nt + g) * C::KH + 8 * s + t;
-                    mma3(acc1[nt], ah, al, kp[0], kp[4]);
+                    mma3((s & 1) ? acc2[nt] : acc1[nt], ah, al, kp[0], kp[4]);
                 }
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) acc1[nt][x] += acc2[nt][x];
             // E = V - G in the accumulator layout (rows g, g + 8; entries 8nt + 2t, +1).
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -438,11 +443,20 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         // back to the tile for a following sub-merge, else straight to HBM.
 #pragma unroll 4
         for (int cb = 0; cb < KS; ++cb) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            float dn[NT][4];  // one accumulator per entry tile: independent chains
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int x = 0; x < 4; ++x) dn[nt][x] = 0.f;
                 const float *fp = ff + (8 * nt + t) * C::WS + 8 * cb + g;
-                mma3(d, xh[nt], xl[nt], fp[0], fp[4 * C::WS]);
+                mma3(dn[nt], xh[nt], xl[nt], fp[0], fp[4 * C::WS]);
+            }
+            float d[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                d[x] = dn[0][x];
+#pragma unroll
+                for (int nt = 1; nt < NT; ++nt) d[x] += dn[nt][x];
             }
             const int col = 8 * cb + 2 * t;
             ST *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
