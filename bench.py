@@ -425,14 +425,28 @@ def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
     S = torch.empty(B, H, w.d_v, w.d_k, dtype=host["S0"].dtype, device=dev)
     log = g.Log.allocate(B, H, w.d_k, w.d_v, L, tdt, chan, device=dev, rwkv6=rw)
     names = ("q", "k", "v", "a") if rw else ("q", "k", "v", "beta", "a")
+    # Each token's inputs sit in one pinned staging row (every field 16-byte
+    # aligned), as a caller's input buffer would hold them, so that one copy per
+    # token moves them; the device slots are views of one buffer the same way.
+    fields, row = [], 0
+    for n in names:
+        t0 = host[n][0]
+        nb = t0.numel() * t0.element_size()
+        fields.append((n, row, nb, t0.dtype, tuple(t0.shape)))
+        row += (nb + 15) // 16 * 16
+    packed = torch.empty(w.T, row, dtype=torch.uint8, pin_memory=True)
+    for t in range(w.T):
+        for n, off, nb, dt, shp in fields:
+            packed[t, off:off + nb].view(dt).view(shp).copy_(host[n][t])
     nslot = 3
-    slots = [{n: torch.empty_like(host[n][0], device=dev) for n in names} for _ in range(nslot)]
+    slot_buf = [torch.empty(row, dtype=torch.uint8, device=dev) for _ in range(nslot)]
+    slots = [{n: slot_buf[j][off:off + nb].view(dt).view(shp) for n, off, nb, dt, shp in fields}
+             for j in range(nslot)]
     o_dev = [torch.empty(B, H, w.d_v, dtype=torch.float32, device=dev) for _ in range(nslot)]
     o_host = torch.empty(w.T, B, H, w.d_v, dtype=torch.float32, pin_memory=True)
     S_host = torch.empty_like(host["S0"], pin_memory=True)
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
-    step_in = sum(host[n][0].numel() * host[n][0].element_size() for n in names)
-    h2d_bytes = host["S0"].numel() * host["S0"].element_size() + w.T * step_in
+    h2d_bytes = host["S0"].numel() * host["S0"].element_size() + w.T * row
     d2h_bytes = o_host.numel() * 4 + S_host.numel() * S_host.element_size()
 
     def one():
@@ -450,8 +464,7 @@ def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
             with torch.cuda.stream(h2d):
                 if ev_used[j] is not None:
                     h2d.wait_event(ev_used[j])
-                for n in names:
-                    slots[j][n].copy_(host[n][t], non_blocking=True)
+                slot_buf[j].copy_(packed[t], non_blocking=True)
                 ev_in[j].record(h2d)
             stream.wait_event(ev_in[j])
             if ev_out[j] is not None:
