@@ -400,12 +400,8 @@ static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, 
     constexpr int WARPS = EMAX <= 32 ? 4 : 2;
     auto kern = replay_prep_kernel<IT, DK, DV, KD, EMAX>;
     const size_t smem = (size_t)WARPS * P::BYTES;
-    static bool configured = false;
-    if (!configured && smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
     const long long heads = (long long)p.B * p.H;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((heads + WARPS - 1) / WARPS));

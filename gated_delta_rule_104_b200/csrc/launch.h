@@ -2,7 +2,10 @@
 // kernels. Arguments are already validated when these are called.
 #pragma once
 
+#include <mutex>
+#include <set>
 #include <type_traits>
+#include <utility>
 
 #include "../../include/deltalog.h"
 #include "common.cuh"
@@ -66,6 +69,22 @@ __device__ __forceinline__ bool pool_head(const PoolIdx &pi, int part, long long
     if (part == POOL_APPEND) return c < pi.L - 1;
     if (part == POOL_MERGE_FULL) return c == pi.L - 1;
     return c > 0;  // POOL_FLUSH
+}
+
+// Lets `kern` use `bytes` (> 48 KB) of dynamic shared memory on the current
+// device: set once per (kernel, device), thread-safe; a no-op for 48 KB or less.
+inline cudaError_t allow_smem(const void *kern, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kern, dev})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.insert({kern, dev});
+    return e;
 }
 
 cudaError_t launch_eager(const StepParams &p, cudaStream_t st);

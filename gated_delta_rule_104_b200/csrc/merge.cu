@@ -502,15 +502,8 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
     auto kern = merge_kernel<ST, DK, KD, WC, NB>;
     constexpr int rows = C::ROWS;
     const size_t smem = merge_smem_bytes<ST, DK, NB>();
-    static bool configured = false;
-    if (!configured) {
-        const size_t want = smem;
-        if (want > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
-            if (e != cudaSuccess) return e;
-        }
-        configured = true;
-    }
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
     const long long blocks = (long long)p.B * p.H * (p.dv / rows);
     kern<<<(unsigned)blocks, rows * 2, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.x, lg.L,
                                                    n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
