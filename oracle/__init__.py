@@ -54,7 +54,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         cmd = ["gcc", "-std=c99", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC]
+               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -66,11 +66,14 @@ class CLib:
     def __init__(self, path: str):
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
-        for name, extra in (("oracle_eager", []), ("oracle_deferred", [ctypes.c_int])):
+        for name, extra in (("oracle_eager", []), ("oracle_deferred", [ctypes.c_int]),
+                            ("oracle_deferred_i8", [ctypes.c_int])):
             fn = getattr(lib, name)
             fn.restype = None
             fn.argtypes = ([ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
                            + extra + [dp] * 7)
+        lib.oracle_quantize_i8.restype = None
+        lib.oracle_quantize_i8.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int, dp]
         lib.oracle_abi_version.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -85,16 +88,26 @@ class CLib:
                               _c(S), _c(q), _c(k), _c(v), _c(beta), _c(a), _c(o))
         return o, S
 
-    def deferred(self, S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False):
+    def deferred(self, S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False,
+                 base_i8: bool = False):
         """DeltaLog schedule with log capacity L (merge when full and at the end).
-        Returns (o [T,NH,d_v], S_T)."""
+        ``base_i8``: the base is held in int8 with a scale per row, quantised at
+        the start and after every merge. Returns (o [T,NH,d_v], S_T)."""
         if L < 1:
             raise ValueError("log capacity L must be >= 1")
         S, q, k, v, beta, a, NH, T, dk, dv = _prep(S0, q, k, v, beta, a, channel_decay or rwkv6)
         o = np.zeros((T, NH, dv), dtype=np.float64)
-        self.lib.oracle_deferred(NH, T, dk, dv, _kind(channel_decay, rwkv6), int(L),
-                                 _c(S), _c(q), _c(k), _c(v), _c(beta), _c(a), _c(o))
+        fn = self.lib.oracle_deferred_i8 if base_i8 else self.lib.oracle_deferred
+        fn(NH, T, dk, dv, _kind(channel_decay, rwkv6), int(L),
+           _c(S), _c(q), _c(k), _c(v), _c(beta), _c(a), _c(o))
         return o, S
+
+    def quantize_i8(self, S):
+        """The int8 base's rounding of states [NH, d_v, d_k] (a copy)."""
+        S = np.array(S, dtype=np.float64, order="C", copy=True)
+        NH, dv, dk = S.shape
+        self.lib.oracle_quantize_i8(NH, dk, dv, _c(S))
+        return S
 
 
 def _kind(channel_decay: bool, rwkv6: bool) -> int:
@@ -136,9 +149,14 @@ def eager(S0, q, k, v, beta, a, channel_decay: bool, rwkv6: bool = False):
     return _load().eager(S0, q, k, v, beta, a, channel_decay, rwkv6)
 
 
-def deferred(S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False):
+def deferred(S0, q, k, v, beta, a, channel_decay: bool, L: int, rwkv6: bool = False, base_i8: bool = False):
     """DeltaLog schedule (see ``CLib.deferred``) with the default build."""
-    return _load().deferred(S0, q, k, v, beta, a, channel_decay, L, rwkv6)
+    return _load().deferred(S0, q, k, v, beta, a, channel_decay, L, rwkv6, base_i8)
+
+
+def quantize_i8(S):
+    """The int8 base's per-row rounding (see ``CLib.quantize_i8``)."""
+    return _load().quantize_i8(S)
 
 
 def brute_force(S0, q, k, v, beta, a, channel_decay: bool, rwkv6: bool = False):

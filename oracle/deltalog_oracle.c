@@ -52,6 +52,7 @@
  *   beta  is not read for RWKV6
  *   o     [T, NH, d_v]             out
  */
+#include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -296,5 +297,84 @@ void oracle_deferred(long NH, int T, int dk, int dv, int kind, int L,
     }
 }
 
+/* ----------------------------------------------------- int8 deferred base */
+
+/* Quantisation of a base held in int8 with one scale per state row (a value
+ * channel): scale = max_c |row_c| / 127 and code_c = the nearest integer to
+ * row_c / scale (ties to even), so that row_c becomes code_c * scale; an
+ * all-zero row stays zero. (The low-precision base of the DAMP abstract,
+ * "Decay-Aware Mixed-Precision Recurrent-State Quantization", which stores
+ * recurrent states in INT8: with the deferred schedule the base is written,
+ * and so rounded, only when a merge writes it.) */
+static void quantize_rows_i8(double *S, int dv, int dk)
+{
+    for (int r = 0; r < dv; ++r) {
+        double *row = S + (long)r * dk;
+        double m = 0.0;
+        for (int c = 0; c < dk; ++c)
+            if (fabs(row[c]) > m)
+                m = fabs(row[c]);
+        if (m == 0.0)
+            continue;
+        double scale = m / 127.0;
+        for (int c = 0; c < dk; ++c) {
+            double code = nearbyint(row[c] / scale);
+            if (code > 127.0) code = 127.0;
+            if (code < -127.0) code = -127.0;
+            row[c] = code * scale;
+        }
+    }
+}
+
+/* oracle_deferred with an int8 base: the initial base is quantised, and so is
+ * the base after every merge (the final one included); reads use the base as
+ * stored plus the exact log. */
+void oracle_deferred_i8(long NH, int T, int dk, int dv, int kind, int L,
+                        double *S, const double *q, const double *k, const double *v,
+                        const double *beta, const double *a, double *o)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long h = 0; h < NH; ++h) {
+        double *Sbar = S + h * (long)dv * dk;
+        head_log lg;
+        lg.cap = L; lg.n = 0; lg.dk = dk; lg.dv = dv; lg.delta = kind != 2;
+        lg.k = (double *)malloc(sizeof(double) * (size_t)L * dk);
+        lg.v = (double *)malloc(sizeof(double) * (size_t)L * dv);
+        lg.beta = (double *)malloc(sizeof(double) * (size_t)L);
+        lg.a = (double *)malloc(sizeof(double) * (size_t)L * dk);
+        double *x = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L);
+        quantize_rows_i8(Sbar, dv, dk);
+        for (int t = 0; t < T; ++t) {
+            int e = lg.n;
+            memcpy(lg.k + (long)e * dk, k + ((long)t * NH + h) * dk, sizeof(double) * (size_t)dk);
+            memcpy(lg.v + (long)e * dv, v + ((long)t * NH + h) * dv, sizeof(double) * (size_t)dv);
+            lg.beta[e] = lg.delta ? beta[(long)t * NH + h] : 0.0;
+            for (int j = 0; j < dk; ++j)
+                lg.a[(long)e * dk + j] = decay_at(a, kind, NH, dk, t, h, j);
+            lg.n = e + 1;
+            deferred_read(Sbar, &lg, q + ((long)t * NH + h) * dk,
+                          o + ((long)t * NH + h) * dv, x, s);
+            if (lg.n == L) {
+                deferred_merge(Sbar, &lg);
+                quantize_rows_i8(Sbar, dv, dk);
+            }
+        }
+        if (lg.n) {
+            deferred_merge(Sbar, &lg);
+            quantize_rows_i8(Sbar, dv, dk);
+        }
+        free(s); free(x);
+        free(lg.a); free(lg.beta); free(lg.v); free(lg.k);
+    }
+}
+
+/* The quantisation alone, for the tests: NH heads of d_v x d_k in place. */
+void oracle_quantize_i8(long NH, int dk, int dv, double *S)
+{
+    for (long h = 0; h < NH; ++h)
+        quantize_rows_i8(S + h * (long)dv * dk, dv, dk);
+}
+
 /* Version tag so the Python side can tell a stale build. */
-int oracle_abi_version(void) { return 2; }
+int oracle_abi_version(void) { return 3; }

@@ -43,6 +43,13 @@ MUTATIONS = {
     "rwkv6_read_drops_decay": ("x[j] = ai[j] * x[j];", "x[j] = x[j];"),
     "rwkv6_merge_decays_own_value": ("delta[i] = lg->v[(long)(i - 1) * dv + r];",
                                      "delta[i] = lg->v[(long)(i - 1) * dv + r] * lg->a[(long)(i - 1) * dk];"),
+    # int8 base
+    "i8_rounds_half_away": ("double code = nearbyint(row[c] / scale);", "double code = round(row[c] / scale);"),
+    "i8_scale_128": ("double scale = m / 127.0;", "double scale = m / 128.0;"),
+    "i8_start_unrounded": ("        quantize_rows_i8(Sbar, dv, dk);\n        for (int t = 0; t < T; ++t) {",
+                           "        for (int t = 0; t < T; ++t) {"),
+    "i8_no_rounding_at_merges": ("                deferred_merge(Sbar, &lg);\n                quantize_rows_i8(Sbar, dv, dk);",
+                                 "                deferred_merge(Sbar, &lg);"),
 }
 
 CHECKS = {
@@ -56,6 +63,7 @@ CHECKS = {
     "p7": pins.check_p7,
     "p9": pins.check_p9,
     "p10": pins.check_p10,
+    "p12": pins.check_p12,
 }
 
 
@@ -66,7 +74,7 @@ def build_mutant(tmp_path, old, new):
     path.write_text(src.replace(old, new))
     so = tmp_path / "libmutant.so"
     subprocess.run(["gcc", "-std=c99", "-O1", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
-                    "-w", "-o", str(so), str(path)], check=True)
+                    "-w", "-o", str(so), str(path), "-lm"], check=True)
     return oracle.CLib(str(so))
 
 

@@ -25,7 +25,13 @@ Pins:
      with its special cases a = 1 (plain linear attention) and a = 0;
   P11 the slot pool (per-sequence states in slots, ragged batches): a
      sequence's outputs and state are those of its own recurrence, whatever
-     the other slots do; slots not listed in a step are left unchanged.
+     the other slots do; slots not listed in a step are left unchanged;
+  P12 the int8 base (a scale per state row, max|row| / 127, codes rounded to
+     the nearest integer, ties to even): a hand-worked row; rounding a rounded
+     state changes nothing; with no merge before the end the outputs are the
+     eager ones from the rounded initial state and the final state is that
+     state rounded; with merges every L steps the base is the exact schedule's
+     rounded once per window.
 The mutation test builds copies of the C oracle with planted mistakes and
 checks that these pins reject each of them.
 """
@@ -393,6 +399,46 @@ def check_p11():
 
 def test_p11_slot_pool_is_per_sequence_recurrence(oracle_mod):
     check_p11()
+
+
+# ------------------------------------------------------------------ P12 (int8 base)
+
+def check_p12(impl):
+    # a hand-worked row: max 127 gives scale 1; 62.5 -> 62 and -3.5 -> -4 (ties to
+    # even), 0.4 -> 0; an all-zero row stays zero
+    S = np.array([[[127.0, 62.5, -3.5, 0.4], [0.0, 0.0, 0.0, 0.0], [-2.0, 1.0, 0.5, 0.25]]])
+    # third row: max 2, scale 2/127: codes -127, 63.5 -> 64 (even), 31.75 -> 32, 15.875 -> 16
+    exp = np.array([[[127.0, 62.0, -4.0, 0.0], [0.0, 0.0, 0.0, 0.0],
+                     [-2.0, 64 * 2 / 127, 32 * 2 / 127, 16 * 2 / 127]]])
+    got = impl.quantize_i8(S)
+    assert np.allclose(got, exp, rtol=0, atol=1e-15), got
+    rng = np.random.default_rng(23)
+    R = rng.standard_normal((3, 6, 8))
+    once = impl.quantize_i8(R)
+    assert np.allclose(impl.quantize_i8(once), once, rtol=0, atol=1e-14)
+    codes = once / (np.abs(R).max(axis=-1, keepdims=True) / 127)
+    assert np.allclose(codes, np.round(codes), atol=1e-9) and np.abs(codes).max() <= 127 + 1e-9
+    for chan, rw in ((False, False), (True, False), (True, True)):
+        NH, T, dk, dv = 2, 9, 8, 6
+        S0, q, k, v, beta, a = rand_case(rng, NH, T, dk, dv, chan or rw)
+        # no merge before the end: eager from the rounded start, final state rounded
+        o_e, S_e = impl.eager(impl.quantize_i8(S0), q, k, v, beta, a, chan, rw)
+        o_d, S_d = impl.deferred(S0, q, k, v, beta, a, chan, T + 1, rw, base_i8=True)
+        assert rel(o_d, o_e) < 1e-12 and rel(S_d, impl.quantize_i8(S_e)) < 1e-12, (chan, rw)
+        # merges every L steps: window by window, the exact schedule then a rounding
+        L = 3
+        o_d, S_d = impl.deferred(S0, q, k, v, beta, a, chan, L, rw, base_i8=True)
+        Sw = impl.quantize_i8(S0)
+        for w0 in range(0, T, L):
+            sl = slice(w0, w0 + L)
+            ow, Sw = impl.deferred(Sw, q[sl], k[sl], v[sl], beta[sl], a[sl], chan, L, rw)
+            assert rel(o_d[sl], ow) < 1e-12, (chan, rw, w0)
+            Sw = impl.quantize_i8(Sw)
+        assert rel(S_d, Sw) < 1e-12, (chan, rw)
+
+
+def test_p12_int8_base(oracle_mod):
+    check_p12(oracle_mod)
 
 
 # ------------------------------------------------------------------ inputs
