@@ -57,6 +57,8 @@ def entry_bytes(w: W.Workload) -> int:
 
 
 def state_bytes_head(w: W.Workload) -> int:
+    if w.state_dtype == "i8":  # int8 codes and a float scale per row
+        return w.d_v * w.d_k + 4 * w.d_v
     return w.d_v * w.d_k * (2 if w.state_dtype == "bf16" else 4)
 
 
@@ -265,7 +267,8 @@ def config_block(w, L, args):
              W.RWKV6: "channel, raw-value update without delta correction (RWKV6)"}[w.decay]
     return {"workload": w.name, "decay": decay,
             "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "T": w.T, "L": L,
-            "state_dtype": w.state_dtype, "in_dtype": w.in_dtype,
+            "state_dtype": ("deferred base int8 (row scales), eager " + w.state_dtype)
+            if getattr(args, "base_i8", False) else w.state_dtype, "in_dtype": w.in_dtype,
             "schedule": {"fused": "DeltaLog deferred, merge fused into the L-th step",
                          "unfused": "DeltaLog deferred, separate merge every L steps",
                          "pool": "slot pool, staggered log fills (each step 1/L of the rows merge)"}[args.schedule],
@@ -525,6 +528,8 @@ def main(argv=None):
     ap.add_argument("--workers", type=int, default=0, help="input-generation processes (0: auto)")
     ap.add_argument("--cpu-seconds-per-step", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--base-i8", action="store_true",
+                    help="the deferred legs on an int8 base (DL_I8, rounded from S0 before timing); eager stays fp32")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
@@ -575,7 +580,14 @@ def main(argv=None):
     sampler = ClockSampler(local_rank)
     with sampler:
         rw = w.decay == W.RWKV6
-        if args.schedule == "pool":
+        if args.base_i8 and args.schedule != "pool":
+            S8 = g.I8State.allocate(w.B, w.H, w.d_k, w.d_v)
+            g.dl_state_to_i8(d["S0"].float().contiguous(), S8)
+            log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, tdt, chan, rwkv6=rw)
+            w_def = W.scaled(w, state_dtype="i8")  # byte model of the deferred kernels
+            lau = Launcher(g, w_def, d, S8, log, o_all, args.schedule, stream)
+            S_def = S8
+        elif args.schedule == "pool":
             pool = g.Pool.allocate(w.B, w.H, w.d_k, w.d_v, L, d["S0"].dtype, tdt, chan, rwkv6=rw)
             pool.S.copy_(d["S0"])
             S_def, log = pool.S, pool.log
@@ -600,12 +612,14 @@ def main(argv=None):
 
     value = w.B * w.T / (ms_def / 1000.0) * ws
     main_kind = "pool" if args.schedule == "pool" else "append_read"
-    rf = roofline_for(w, kinds_def, main_kind, peak, peak_note, traffic if main_kind == "append_read" else None)
-    other = {k: roofline_for(w, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != main_kind}
+    wb = W.scaled(w, state_dtype="i8") if args.base_i8 else w
+    measured_traffic = traffic if (main_kind == "append_read" and not args.base_i8) else None
+    rf = roofline_for(wb, kinds_def, main_kind, peak, peak_note, measured_traffic)
+    other = {k: roofline_for(wb, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != main_kind}
     step_time = {k: round(sum(ms for _, ms in v) / args.steps, 3) for k, v in kinds_def.items()}
 
     e2e = None
-    if not args.no_e2e and args.schedule != "pool":
+    if not args.no_e2e and args.schedule != "pool" and not args.base_i8:
         host = {}
         for n in ("S0", "q", "k", "v", "beta", "a"):
             if n == "beta" and w.decay == W.RWKV6:

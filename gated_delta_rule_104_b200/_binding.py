@@ -15,14 +15,14 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdeltalog.so")
 
 DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = range(5)
-DL_F32, DL_BF16 = 0, 1
+DL_F32, DL_BF16, DL_I8 = 0, 1, 2
 DL_DECAY_HEAD, DL_DECAY_CHANNEL, DL_RWKV6 = 0, 1, 2
 DL_MAX_LOG = 64
-ABI_VERSION = 6
+ABI_VERSION = 7
 
 EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read", "dl_log_merge",
            "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_pool_step",
-           "dl_pool_flush", "dl_status_string",
+           "dl_pool_flush", "dl_state_bytes", "dl_state_to_i8", "dl_state_from_i8", "dl_status_string",
            "dl_last_error", "dl_abi_version")
 DL_NOALLOC_WORK_BYTES = 16 << 20
 
@@ -69,10 +69,14 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     pp = ctypes.POINTER(dl_pool)
     lib.dl_pool_step.argtypes = [pp, i, vp, vp, vp, vp, vp, vp, i, f, i, i, i, i, vp]
     lib.dl_pool_flush.argtypes = [pp, i, vp, i, i, i, i, vp]
+    lib.dl_state_bytes.argtypes = [i, i, i, i, i]
+    lib.dl_state_bytes.restype = ctypes.c_size_t
+    lib.dl_state_to_i8.argtypes = [vp, i, vp, i, i, i, i, vp]
+    lib.dl_state_from_i8.argtypes = [vp, vp, i, i, i, i, i, vp]
     lib.dl_log_merge.argtypes = [vp, i, i, lp, i, i, i, i, i, vp]
     for name in ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read",
                  "dl_log_merge", "dl_log_merge_read", "dl_log_append_read_noalloc", "dl_pool_step",
-                 "dl_pool_flush"):
+                 "dl_pool_flush", "dl_state_to_i8", "dl_state_from_i8"):
         getattr(lib, name).restype = ctypes.c_int
     lib.dl_status_string.argtypes = [ctypes.c_int]
     lib.dl_status_string.restype = ctypes.c_char_p
@@ -137,11 +141,67 @@ def _stream(stream) -> int:
     return stream.cuda_stream
 
 
+class I8State:
+    """A deferred base in the int8 layout (DL_I8): one device buffer of
+    B*H*d_v*d_k int8 codes followed by B*H*d_v float32 row scales; an element's
+    value is code * scale. ``codes`` and ``scales`` are views of the buffer."""
+
+    def __init__(self, buf, B: int, H: int, d_k: int, d_v: int):
+        self.buf, self.B, self.H, self.d_k, self.d_v = buf, int(B), int(H), int(d_k), int(d_v)
+        self.shape = (self.B, self.H, self.d_v, self.d_k)
+
+    @classmethod
+    def allocate(cls, B, H, d_k, d_v, device="cuda"):
+        torch = _torch()
+        n = B * H * d_v * d_k
+        return cls(torch.zeros(n + 4 * B * H * d_v, dtype=torch.uint8, device=device), B, H, d_k, d_v)
+
+    @property
+    def codes(self):
+        torch = _torch()
+        n = self.B * self.H * self.d_v * self.d_k
+        return self.buf[:n].view(torch.int8).view(self.shape)
+
+    @property
+    def scales(self):
+        torch = _torch()
+        n = self.B * self.H * self.d_v * self.d_k
+        return self.buf[n:].view(torch.float32).view(self.B, self.H, self.d_v)
+
+    def data_ptr(self) -> int:
+        return self.buf.data_ptr()
+
+
+def dl_state_to_i8(S, out: "I8State", stream=None) -> None:
+    """Round a float32 / bfloat16 state [B,H,d_v,d_k] into ``out``."""
+    B, H, dk, dv = _dims(S)
+    check("dl_state_to_i8", load().dl_state_to_i8(_ptr(S, "S"), _dtype_code(S), out.data_ptr(), B, H, dk, dv,
+                                                  _stream(stream)))
+
+
+def dl_state_from_i8(S8: "I8State", out, stream=None) -> None:
+    """The values of an int8 state into ``out`` (float32 or bfloat16 [B,H,d_v,d_k])."""
+    check("dl_state_from_i8", load().dl_state_from_i8(S8.data_ptr(), _ptr(out, "S"), _dtype_code(out), S8.B, S8.H,
+                                                      S8.d_k, S8.d_v, _stream(stream)))
+
+
 def _dims(S):
+    if isinstance(S, I8State):
+        return S.B, S.H, S.d_k, S.d_v
     if S.dim() != 4:
         raise ValueError("state must be [B, H, d_v, d_k]")
     B, H, dv, dk = S.shape
     return int(B), int(H), int(dk), int(dv)
+
+
+def _state_code(S) -> int:
+    return DL_I8 if isinstance(S, I8State) else _dtype_code(S)
+
+
+def _state_ptr(S, name: str) -> int:
+    if isinstance(S, I8State):
+        return _ptr(S.buf, name)
+    return _ptr(S, name)
 
 
 def _in_dtype(*ts) -> int:
@@ -184,6 +244,8 @@ def dl_rwkv6_decode_step(S, q, k, v, a, o, stream=None) -> None:
 
 
 def _eager(fn, S, q, k, v, beta, a, o, stream, chan):
+    if isinstance(S, I8State):
+        raise TypeError("the eager step takes a float32 or bfloat16 state")
     B, H, dk, dv = _dims(S)
     _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, chan)
     st = _stream(stream)
@@ -247,7 +309,7 @@ def _log_step(fn, S, log, n, q, k, v, beta, a, o, stream):
     _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, log.channel_decay)
     st = _stream(stream)
     ls = log.struct()
-    status = getattr(load(), fn)(_ptr(S, "S_base"), _dtype_code(S), log.kind, ctypes.byref(ls), int(n),
+    status = getattr(load(), fn)(_state_ptr(S, "S_base"), _state_code(S), log.kind, ctypes.byref(ls), int(n),
                                  _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(beta, "beta", log.rwkv6),
                                  _ptr(a, "a"),
                                  _in_dtype(q, k, v, beta, a), _ptr(o, "o"), B, H, dk, dv, st)
@@ -259,7 +321,7 @@ def dl_log_merge(S_base, log: Log, n: int, stream=None) -> None:
     B, H, dk, dv = _dims(S_base)
     st = _stream(stream)
     ls = log.struct()
-    status = load().dl_log_merge(_ptr(S_base, "S_base"), _dtype_code(S_base), log.kind, ctypes.byref(ls),
+    status = load().dl_log_merge(_state_ptr(S_base, "S_base"), _state_code(S_base), log.kind, ctypes.byref(ls),
                                  int(n), B, H, dk, dv, st)
     check("dl_log_merge", status)
 
@@ -285,26 +347,37 @@ class Pool:
 
     def __init__(self, S, log: Log, n, status=None):
         self.S, self.log, self.n, self.status = S, log, n, status
-        self.P = int(S.shape[0])
+        self.P = int(S.shape[0])  # (S may be an I8State: an int8 pool)
 
     @classmethod
     def allocate(cls, P, H, d_k, d_v, L, s_dtype, in_dtype, channel_decay, rwkv6: bool = False, device="cuda"):
+        """``s_dtype``: torch.float32, torch.bfloat16, or torch.int8 for an int8 pool (DL_I8)."""
         torch = _torch()
-        S = torch.zeros(P, H, d_v, d_k, dtype=s_dtype, device=device)
+        if s_dtype == torch.int8:
+            S = I8State.allocate(P, H, d_k, d_v, device=device)
+        else:
+            S = torch.zeros(P, H, d_v, d_k, dtype=s_dtype, device=device)
         log = Log.allocate(P, H, d_k, d_v, L, in_dtype, channel_decay, device=device, rwkv6=rwkv6)
         n = torch.zeros(P, dtype=torch.int32, device=device)
         status = torch.zeros(1, dtype=torch.int32, device=device)
         return cls(S, log, n, status)
 
     def reset(self, slot: int, S0) -> None:
-        """Start a new sequence in ``slot`` from state S0 [H, d_v, d_k] (stream-ordered copies)."""
-        self.S[slot].copy_(S0)
+        """Start a new sequence in ``slot`` from state S0 [H, d_v, d_k] (stream-ordered copies;
+        an int8 pool takes S0 rounded to its layout)."""
+        if isinstance(self.S, I8State):
+            tmp = I8State.allocate(1, self.S.H, self.S.d_k, self.S.d_v, device=self.S.buf.device)
+            dl_state_to_i8(S0.reshape(1, *S0.shape).contiguous(), tmp)
+            self.S.codes[slot].copy_(tmp.codes[0])
+            self.S.scales[slot].copy_(tmp.scales[0])
+        else:
+            self.S[slot].copy_(S0)
         self.n[slot] = 0
 
     def struct(self) -> dl_pool:
         if self.n.dtype != _torch().int32:
             raise TypeError("pool.n must be int32")
-        return dl_pool(_ptr(self.S, "pool.S"), _dtype_code(self.S), self.P, _ptr(self.n, "pool.n"),
+        return dl_pool(_state_ptr(self.S, "pool.S"), _state_code(self.S), self.P, _ptr(self.n, "pool.n"),
                        _ptr(self.status, "pool.status", True), self.log.struct())
 
 
@@ -320,7 +393,7 @@ def dl_pool_step(pool: Pool, slot, q, k, v, beta, a, o, stream=None) -> None:
     (inputs and o are [B,H,...]); each row appends or, on its L-th entry,
     merges, following its own log count."""
     B, H, dk = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
-    dv = int(pool.S.shape[2])
+    dv = int(pool.S.shape[2])  # (an I8State has .shape too)
     _check_shapes(B, H, dk, dv, q, k, v, beta, a, o, pool.log.channel_decay)
     ps = pool.struct()
     status = load().dl_pool_step(ctypes.byref(ps), pool.log.kind, _slots(slot, B), _ptr(q, "q"), _ptr(k, "k"),

@@ -26,6 +26,12 @@ dl_status ok() {
 
 size_t elem_size(dl_dtype t) { return t == DL_BF16 ? 2 : 4; }
 bool valid_dtype(int t) { return t == DL_F32 || t == DL_BF16; }
+bool valid_state_dtype(int t) { return t == DL_F32 || t == DL_BF16 || t == DL_I8; }
+// Bytes of BH heads of d_v x d_k state (DL_I8: codes, then a float scale per row).
+size_t state_bytes(dl_dtype t, size_t bh, int dk, int dv) {
+    if (t == DL_I8) return bh * dv * dk + bh * dv * sizeof(float);
+    return bh * dv * dk * elem_size(t);
+}
 bool valid_decay(int t) { return t == DL_DECAY_HEAD || t == DL_DECAY_CHANNEL || t == DL_RWKV6; }
 
 struct Buf {
@@ -66,7 +72,7 @@ dl_status check_overlap(const Buf *writers, int nw, const Buf *all, int na) {
 dl_status check_dims(int B, int H, int dk, int dv, int s_dt, int in_dt) {
     if (B < 1 || H < 1) return fail(DL_ERR_INVALID_ARG, "B and H must be >= 1 (got B=%d, H=%d)", B, H);
     if ((long long)B * H > (1LL << 26)) return fail(DL_ERR_UNSUPPORTED, "B*H=%lld exceeds 2^26", (long long)B * H);
-    if (!valid_dtype(s_dt)) return fail(DL_ERR_INVALID_ARG, "unknown state dtype %d", s_dt);
+    if (!valid_state_dtype(s_dt)) return fail(DL_ERR_INVALID_ARG, "unknown state dtype %d", s_dt);
     if (!valid_dtype(in_dt)) return fail(DL_ERR_INVALID_ARG, "unknown input dtype %d", in_dt);
     if (dk != 64 && dk != 128) return fail(DL_ERR_UNSUPPORTED, "d_k=%d not in {64, 128}", dk);
     if (dv != 64 && dv != 128 && dv != 256) return fail(DL_ERR_UNSUPPORTED, "d_v=%d not in {64, 128, 256}", dv);
@@ -79,7 +85,7 @@ int step_bufs(Buf *out, const void *S, const char *sname, dl_dtype s_dt, const v
               int H, int dk, int dv, int kind) {
     const size_t bh = (size_t)B * H, is = elem_size(in_dt);
     const bool chan = kind != DL_DECAY_HEAD;
-    out[0] = {sname, S, bh * dv * dk * elem_size(s_dt), 16};
+    out[0] = {sname, S, state_bytes(s_dt, bh, dk, dv), 16};
     out[1] = {"q", q, bh * dk * is, 16};
     out[2] = {"k", k, bh * dk * is, 16};
     out[3] = {"v", v, bh * dv * is, 16};
@@ -115,6 +121,7 @@ dl_status eager_step(void *S, dl_dtype s_dt, const void *q, const void *k, const
                      cudaStream_t stream, int kind) {
     dl_status s = check_dims(B, H, dk, dv, s_dt, in_dt);
     if (s != DL_OK) return s;
+    if (s_dt == DL_I8) return fail(DL_ERR_UNSUPPORTED, "the eager step takes a float32 or bfloat16 state");
     Buf b[7];
     int nb = step_bufs(b, S, "S", s_dt, q, k, v, beta, a, in_dt, o, B, H, dk, dv, kind);
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
@@ -182,7 +189,7 @@ dl_status dl_log_merge(void *S_base, dl_dtype s_dtype, dl_decay kind, const dl_l
     if (!valid_decay(kind)) return fail(DL_ERR_INVALID_ARG, "unknown decay kind %d", (int)kind);
     if (!log) return fail(DL_ERR_INVALID_ARG, "log is a null pointer");
     Buf b[6];
-    b[0] = {"S_base", S_base, (size_t)B * H * d_v * d_k * elem_size(s_dtype), 16};
+    b[0] = {"S_base", S_base, state_bytes(s_dtype, (size_t)B * H, d_k, d_v), 16};
     if ((s = check_log(log, b + 1, log->dtype, B, H, d_k, d_v, kind)) != DL_OK) return s;
     if ((s = check_bufs(b, 6)) != DL_OK) return s;
     if (n < 1 || n > log->L) return fail(DL_ERR_INVALID_ARG, "merge needs 1 <= n <= L (n=%d, L=%d)", n, log->L);
@@ -271,7 +278,7 @@ dl_status dl_pool_step(const dl_pool *pool, dl_decay kind, const int *slot, cons
     if (pool) step_bufs(b, pool->S, "pool.S", pool->s_dtype, q, k, v, beta, a, in_dtype, o, B, H, d_k, d_v, kind);
     dl_status s = pool_checks(pool, kind, slot, in_dtype, B, H, d_k, d_v, b, nb);
     if (s != DL_OK) return s;
-    b[0].bytes = (size_t)pool->P * H * d_v * d_k * elem_size(pool->s_dtype);  // the whole pool
+    b[0].bytes = state_bytes(pool->s_dtype, (size_t)pool->P * H, d_k, d_v);  // the whole pool
     const size_t need = dl::read_work_bytes(B, H, d_k, d_v);
     b[nb++] = {"log.work", pool->log.work, need, 16};
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
@@ -302,7 +309,7 @@ dl_status dl_pool_flush(const dl_pool *pool, dl_decay kind, const int *slot, int
                         cudaStream_t stream) {
     Buf b[10];
     int nb = 1;
-    if (pool) b[0] = {"pool.S", pool->S, (size_t)pool->P * H * d_v * d_k * elem_size(pool->s_dtype), 16};
+    if (pool) b[0] = {"pool.S", pool->S, state_bytes(pool->s_dtype, (size_t)pool->P * H, d_k, d_v), 16};
     dl_status s = pool_checks(pool, kind, slot, pool ? pool->log.dtype : DL_F32, B, H, d_k, d_v, b, nb);
     if (s != DL_OK) return s;
     if ((s = check_bufs(b, nb)) != DL_OK) return s;
@@ -322,6 +329,36 @@ dl_status dl_pool_flush(const dl_pool *pool, dl_decay kind, const int *slot, int
     cudaError_t e = dl::launch_merge(p, lg, lg0->L - 1, false, stream, pi, dl::POOL_FLUSH);
     if (e == cudaSuccess) e = dl::launch_pool_counts(pi, B, false, stream);
     return cuda_status(e, "pool flush launch");
+}
+
+size_t dl_state_bytes(dl_dtype s_dtype, int B, int H, int d_k, int d_v) {
+    if (B < 1 || H < 1 || d_k < 1 || d_v < 1 || !valid_state_dtype(s_dtype)) return 0;
+    return state_bytes(s_dtype, (size_t)B * H, d_k, d_v);
+}
+
+static dl_status convert_checks(const void *S, dl_dtype s_dtype, const void *S_i8, int B, int H, int d_k, int d_v) {
+    dl_status s = check_dims(B, H, d_k, d_v, s_dtype, DL_F32);
+    if (s != DL_OK) return s;
+    if (s_dtype == DL_I8) return fail(DL_ERR_INVALID_ARG, "the other state must be float32 or bfloat16");
+    const size_t bh = (size_t)B * H;
+    Buf b[2] = {{"S", S, state_bytes(s_dtype, bh, d_k, d_v), 16}, {"S_i8", S_i8, state_bytes(DL_I8, bh, d_k, d_v), 16}};
+    if ((s = check_bufs(b, 2)) != DL_OK) return s;
+    return check_overlap(b, 2, b, 2);
+}
+
+dl_status dl_state_to_i8(const void *S, dl_dtype s_dtype, void *S_i8, int B, int H, int d_k, int d_v,
+                         cudaStream_t stream) {
+    dl_status s = convert_checks(S, s_dtype, S_i8, B, H, d_k, d_v);
+    if (s != DL_OK) return s;
+    return cuda_status(dl::launch_to_i8(S, s_dtype, S_i8, (long long)B * H * d_v, d_k, stream), "to-int8 launch");
+}
+
+dl_status dl_state_from_i8(const void *S_i8, void *S, dl_dtype s_dtype, int B, int H, int d_k, int d_v,
+                           cudaStream_t stream) {
+    dl_status s = convert_checks(S, s_dtype, S_i8, B, H, d_k, d_v);
+    if (s != DL_OK) return s;
+    return cuda_status(dl::launch_from_i8(S_i8, S, s_dtype, (long long)B * H * d_v, d_k, stream),
+                       "from-int8 launch");
 }
 
 const char *dl_status_string(dl_status s) {

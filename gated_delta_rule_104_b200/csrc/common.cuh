@@ -100,6 +100,34 @@ template <> struct StateVec<bf16> {
     }
 };
 
+// int8 state codes (a deferred base of type DL_I8): 16 per 16-byte slice,
+// widened here; the row scale is applied by the caller.
+template <> struct StateVec<int8_t> {
+    static constexpr int N = 16;
+    __device__ __forceinline__ static void unpack(const uint4 &r, float (&x)[16]) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[4 * i + j] = (float)(int8_t)(w[i] >> (8 * j));
+    }
+};
+
+// The int8 state's row rounding: scale = max|value| / 127, code = the nearest
+// integer to value / scale (ties to even) in [-127, 127]; an all-zero row has
+// scale 0 and every code 0.
+__device__ __forceinline__ float i8_scale(float row_max) { return row_max / 127.f; }
+__device__ __forceinline__ int i8_code(float x, float scale) {
+    if (scale == 0.f) return 0;
+    const int c = __float2int_rn(x / scale);
+    return c > 127 ? 127 : (c < -127 ? -127 : c);
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+    return x;
+}
+
 // Streaming 16-byte state accesses: the state is touched once per step, so
 // it is read and written with the evict-first (".cs") cache hint and kept out
 // of L1, leaving L2 to the small per-step operands.

@@ -331,7 +331,7 @@ struct DecodeShape {
 template <class ST, int DK, int DV>
 __global__ void __launch_bounds__(256)
 append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work, float *__restrict__ o,
-                     long long num_units, PoolIdx pool) {
+                     long long num_units, PoolIdx pool, const float *__restrict__ row_scale) {
     using C = DecodeShape<ST, DK>;
     constexpr int VEC = C::VEC;
     static_assert(DV % C::UNIT == 0, "unit divides d_v");
@@ -346,13 +346,20 @@ append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work
     int n_unused = 0;
     const bool active = unit < num_units && pool_head(pool, POOL_APPEND, head, shead, n_unused);
 
-    // D3 operands: the base rows first (read only, streamed).
+    // D3 operands: the base rows first (read only, streamed); an int8 base's
+    // row scales with them.
+    constexpr bool Q8 = std::is_same<ST, int8_t>::value;
     uint4 raw[C::R];
+    float rsc[Q8 ? C::R : 1];
     if (active) {
         const uint64_t stream = l2_policy_stream();
         const ST *src = Sbar + (shead * DV + rin0 + sub) * DK + col;
 #pragma unroll
         for (int r = 0; r < C::R; ++r) raw[r] = ld_ro_hint(src + (long long)r * C::RPW * DK, stream);
+        if constexpr (Q8) {
+#pragma unroll
+            for (int r = 0; r < C::R; ++r) rsc[r] = row_scale[shead * DV + rin0 + r * C::RPW + sub];
+        }
     }
     pdl_wait();  // replay_prep's (x_0, w) are complete and visible from here on
     if (!active) return;
@@ -367,6 +374,7 @@ append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc = fmaf(s[e], xv[e], acc);
         acc = group_sum<C::G>(acc);
+        if constexpr (Q8) acc *= rsc[r];
         const int rr = rin0 + r * C::RPW + sub;
         if ((lane % C::G) == 0) o[head * DV + rr] = acc + wk[DK + rr];
     }
@@ -389,8 +397,14 @@ static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // an int8 base's row scales follow its codes (all the state's heads: the pool's, or B*H)
+    const long long state_heads = pool.slot ? (long long)pool.P * pool.H : (long long)p.B * p.H;
+    const float *row_scale = std::is_same<ST, int8_t>::value
+                                 ? reinterpret_cast<const float *>(static_cast<const int8_t *>(p.S) +
+                                                                   state_heads * DV * DK)
+                                 : nullptr;
     return cudaLaunchKernelEx(&cfg, append_decode_kernel<ST, DK, DV>, static_cast<const ST *>(p.S), work, p.o,
-                              units, pool);
+                              units, pool, row_scale);
 }
 
 template <class IT, int DK, int DV, int KD, int EMAX>
@@ -432,7 +446,8 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
         else if (lg.L <= 32) e = launch_prep<IT, DK, DV, KD, 32>(p, lg, n, work, st, pool);
         else e = launch_prep<IT, DK, DV, KD, 64>(p, lg, n, work, st, pool);
         if (e != cudaSuccess) return e;
-        e = launch_decode<ST, DK, DV>(p, work, st, pool);
+        if (p.s_dt == DL_I8) e = launch_decode<int8_t, DK, DV>(p, work, st, pool);
+        else e = launch_decode<ST, DK, DV>(p, work, st, pool);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     });

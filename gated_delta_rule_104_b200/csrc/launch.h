@@ -98,6 +98,10 @@ cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg,
 // entry, and then o = S_new q) into the base.
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,
                          cudaStream_t st, const PoolIdx &pool = PoolIdx{}, int part = POOL_MERGE_FULL);
+// State conversions to / from the int8 layout (rows = B*H*d_v rows of d_k).
+cudaError_t launch_to_i8(const void *S, dl_dtype s_dt, void *S_i8, long long rows, int dk, cudaStream_t st);
+cudaError_t launch_from_i8(const void *S_i8, void *S, dl_dtype s_dt, long long rows, int dk, cudaStream_t st);
+
 // Pool bookkeeping after a step (advance = true: count + 1, or 0 after the L-th
 // entry merged) or a flush (advance = false: count = 0), for each batch row's slot.
 cudaError_t launch_pool_counts(const PoolIdx &pool, int B, bool advance, cudaStream_t st);

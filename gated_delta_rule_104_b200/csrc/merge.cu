@@ -116,18 +116,24 @@ struct BaseTile {
 };
 
 // Shared memory (bytes) of one block for NB-entry sub-merges:
-//   tile [ROWS][DK] of ST (swizzled base rows), then floats:
+//   tile [ROWS][DK] of the tile type (swizzled base rows: float for an int8
+//   base, else the state type), then floats:
 //   kh [NB][KH] keys, turned into Khat in place
 //   ff [NB][WS] F (channel decay: holds the decays until F replaces them)
 //   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
 //   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
 //   sxw [4][XS] each warp's copy of the fused entry's X row
+//   int8 base only: raw [ROWS][DK] codes, scl [ROWS] row scales, wsc [4][16]
+//   the new row scales of each warp's rows
 template <class ST, int DK, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
     using C = MergeShape<DK, NB>;
+    constexpr bool Q8 = std::is_same<ST, int8_t>::value;
+    using TT = typename std::conditional<Q8, float, ST>::type;
     const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK +
                           (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS + 4 * (size_t)C::XS;
-    return (size_t)C::ROWS * DK * sizeof(ST) + floats * sizeof(float);
+    const size_t q8 = Q8 ? (size_t)C::ROWS * DK + (size_t)C::ROWS * 4 + 64 * 4 : 0;
+    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8;
 }
 
 __device__ __forceinline__ float2 ld_tile2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
@@ -171,9 +177,13 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
              const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_x,
              int L, int n_log, const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
              const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV, bool bf,
-             PoolIdx pool, int part) {
+             PoolIdx pool, int part, float *__restrict__ i8_scales) {
     using C = MergeShape<DK, NB>;
-    using TL = BaseTile<ST, DK>;
+    // An int8 base (row scales in i8_scales) is widened into a float tile, merged
+    // as a float base, and its rows rounded back to int8 when they are stored.
+    constexpr bool Q8 = std::is_same<ST, int8_t>::value;
+    using TT = typename std::conditional<Q8, float, ST>::type;
+    using TL = BaseTile<TT, DK>;
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
     constexpr int KS = DK / 8;   // k-steps of the first product / column tiles of the second
     constexpr int NT = NB / 8;   // entry tiles
@@ -181,7 +191,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     constexpr int nthr = 2 * ROWS;  // 4 warps, 16 rows each
 
     extern __shared__ float4 smem_raw[];
-    ST *tile = reinterpret_cast<ST *>(smem_raw);
+    TT *tile = reinterpret_cast<TT *>(smem_raw);
     float *kh = reinterpret_cast<float *>(tile + ROWS * DK);
     float *ff = kh + NB * C::KH;
     float *fa = ff + NB * C::WS;
@@ -191,6 +201,9 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     float *sb = sx + NB * C::XS;
     float *sv = sb + round4(NB);
     float *sxw = sv + NB * C::VS;
+    int8_t *raw = reinterpret_cast<int8_t *>(sxw + 4 * C::XS);  // int8 base only
+    float *scl = reinterpret_cast<float *>(raw + ROWS * DK);
+    float *wsc = scl + ROWS;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;  // fragment coordinates
@@ -209,12 +222,23 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     // block's loads are issued (those come first, so that they do not queue
     // behind the tile); the tile lands while the key side is worked out.
     auto fetch_tile = [&]() {
-        constexpr int CPR = DK / TL::CE;  // chunks per row
-        const ST *src = S + (shead * DV + row0) * DK;
+        if constexpr (Q8) {  // the codes (unswizzled) and the row scales
+            constexpr int CPR = DK / 16;
+            const int8_t *src = S + (shead * DV + row0) * DK;
 #pragma unroll 4
-        for (int u = tid; u < ROWS * CPR; u += nthr) {
-            const int r = u / CPR, ch = u % CPR;
-            cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
+            for (int u = tid; u < ROWS * CPR; u += nthr) {
+                const int r = u / CPR, ch = u % CPR;
+                cp_async16(raw + r * DK + ch * 16, src + (long long)r * DK + ch * 16);
+            }
+            if (tid < ROWS / 4) cp_async16(scl + 4 * tid, i8_scales + shead * DV + row0 + 4 * tid);
+        } else {
+            constexpr int CPR = DK / TL::CE;  // chunks per row
+            const ST *src = S + (shead * DV + row0) * DK;
+#pragma unroll 4
+            for (int u = tid; u < ROWS * CPR; u += nthr) {
+                const int r = u / CPR, ch = u % CPR;
+                cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
+            }
         }
         cp_async_commit();
     };
@@ -341,6 +365,19 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         }
         cp_async_wait_all();  // this thread's share of the base tile has landed
         __syncthreads();
+        if constexpr (Q8) {
+            if (b0 == 0) {  // codes * scale into the float tile, 4 at a time
+                for (int u = tid; u < ROWS * DK / 4; u += nthr) {
+                    const int r = u / (DK / 4), c4 = (u % (DK / 4)) * 4;
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(raw + r * DK + c4);
+                    const float sc = scl[r];
+                    *reinterpret_cast<float4 *>(tile + TL::off(r, c4)) =
+                        make_float4((float)(int8_t)w * sc, (float)(int8_t)(w >> 8) * sc,
+                                    (float)(int8_t)(w >> 16) * sc, (float)(int8_t)(w >> 24) * sc);
+                }
+                __syncthreads();
+            }
+        }
         // The fused read's current entry is the block's last real one: F_nl = k_nl
         // exactly (every later factor is a padded 1) and D(nl, j) is F_j's suffix
         // product, so C(nl, j) = F_nl . F_j. Every warp forms that C row and the
@@ -440,7 +477,9 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
         }
         // S <- S o gamma + delta F, one 16 x 8 column tile at a time (rows g, g + 8;
         // columns 8c + 2t, 8c + 2t + 1 of the accumulator layout): from the tile,
-        // back to the tile for a following sub-merge, else straight to HBM.
+        // back to the tile for a following sub-merge (or, for an int8 base, for the
+        // rounding below), else straight to HBM.
+        float rmax0 = 0.f, rmax1 = 0.f;  // int8 base: |value| maxima of rows g, g + 8 (this lane's columns)
 #pragma unroll 4
         for (int cb = 0; cb < KS; ++cb) {
             float dn[NT][4];  // one accumulator per entry tile: independent chains
@@ -459,7 +498,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 for (int nt = 1; nt < NT; ++nt) d[x] += dn[nt][x];
             }
             const int col = 8 * cb + 2 * t;
-            ST *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
+            TT *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
             const float2 r0 = ld_tile2(p0), r1 = ld_tile2(p1);
             float s00 = r0.x, s01 = r0.y, s10 = r1.x, s11 = r1.y;
             const float2 gv = *reinterpret_cast<const float2 *>(gn + col);
@@ -472,12 +511,46 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 oacc[0] = fmaf(s00, qv.x, fmaf(s01, qv.y, oacc[0]));
                 oacc[1] = fmaf(s10, qv.x, fmaf(s11, qv.y, oacc[1]));
             }
-            if (last) {
+            if constexpr (Q8) {
+                st_tile2(p0, s00, s01);
+                st_tile2(p1, s10, s11);
+                rmax0 = fmaxf(rmax0, fmaxf(fabsf(s00), fabsf(s01)));
+                rmax1 = fmaxf(rmax1, fmaxf(fabsf(s10), fabsf(s11)));
+            } else if (last) {
                 st_state2(Sw + g * DK + col, s00, s01);
                 st_state2(Sw + (g + 8) * DK + col, s10, s11);
             } else {
                 st_tile2(p0, s00, s01);
                 st_tile2(p1, s10, s11);
+            }
+        }
+        if constexpr (Q8) {
+            if (last) {  // round the warp's 16 rows to int8 (one scale per row) and store them
+#pragma unroll
+                for (int off = 1; off <= 2; off <<= 1) {  // the quad holds a row's columns
+                    rmax0 = fmaxf(rmax0, __shfl_xor_sync(0xffffffffu, rmax0, off));
+                    rmax1 = fmaxf(rmax1, __shfl_xor_sync(0xffffffffu, rmax1, off));
+                }
+                if (t == 0) {
+                    wsc[warp * 16 + g] = i8_scale(rmax0);
+                    wsc[warp * 16 + g + 8] = i8_scale(rmax1);
+                }
+                __syncwarp();
+                constexpr int CPR = DK / 16;  // 16-code chunks per row
+                for (int i = lane; i < 16 * CPR; i += 32) {
+                    const int rl = i / CPR, c0 = (i % CPR) * 16;
+                    const float sc = wsc[warp * 16 + rl];
+                    uint32_t wd[4];
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd) {
+                        const float4 x = *reinterpret_cast<const float4 *>(tile + TL::off(tr + rl, c0 + 4 * qd));
+                        wd[qd] = (uint32_t)(i8_code(x.x, sc) & 0xff) | ((uint32_t)(i8_code(x.y, sc) & 0xff) << 8) |
+                                 ((uint32_t)(i8_code(x.z, sc) & 0xff) << 16) |
+                                 ((uint32_t)(i8_code(x.w, sc) & 0xff) << 24);
+                    }
+                    st_stream(Sw + rl * DK + c0, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+                }
+                if (lane < 16) i8_scales[shead * DV + row0 + tr + lane] = wsc[warp * 16 + lane];
             }
         }
         __syncthreads();  // the next entry block reuses the shared buffers
@@ -505,9 +578,14 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)p.B * p.H * (p.dv / rows);
+    // an int8 base's row scales follow its codes (all the state's heads: the pool's, or B*H)
+    const long long state_heads = pool.slot ? (long long)pool.P * pool.H : (long long)p.B * p.H;
+    float *i8_scales = std::is_same<ST, int8_t>::value
+                           ? reinterpret_cast<float *>(static_cast<int8_t *>(p.S) + state_heads * p.dv * DK)
+                           : nullptr;
     kern<<<(unsigned)blocks, rows * 2, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.x, lg.L,
                                                    n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
-                                                   p.in_dt == DL_BF16, pool, part);
+                                                   p.in_dt == DL_BF16, pool, part, i8_scales);
     return cudaGetLastError();
 }
 
@@ -543,6 +621,7 @@ cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bo
         return go(st_t, std::integral_constant<int, 128>{});
     };
     if (p.s_dt == DL_BF16) return with_dk(bf16{});
+    if (p.s_dt == DL_I8) return with_dk(int8_t{});
     return with_dk(float{});
 }
 

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 6
+#define DL_ABI_VERSION 7
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -73,7 +73,18 @@ typedef enum {
     DL_ERR_CUDA = 4         /* the kernel launch failed (cudaGetLastError) */
 } dl_status;
 
-typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
+/* Element types. DL_I8 is a state type only, and only for a deferred base
+ * (dl_log_append_read, dl_log_merge, dl_log_merge_read, the no-alloc read and
+ * the pool): the base is held as int8 codes with one fp32 scale per state row
+ * (a value channel), packed in one buffer -- B*H*d_v*d_k int8 codes, row-major
+ * as for the other types, then B*H*d_v fp32 scales (dl_state_bytes) -- and an
+ * element's value is code * scale. Every merge re-rounds the rows it writes:
+ * scale = max|row| / 127, code = the nearest integer to value / scale, ties to
+ * even (an all-zero row stays zero). (The low-precision base of the DAMP
+ * abstract, "Decay-Aware Mixed-Precision Recurrent-State Quantization": with
+ * the deferred schedule the base is rounded once per merge, not every step.)
+ * The eager steps take DL_F32 or DL_BF16 only (DL_I8 -> DL_ERR_UNSUPPORTED). */
+typedef enum { DL_F32 = 0, DL_BF16 = 1, DL_I8 = 2 } dl_dtype;
 
 /* The model's update rule: its decay shape and whether the delta-rule
  * correction applies. */
@@ -272,6 +283,21 @@ dl_status dl_pool_step(const dl_pool *pool, dl_decay kind, const int *slot,
  * that sequence (for a sequence that ends, or a state handed elsewhere). */
 dl_status dl_pool_flush(const dl_pool *pool, dl_decay kind, const int *slot,
                         int B, int H, int d_k, int d_v, cudaStream_t stream);
+
+/* Bytes of a [B, H, d_v, d_k] state of element type s_dtype (for DL_I8 the
+ * codes and the row scales); 0 for a bad argument. */
+size_t dl_state_bytes(dl_dtype s_dtype, int B, int H, int d_k, int d_v);
+
+/* Round a state into the int8 layout of DL_I8 (scale per row, ties to even):
+ *   S     [B, H, d_v, d_k] s_dtype (DL_F32 or DL_BF16), read
+ *   S_i8  dl_state_bytes(DL_I8, ...) bytes, written; 16-byte aligned, no overlap */
+dl_status dl_state_to_i8(const void *S, dl_dtype s_dtype, void *S_i8,
+                         int B, int H, int d_k, int d_v, cudaStream_t stream);
+
+/* The values of an int8 state (code * scale) into S of type s_dtype (DL_F32 or
+ * DL_BF16, rounded to nearest-even for DL_BF16). */
+dl_status dl_state_from_i8(const void *S_i8, void *S, dl_dtype s_dtype,
+                           int B, int H, int d_k, int d_v, cudaStream_t stream);
 
 /* Static text for a status code. */
 const char *dl_status_string(dl_status s);

@@ -71,6 +71,20 @@ def test_eager_argument_checks(lib, fn):
     assert step(lib, fn, q=addr(0) + 1024) == b.DL_ERR_INVALID_ARG      # S written over an input
 
 
+def test_int8_state_is_a_deferred_base_only(lib):
+    # the eager step refuses an int8 state before any launch; sizes of the packed layout
+    for fn in ("dl_gdn_decode_step", "dl_kda_decode_step"):
+        assert step(lib, fn, s_dt=b.DL_I8) == b.DL_ERR_UNSUPPORTED
+    assert lib.dl_state_bytes(b.DL_I8, 2, 3, 128, 64) == 2 * 3 * 64 * (128 + 4)
+    assert lib.dl_state_bytes(b.DL_BF16, 2, 3, 128, 64) == 2 * 3 * 64 * 128 * 2
+    assert lib.dl_state_bytes(7, 2, 3, 128, 64) == 0
+    # conversions: the other state must be float32 / bfloat16, and the two must not overlap
+    assert lib.dl_state_to_i8(addr(0), b.DL_I8, addr(1), 2, 3, 128, 64, None) == b.DL_ERR_INVALID_ARG
+    assert lib.dl_state_to_i8(addr(0), b.DL_F32, addr(0) + 1024, 2, 3, 128, 64, None) == b.DL_ERR_INVALID_ARG
+    assert "overlaps" in lib.dl_last_error().decode()
+    assert lib.dl_state_from_i8(addr(1), None, b.DL_F32, 2, 3, 128, 64, None) == b.DL_ERR_INVALID_ARG
+
+
 def test_scalar_operands_need_only_element_alignment(lib):
     # beta (and a head-wise a) may sit at any element boundary; the check that
     # fails here is a deliberate misaligned q, reached only after beta passed.

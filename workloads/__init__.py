@@ -70,6 +70,8 @@ class Workload:
         return self.B * self.H
 
     def state_bytes(self) -> int:
+        if self.state_dtype == "i8":  # int8 codes and a float scale per row
+            return self.heads * self.d_v * (self.d_k + 4)
         return self.heads * self.d_v * self.d_k * (4 if self.state_dtype == "f32" else 2)
 
 
