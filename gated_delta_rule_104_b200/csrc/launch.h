@@ -2,6 +2,7 @@
 // kernels. Arguments are already validated when these are called.
 #pragma once
 
+#include <algorithm>
 #include <mutex>
 #include <set>
 #include <type_traits>

@@ -75,13 +75,34 @@ __device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ah)[4], con
     mma_tf32(d, ah, b0h, b1h);
 }
 
-__device__ __forceinline__ float ld_state(const float *p) { return *p; }
-__device__ __forceinline__ float ld_state(const bf16 *p) { return to_f(*p); }
-__device__ __forceinline__ void st_state2(float *p, float x, float y) {
-    __stcs(reinterpret_cast<float2 *>(p), make_float2(x, y));
+// Four consecutive state elements (16 bytes of fp32, 8 of bf16), widened to fp32.
+__device__ __forceinline__ float4 ld_tile4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld_tile4(const bf16 *p) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
 }
-__device__ __forceinline__ void st_state2(bf16 *p, float x, float y) {
-    __stcs(reinterpret_cast<unsigned int *>(p), pack_bf2(x, y));
+__device__ __forceinline__ void st_tile4(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
+__device__ __forceinline__ void st_tile4(bf16 *p, float4 x) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf2(x.x, x.y), pack_bf2(x.z, x.w));
+}
+__device__ __forceinline__ void st_state4(float *p, float4 x) { __stcs(reinterpret_cast<float4 *>(p), x); }
+__device__ __forceinline__ void st_state4(bf16 *p, float4 x) {
+    __stcs(reinterpret_cast<uint2 *>(p), make_uint2(pack_bf2(x.x, x.y), pack_bf2(x.z, x.w)));
+}
+
+// Column order of the two products. Both are sums over, or maps of, the key
+// columns, so any order that the state, Khat and F share gives the same
+// result. Within each group of 16 columns [16j, 16j + 16):
+//  - G's k-steps 2j + h (h = 0, 1) take fragment positions t and t + 4 to
+//    columns 16j + 4t + 2h and 16j + 4t + 2h + 1;
+//  - the update's column tiles 2j + h take accumulator column n to
+//    16j + 4 (n / 2) + 2h + n mod 2.
+// Either way lane (g, t) holds columns 16j + 4t .. 16j + 4t + 3 of its rows, so
+// the base tile, Khat, gamma, q and the merged rows move 16 bytes per access.
+// F is stored in the order the update's B fragments read it: column c at
+// position f_pos(c) = 16j + 8h + n of its group.
+__device__ __forceinline__ int f_pos(int c) {
+    return (c & ~15) | (((c >> 1) & 1) << 3) | (((c >> 2) & 3) << 1) | (c & 1);
 }
 
 // ------------------------------------------------------------------ layout
@@ -91,26 +112,33 @@ __host__ __device__ constexpr size_t round4(size_t x) { return (x + 3) & ~(size_
 template <int DK, int NB>
 struct MergeShape {
     static constexpr int ROWS = 64;     // base rows per block: 4 warps of 16
-    static constexpr int KH = DK + 4;   // Khat row stride (conflict-free B-fragment reads)
+    static constexpr int KH = DK;       // Khat row stride (no padding: the rows are swizzled, kof)
     static constexpr int WS = DK + 8;   // F row stride (conflict-free B-fragment reads)
     static constexpr int XS = NB + 4;   // X row stride (conflict-free B-fragment reads)
     static constexpr int VS = ROWS + 4; // value row stride (conflict-free accumulator-layout reads)
     static constexpr int CW = DK / 32;  // key channels per lane (warp-wide dots)
+    // Khat element (i, c): the 16-byte chunks of row i XOR-swizzled by 4 (i mod 2),
+    // so that a 16-byte B-fragment read (rows 2m and 2m + 1 in one 8-lane phase)
+    // hits every bank; a pair of chunks 2u, 2u + 1 stays adjacent.
+    __device__ static __forceinline__ int kof(int i, int c) {
+        return i * KH + ((((c >> 2) ^ ((i & 1) << 2)) << 2) | (c & 3));
+    }
 };
 
-// The block's base rows in shared memory: ROWS x DK elements of the state
-// type, row-major with the 16-byte chunks of row r XOR-swizzled by
-// f(r) = 2 (r mod 4) + (r / 4 mod 2), a permutation of 0..7. Over the 8 rows
-// of a fragment f takes every value, so an 8-row x 4-column operand read hits
-// 32 distinct banks; over each 4-row half it takes distinct pairs f / 2, so
-// the accumulator-layout accesses (4 rows x 8 consecutive fp32 per half warp)
-// do too. No padding.
+// The block's base rows in shared memory: ROWS x DK elements of the tile
+// type, row-major, with the 16-byte chunks of row r XOR-swizzled by f(r). Every
+// access is lane (g, t) moving columns 16j + 4t .. + 3 of row g (or g + 8):
+//  - fp32: one 128-byte phase is 8 lanes, rows r, r + 1 with 4 chunks each;
+//    f(r) = 4 (r mod 2) puts the two rows in opposite halves of the banks;
+//  - bf16: one phase is 16 lanes of 8 bytes, rows r .. r + 3 with a chunk pair
+//    each; f(r) = 2 (r mod 4) puts the four pairs on distinct banks.
+// No padding.
 template <class ST, int DK>
 struct BaseTile {
     static constexpr int CE = 16 / (int)sizeof(ST);  // elements per 16-byte chunk
     static_assert(DK / CE >= 8, "swizzle spans 8 chunks");
     __device__ static __forceinline__ int off(int r, int c) {
-        const int f = ((r & 3) << 1) | ((r >> 2) & 1);
+        const int f = CE == 4 ? (r & 1) << 2 : (r & 3) << 1;
         return r * DK + (((c / CE) ^ f) * CE) + (c % CE);
     }
 };
@@ -123,8 +151,11 @@ struct BaseTile {
 //   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
 //   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
 //   sxw [4][XS] each warp's copy of the fused entry's X row
-//   int8 base only: raw [ROWS][DK] codes, scl [ROWS] row scales, wsc [4][16]
-//   the new row scales of each warp's rows
+//   xw [4] (after the int8 arrays, if any) a compact grid's unit ballots
+//   int8 base only: scl [ROWS] row scales, wsc [4][16] the new row scales of
+//   each warp's rows; the codes [ROWS][DK] land in the last ROWS * DK bytes of
+//   the float tile and are read out into registers before it is widened over
+//   them (no separate code buffer: four blocks per SM, as for a float base)
 template <class ST, int DK, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
     using C = MergeShape<DK, NB>;
@@ -132,20 +163,8 @@ __host__ __device__ constexpr size_t merge_smem_bytes() {
     using TT = typename std::conditional<Q8, float, ST>::type;
     const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK +
                           (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS + 4 * (size_t)C::XS;
-    const size_t q8 = Q8 ? (size_t)C::ROWS * DK + (size_t)C::ROWS * 4 + 64 * 4 : 0;
-    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8;
-}
-
-__device__ __forceinline__ float2 ld_tile2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
-__device__ __forceinline__ float2 ld_tile2(const bf16 *p) {
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
-    return make_float2(bf_lo(w), bf_hi(w));
-}
-__device__ __forceinline__ void st_tile2(float *p, float x, float y) {
-    *reinterpret_cast<float2 *>(p) = make_float2(x, y);
-}
-__device__ __forceinline__ void st_tile2(bf16 *p, float x, float y) {
-    *reinterpret_cast<uint32_t *>(p) = pack_bf2(x, y);
+    const size_t q8 = Q8 ? (size_t)C::ROWS * 4 + 64 * 4 : 0;
+    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8 + 16;  // + 16: xw
 }
 
 // Accumulator layout (rows g, g + 8; columns 8i + 2t, 8i + 2t + 1) to A-operand
@@ -177,7 +196,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
              const void *__restrict__ log_b, const void *__restrict__ log_a, const float *__restrict__ log_x,
              int L, int n_log, const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
              const void *__restrict__ beta, const void *__restrict__ a, float *__restrict__ o, int DV, bool bf,
-             PoolIdx pool, int part, float *__restrict__ i8_scales) {
+             PoolIdx pool, int part, float *__restrict__ i8_scales, long long units) {
     using C = MergeShape<DK, NB>;
     // An int8 base (row scales in i8_scales) is widened into a float tile, merged
     // as a float base, and its rows rounded back to int8 when they are stored.
@@ -185,7 +204,6 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     using TT = typename std::conditional<Q8, float, ST>::type;
     using TL = BaseTile<TT, DK>;
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
-    constexpr int KS = DK / 8;   // k-steps of the first product / column tiles of the second
     constexpr int NT = NB / 8;   // entry tiles
     constexpr int ROWS = C::ROWS;
     constexpr int nthr = 2 * ROWS;  // 4 warps, 16 rows each
@@ -201,368 +219,458 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     float *sb = sx + NB * C::XS;
     float *sv = sb + round4(NB);
     float *sxw = sv + NB * C::VS;
-    int8_t *raw = reinterpret_cast<int8_t *>(sxw + 4 * C::XS);  // int8 base only
-    float *scl = reinterpret_cast<float *>(raw + ROWS * DK);
+    // int8 base only: the codes at the end of the (float) tile, the scales after sxw
+    int8_t *raw = reinterpret_cast<int8_t *>(tile) + (size_t)ROWS * DK * (sizeof(TT) - 1);
+    float *scl = sxw + 4 * C::XS;
     float *wsc = scl + ROWS;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;  // fragment coordinates
     const int tiles = DV / ROWS;
-    const long long head = blockIdx.x / tiles;  // batch head (this step's inputs, o)
-    const int row0 = (blockIdx.x % tiles) * ROWS;
-    long long shead;                            // state / log head
     pdl_launch_dependents();  // a pool step's append part (other slots) may start beside this grid
-    if (!pool_head(pool, part, head, shead, n_log)) return;  // the whole block: no barrier passed yet
-    const int NTOT = n_log + (WITH_CUR ? 1 : 0);
-    const long long lrow = shead * L;
-    ST *Sw = S + (shead * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
-    const int tr = 16 * warp;                           // and their first row in the tile
 
-    // The block's base rows, fetched by cp.async right after the first entry
-    // block's loads are issued (those come first, so that they do not queue
-    // behind the tile); the tile lands while the key side is worked out.
-    auto fetch_tile = [&]() {
-        if constexpr (Q8) {  // the codes (unswizzled) and the row scales
-            constexpr int CPR = DK / 16;
-            const int8_t *src = S + (shead * DV + row0) * DK;
-#pragma unroll 4
-            for (int u = tid; u < ROWS * CPR; u += nthr) {
-                const int r = u / CPR, ch = u % CPR;
-                cp_async16(raw + r * DK + ch * 16, src + (long long)r * DK + ch * 16);
-            }
-            if (tid < ROWS / 4) cp_async16(scl + 4 * tid, i8_scales + shead * DV + row0 + 4 * tid);
-        } else {
-            constexpr int CPR = DK / TL::CE;  // chunks per row
-            const ST *src = S + (shead * DV + row0) * DK;
-#pragma unroll 4
-            for (int u = tid; u < ROWS * CPR; u += nthr) {
-                const int r = u / CPR, ch = u % CPR;
-                cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
-            }
-        }
-        cp_async_commit();
-    };
-
-    float oacc[2] = {0.f, 0.f};  // o for rows g and g + 8 (fused read), partial over this lane's columns
-    for (int b0 = 0; b0 < NTOT; b0 += NB) {
-        const int nb = NTOT - b0 < NB ? NTOT - b0 : NB;
-        const int nl = (n_log - b0 < nb ? n_log - b0 : nb);  // of which from the log (the rest: this step)
-        const bool cur_here = WITH_CUR && nl < nb;
-        const bool last = b0 + NB >= NTOT;
-
-        // 1. entries b0 .. b0+nb-1 (log entries, then the fused read's own); all
-        // global loads are issued before the first shared store.
-        auto stage = [&](auto tag) {
-            using IT = decltype(tag);
-            constexpr int E = 16 / (int)sizeof(IT);
-            constexpr int KC = DK / E;
-            constexpr int KN = (NB * KC + 127) / 128;       // >= 128 threads per block
-            constexpr int VN = (NB * 128 / E + 127) / 128;  // rows <= 128
-            const int VC = ROWS / E;
-            float kx[KN][E], ax[KN][E], vx[VN][E], qx[E];
-            (void)ax;
-            (void)qx;
-            const bool qload = WITH_CUR && b0 == 0 && tid < KC;  // this step's q, with the first block
-            if (qload) load_vec<E>(static_cast<const IT *>(q) + head * DK + tid * E, qx);
-            auto key_src = [&](const void *logp, const void *cur, int r) -> const IT * {
-                return r < nl ? static_cast<const IT *>(logp) + (lrow + b0 + r) * DK
-                              : static_cast<const IT *>(cur) + head * DK;
-            };
-#pragma unroll
-            for (int u = 0; u < KN; ++u) {
-                const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
-                if (c < NB * KC && r < nb) {
-                    load_vec<E>(key_src(log_k, k, r) + col, kx[u]);
-                    if constexpr (CHAN) load_vec<E>(key_src(log_a, a, r) + col, ax[u]);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < VN; ++u) {
-                const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
-                if (c < NB * VC && r < nb) {
-                    const IT *src = r < nl ? static_cast<const IT *>(log_v) + (lrow + b0 + r) * DV
-                                           : static_cast<const IT *>(v) + head * DV;
-                    load_vec<E>(src + row0 + col, vx[u]);
-                }
-            }
-            float bsc = 0.f, asc = 1.f;
-            (void)asc;
-            if (tid < nb) {
-                if constexpr (DELTA)
-                    bsc = tid < nl ? to_f(static_cast<const IT *>(log_b)[lrow + b0 + tid])
-                                   : to_f(static_cast<const IT *>(beta)[head]);
-                if constexpr (!CHAN)
-                    asc = tid < nl ? to_f(static_cast<const IT *>(log_a)[lrow + b0 + tid])
-                                   : to_f(static_cast<const IT *>(a)[head]);
-            }
-            // X(i, j), j <= i, of the logged entries (the block's diagonal block; the
-            // current entry's row is formed below; padded entries are zero)
-            constexpr int CN = (NB * NB + 127) / 128;
-            float cval[CN];
-#pragma unroll
-            for (int u = 0; u < CN; ++u) {
-                const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
-                cval[u] = (DELTA && idx < NB * NB && cj <= ci && ci < nl) ? log_x[(lrow + b0 + ci) * L + b0 + cj]
-                                                                            : 0.f;
-            }
-            if (b0 == 0) fetch_tile();
-            auto put = [](float *dst, const float *x, bool real, float pad) {
-#pragma unroll
-                for (int e = 0; e < E; e += 4)
-                    *reinterpret_cast<float4 *>(dst + e) =
-                        real ? make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]) : make_float4(pad, pad, pad, pad);
-            };
-#pragma unroll
-            for (int u = 0; u < KN; ++u) {
-                const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
-                if (c < NB * KC) {  // padded entries: k = 0, a = 1
-                    put(kh + r * C::KH + col, kx[u], r < nb, 0.f);
-                    if constexpr (CHAN) put(ff + r * C::WS + col, ax[u], r < nb, 1.f);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < VN; ++u) {
-                const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
-                if (c < NB * VC) put(sv + r * C::VS + col, vx[u], r < nb, 0.f);
-            }
-            if (tid < NB) {
-                sb[tid] = bsc;  // 0 for padded entries
-                if constexpr (!CHAN) fa[tid] = asc;
-            }
-            if (qload) put(sq + tid * E, qx, true, 0.f);
-#pragma unroll
-            for (int u = 0; u < CN; ++u) {
-                const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
-                if (idx < NB * NB && !(cur_here && ci == nl)) sx[ci * C::XS + cj] = cval[u];
-            }
-        };
-        if (bf) stage(bf16{});
-        else stage(float{});
+    // A unit is (batch head, tile of ROWS rows); one unit per block, except in a
+    // compact grid (a pool step's merge part, where only the slots on their L-th
+    // entry merge). There block b owns units b, b + G, b + 2G, ... (G = gridDim.x):
+    // it checks them 128 at a time, one per thread, keeps each warp's ballot of
+    // those that merge in shared memory (xw[0..3], the batch in xw[4]), and merges
+    // them one after another. The walk's state lives in shared memory, so that
+    // nothing of it stays in registers across a merge.
+    const bool compact = units != (long long)gridDim.x;
+    uint32_t *xw = reinterpret_cast<uint32_t *>(Q8 ? wsc + 64 : sxw + 4 * C::XS);
+    if (compact) {
+        if (tid < 4) xw[tid] = 0u;
+        if (tid == 0) xw[4] = 0xffffffffu;  // batch -1: none checked yet
         __syncthreads();
-
-        // 2. per key channel, in place: Khat_i = gamma_i o k_i, gamma,
-        // F_j = k_j o D(NB-1, j) (padded entries have a = 1, so D(NB-1, j) = D(nb-1, j)).
-        for (int c = tid; c < DK; c += nthr) {
-            float ac[NB], kc[NB];
-#pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                ac[i] = CHAN ? ff[i * C::WS + c] : fa[i];
-                kc[i] = kh[i * C::KH + c];
-            }
-            float gm = 1.f;
-#pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                gm *= ac[i];
-                kh[i * C::KH + c] = gm * kc[i];
-            }
-            gn[c] = gm;
-            float f = 1.f;
-#pragma unroll
-            for (int j = NB - 1; j >= 0; --j) {
-                ff[j * C::WS + c] = kc[j] * f;
-                f *= ac[j];
-            }
-        }
-        cp_async_wait_all();  // this thread's share of the base tile has landed
-        __syncthreads();
-        if constexpr (Q8) {
-            if (b0 == 0) {  // codes * scale into the float tile, 4 at a time
-                for (int u = tid; u < ROWS * DK / 4; u += nthr) {
-                    const int r = u / (DK / 4), c4 = (u % (DK / 4)) * 4;
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(raw + r * DK + c4);
-                    const float sc = scl[r];
-                    *reinterpret_cast<float4 *>(tile + TL::off(r, c4)) =
-                        make_float4((float)(int8_t)w * sc, (float)(int8_t)(w >> 8) * sc,
-                                    (float)(int8_t)(w >> 16) * sc, (float)(int8_t)(w >> 24) * sc);
-                }
-                __syncthreads();
-            }
-        }
-        // The fused read's current entry is the block's last real one: F_nl = k_nl
-        // exactly (every later factor is a padded 1) and D(nl, j) is F_j's suffix
-        // product, so C(nl, j) = F_nl . F_j. Every warp forms that C row and the
-        // entry's X row itself, with no block barrier: lane-partial dots over its
-        // key channels, one transposing butterfly (lane l ends with C(nl, l >> SH)),
-        // then on lane j: X(nl, j) = -beta sum_{m=j..nl-1} C(nl, m) X(m, j),
-        // X(nl, nl) = beta, kept in the warp's own row sxw.
-        if (DELTA && cur_here) {
-            constexpr int SH = NB == 16 ? 1 : 2;
-            float fn[C::CW], pc[NB];
-#pragma unroll
-            for (int e = 0; e < C::CW; ++e) fn[e] = ff[nl * C::WS + e * 32 + lane];
-#pragma unroll
-            for (int j = 0; j < NB; ++j) {
-                pc[j] = 0.f;
-#pragma unroll
-                for (int e = 0; e < C::CW; ++e) pc[j] = fmaf(fn[e], ff[j * C::WS + e * 32 + lane], pc[j]);
-            }
-            multi_sum<NB>(pc, lane);
-            float acc = 0.f;
-#pragma unroll
-            for (int m = 0; m < NB; ++m) {
-                const float cnm = __shfl_sync(0xffffffffu, pc[0], m << SH);
-                if (lane <= m && m < nl) acc = fmaf(cnm, sx[m * C::XS + lane], acc);
-            }
-            const float bn = sb[nl];
-            if (lane < NB) sxw[warp * C::XS + lane] = lane < nl ? -bn * acc : (lane == nl ? bn : 0.f);
-            __syncwarp();
-        }
-
-        // 3. this warp's 16 rows: delta in the A-operand layout (split hi + lo).
-        __syncwarp();  // a previous block's rows, written by this warp, are visible
-        const int rg = 16 * warp + g;
-        uint32_t xh[NT][4], xl[NT][4];
-        if constexpr (!DELTA) {
-            // delta = V, read straight into the operand layout (entries 8nt + t, + 4).
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int i0 = 8 * nt + t;
-                split_tf32(sv[i0 * C::VS + rg], xh[nt][0], xl[nt][0]);
-                split_tf32(sv[i0 * C::VS + rg + 8], xh[nt][1], xl[nt][1]);
-                split_tf32(sv[(i0 + 4) * C::VS + rg], xh[nt][2], xl[nt][2]);
-                split_tf32(sv[(i0 + 4) * C::VS + rg + 8], xh[nt][3], xl[nt][3]);
-            }
-        } else {
-            // G = S Khat^T, the A fragments from the base tile: a0 = S[g][8s + t],
-            // a1 = S[g + 8][8s + t], a2 = S[g][8s + t + 4], a3 = S[g + 8][8s + t + 4].
-            // (two accumulator sets, even and odd k-steps, halve the dependent chains)
-            float acc1[NT][4], acc2[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int x = 0; x < 4; ++x) acc1[nt][x] = acc2[nt][x] = 0.f;
-#pragma unroll
-            for (int s = 0; s < KS; ++s) {
-                uint32_t ah[4], al[4];
-                split_tf32(ld_state(tile + TL::off(tr + g, 8 * s + t)), ah[0], al[0]);
-                split_tf32(ld_state(tile + TL::off(tr + g + 8, 8 * s + t)), ah[1], al[1]);
-                split_tf32(ld_state(tile + TL::off(tr + g, 8 * s + t + 4)), ah[2], al[2]);
-                split_tf32(ld_state(tile + TL::off(tr + g + 8, 8 * s + t + 4)), ah[3], al[3]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const float *kp = kh + (8 * nt + g) * C::KH + 8 * s + t;
-                    mma3((s & 1) ? acc2[nt] : acc1[nt], ah, al, kp[0], kp[4]);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int x = 0; x < 4; ++x) acc1[nt][x] += acc2[nt][x];
-            // E = V - G in the accumulator layout (rows g, g + 8; entries 8nt + 2t, +1).
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int i0 = 8 * nt + 2 * t;
-                acc1[nt][0] = sv[i0 * C::VS + rg] - acc1[nt][0];
-                acc1[nt][1] = sv[(i0 + 1) * C::VS + rg] - acc1[nt][1];
-                acc1[nt][2] = sv[i0 * C::VS + rg + 8] - acc1[nt][2];
-                acc1[nt][3] = sv[(i0 + 1) * C::VS + rg + 8] - acc1[nt][3];
-            }
-            // delta = E X^T (the triangular solve, one small product per warp; X is
-            // lower triangular, so tiles above the diagonal are skipped).
-            acc_to_operand<NT>(acc1, xh, xl, lane);
-            float dl[NT][4];
-#pragma unroll
-            for (int mt = 0; mt < NT; ++mt) {
-#pragma unroll
-                for (int x = 0; x < 4; ++x) dl[mt][x] = 0.f;
-                const int xr = 8 * mt + g;  // the fused entry's row is the warp's own copy
-                const float *xrow = (cur_here && xr == nl) ? sxw + warp * C::XS : sx + xr * C::XS;
-#pragma unroll
-                for (int kt = 0; kt <= mt; ++kt) {
-                    const float *xp = xrow + 8 * kt + t;
-                    mma3(dl[mt], xh[kt], xl[kt], xp[0], xp[4]);
-                }
-            }
-            acc_to_operand<NT>(dl, xh, xl, lane);
-        }
-        // S <- S o gamma + delta F, one 16 x 8 column tile at a time (rows g, g + 8;
-        // columns 8c + 2t, 8c + 2t + 1 of the accumulator layout): from the tile,
-        // back to the tile for a following sub-merge (or, for an int8 base, for the
-        // rounding below), else straight to HBM.
-        float rmax0 = 0.f, rmax1 = 0.f;  // int8 base: |value| maxima of rows g, g + 8 (this lane's columns)
-#pragma unroll 4
-        for (int cb = 0; cb < KS; ++cb) {
-            float dn[NT][4];  // one accumulator per entry tile: independent chains
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int x = 0; x < 4; ++x) dn[nt][x] = 0.f;
-                const float *fp = ff + (8 * nt + t) * C::WS + 8 * cb + g;
-                mma3(dn[nt], xh[nt], xl[nt], fp[0], fp[4 * C::WS]);
-            }
-            float d[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                d[x] = dn[0][x];
-#pragma unroll
-                for (int nt = 1; nt < NT; ++nt) d[x] += dn[nt][x];
-            }
-            const int col = 8 * cb + 2 * t;
-            TT *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
-            const float2 r0 = ld_tile2(p0), r1 = ld_tile2(p1);
-            float s00 = r0.x, s01 = r0.y, s10 = r1.x, s11 = r1.y;
-            const float2 gv = *reinterpret_cast<const float2 *>(gn + col);
-            s00 = fmaf(s00, gv.x, d[0]);
-            s01 = fmaf(s01, gv.y, d[1]);
-            s10 = fmaf(s10, gv.x, d[2]);
-            s11 = fmaf(s11, gv.y, d[3]);
-            if (WITH_CUR && last) {
-                const float2 qv = *reinterpret_cast<const float2 *>(sq + col);
-                oacc[0] = fmaf(s00, qv.x, fmaf(s01, qv.y, oacc[0]));
-                oacc[1] = fmaf(s10, qv.x, fmaf(s11, qv.y, oacc[1]));
-            }
-            if constexpr (Q8) {
-                st_tile2(p0, s00, s01);
-                st_tile2(p1, s10, s11);
-                rmax0 = fmaxf(rmax0, fmaxf(fabsf(s00), fabsf(s01)));
-                rmax1 = fmaxf(rmax1, fmaxf(fabsf(s10), fabsf(s11)));
-            } else if (last) {
-                st_state2(Sw + g * DK + col, s00, s01);
-                st_state2(Sw + (g + 8) * DK + col, s10, s11);
-            } else {
-                st_tile2(p0, s00, s01);
-                st_tile2(p1, s10, s11);
-            }
-        }
-        if constexpr (Q8) {
-            if (last) {  // round the warp's 16 rows to int8 (one scale per row) and store them
-#pragma unroll
-                for (int off = 1; off <= 2; off <<= 1) {  // the quad holds a row's columns
-                    rmax0 = fmaxf(rmax0, __shfl_xor_sync(0xffffffffu, rmax0, off));
-                    rmax1 = fmaxf(rmax1, __shfl_xor_sync(0xffffffffu, rmax1, off));
-                }
-                if (t == 0) {
-                    wsc[warp * 16 + g] = i8_scale(rmax0);
-                    wsc[warp * 16 + g + 8] = i8_scale(rmax1);
-                }
-                __syncwarp();
-                constexpr int CPR = DK / 16;  // 16-code chunks per row
-                for (int i = lane; i < 16 * CPR; i += 32) {
-                    const int rl = i / CPR, c0 = (i % CPR) * 16;
-                    const float sc = wsc[warp * 16 + rl];
-                    uint32_t wd[4];
-#pragma unroll
-                    for (int qd = 0; qd < 4; ++qd) {
-                        const float4 x = *reinterpret_cast<const float4 *>(tile + TL::off(tr + rl, c0 + 4 * qd));
-                        wd[qd] = (uint32_t)(i8_code(x.x, sc) & 0xff) | ((uint32_t)(i8_code(x.y, sc) & 0xff) << 8) |
-                                 ((uint32_t)(i8_code(x.z, sc) & 0xff) << 16) |
-                                 ((uint32_t)(i8_code(x.w, sc) & 0xff) << 24);
-                    }
-                    st_stream(Sw + rl * DK + c0, make_uint4(wd[0], wd[1], wd[2], wd[3]));
-                }
-                if (lane < 16) i8_scales[shead * DV + row0 + tr + lane] = wsc[warp * 16 + lane];
-            }
-        }
-        __syncthreads();  // the next entry block reuses the shared buffers
     }
-
-    if constexpr (WITH_CUR) {
-        oacc[0] = group_sum<4>(oacc[0]);
-        oacc[1] = group_sum<4>(oacc[1]);
-        if (t == 0) {
-            o[head * DV + row0 + 16 * warp + g] = oacc[0];
-            o[head * DV + row0 + 16 * warp + g + 8] = oacc[1];
+    for (;;) {
+        long long unit = blockIdx.x;
+        if (compact) {
+            int batch = (int)xw[4];
+            uint32_t m[4] = {xw[0], xw[1], xw[2], xw[3]};
+            bool done = false;
+            while ((m[0] | m[1] | m[2] | m[3]) == 0u) {  // the next batch with a unit to merge
+                ++batch;
+                const long long u0 = (long long)blockIdx.x + (long long)batch * nthr * gridDim.x;
+                if (u0 >= units) {
+                    done = true;
+                    break;
+                }
+                const long long u = u0 + (long long)tid * gridDim.x;
+                bool mine = false;
+                if (u < units) {
+                    long long sh;
+                    int nn = n_log;
+                    mine = pool_head(pool, part, u / tiles, sh, nn);
+                }
+                const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+                __syncthreads();  // every thread has read the previous words
+                if (lane == 0) xw[warp] = bal;
+                __syncthreads();
+#pragma unroll
+                for (int w = 0; w < 4; ++w) m[w] = xw[w];
+            }
+            if (done) break;
+            const int w = m[0] ? 0 : m[1] ? 1 : m[2] ? 2 : 3;
+            const int bit = __ffs(m[w]) - 1;
+            unit = (long long)blockIdx.x + ((long long)batch * nthr + 32 * w + bit) * gridDim.x;
+            __syncthreads();  // every thread has read the words before they change
+            if (tid == 0) {
+                xw[w] = m[w] & (m[w] - 1u);
+                xw[4] = (uint32_t)batch;
+            }
         }
+        const long long head = unit / tiles;  // batch head (this step's inputs, o)
+        const int row0 = (int)(unit % tiles) * ROWS;
+        long long shead;                      // state / log head
+        int n_log_u = n_log;                  // this unit's log count (a pool slot's own)
+        // a unit that is not this launch's to merge (a pool slot at another count)
+        // is left by the whole block before any barrier
+        if (pool_head(pool, part, head, shead, n_log_u)) {
+            const int n_log = n_log_u;
+            const int NTOT = n_log + (WITH_CUR ? 1 : 0);
+            const long long lrow = shead * L;
+            ST *Sw = S + (shead * DV + row0 + 16 * warp) * DK;  // this warp's 16 rows
+            const int tr = 16 * warp;                           // and their first row in the tile
+
+            // The block's base rows, fetched by cp.async right after the first entry
+            // block's loads are issued (those come first, so that they do not queue
+            // behind the tile); the tile lands while the key side is worked out.
+            auto fetch_tile = [&]() {
+                if constexpr (Q8) {  // the codes (unswizzled) and the row scales
+                    constexpr int CPR = DK / 16;
+                    const int8_t *src = S + (shead * DV + row0) * DK;
+#pragma unroll 4
+                    for (int u = tid; u < ROWS * CPR; u += nthr) {
+                        const int r = u / CPR, ch = u % CPR;
+                        cp_async16(raw + r * DK + ch * 16, src + (long long)r * DK + ch * 16);
+                    }
+                    if (tid < ROWS / 4) cp_async16(scl + 4 * tid, i8_scales + shead * DV + row0 + 4 * tid);
+                } else {
+                    constexpr int CPR = DK / TL::CE;  // chunks per row
+                    const ST *src = S + (shead * DV + row0) * DK;
+#pragma unroll 4
+                    for (int u = tid; u < ROWS * CPR; u += nthr) {
+                        const int r = u / CPR, ch = u % CPR;
+                        cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
+                    }
+                }
+                cp_async_commit();
+            };
+
+            float oacc[2] = {0.f, 0.f};  // o for rows g and g + 8 (fused read), partial over this lane's columns
+            for (int b0 = 0; b0 < NTOT; b0 += NB) {
+                const int nb = NTOT - b0 < NB ? NTOT - b0 : NB;
+                const int nl = (n_log - b0 < nb ? n_log - b0 : nb);  // of which from the log (the rest: this step)
+                const bool cur_here = WITH_CUR && nl < nb;
+                const bool last = b0 + NB >= NTOT;
+
+                // 1. entries b0 .. b0+nb-1 (log entries, then the fused read's own); all
+                // global loads are issued before the first shared store.
+                auto stage = [&](auto tag) {
+                    using IT = decltype(tag);
+                    constexpr int E = 16 / (int)sizeof(IT);
+                    constexpr int KC = DK / E;
+                    constexpr int KN = (NB * KC + 127) / 128;       // >= 128 threads per block
+                    constexpr int VN = (NB * 128 / E + 127) / 128;  // rows <= 128
+                    const int VC = ROWS / E;
+                    float kx[KN][E], ax[KN][E], vx[VN][E], qx[E];
+                    (void)ax;
+                    (void)qx;
+                    const bool qload = WITH_CUR && b0 == 0 && tid < KC;  // this step's q, with the first block
+                    if (qload) load_vec<E>(static_cast<const IT *>(q) + head * DK + tid * E, qx);
+                    auto key_src = [&](const void *logp, const void *cur, int r) -> const IT * {
+                        return r < nl ? static_cast<const IT *>(logp) + (lrow + b0 + r) * DK
+                                      : static_cast<const IT *>(cur) + head * DK;
+                    };
+#pragma unroll
+                    for (int u = 0; u < KN; ++u) {
+                        const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
+                        if (c < NB * KC && r < nb) {
+                            load_vec<E>(key_src(log_k, k, r) + col, kx[u]);
+                            if constexpr (CHAN) load_vec<E>(key_src(log_a, a, r) + col, ax[u]);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < VN; ++u) {
+                        const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
+                        if (c < NB * VC && r < nb) {
+                            const IT *src = r < nl ? static_cast<const IT *>(log_v) + (lrow + b0 + r) * DV
+                                                   : static_cast<const IT *>(v) + head * DV;
+                            load_vec<E>(src + row0 + col, vx[u]);
+                        }
+                    }
+                    float bsc = 0.f, asc = 1.f;
+                    (void)asc;
+                    if (tid < nb) {
+                        if constexpr (DELTA)
+                            bsc = tid < nl ? to_f(static_cast<const IT *>(log_b)[lrow + b0 + tid])
+                                           : to_f(static_cast<const IT *>(beta)[head]);
+                        if constexpr (!CHAN)
+                            asc = tid < nl ? to_f(static_cast<const IT *>(log_a)[lrow + b0 + tid])
+                                           : to_f(static_cast<const IT *>(a)[head]);
+                    }
+                    // X(i, j), j <= i, of the logged entries (the block's diagonal block; the
+                    // current entry's row is formed below; padded entries are zero)
+                    constexpr int CN = (NB * NB + 127) / 128;
+                    float cval[CN];
+#pragma unroll
+                    for (int u = 0; u < CN; ++u) {
+                        const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
+                        cval[u] = (DELTA && idx < NB * NB && cj <= ci && ci < nl)
+                                      ? log_x[(lrow + b0 + ci) * L + b0 + cj]
+                                                                                    : 0.f;
+                    }
+                    if (b0 == 0) fetch_tile();
+                    auto put = [](float *dst, const float *x, bool real, float pad) {
+#pragma unroll
+                        for (int e = 0; e < E; e += 4)
+                            *reinterpret_cast<float4 *>(dst + e) =
+                                real ? make_float4(x[e], x[e + 1], x[e + 2], x[e + 3])
+                                     : make_float4(pad, pad, pad, pad);
+                    };
+#pragma unroll
+                    for (int u = 0; u < KN; ++u) {
+                        const int c = tid + u * nthr, r = c / KC, col = (c % KC) * E;
+                        if (c < NB * KC) {  // padded entries: k = 0, a = 1
+                            put(kh + C::kof(r, col), kx[u], r < nb, 0.f);
+                            if constexpr (CHAN) put(ff + r * C::WS + col, ax[u], r < nb, 1.f);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < VN; ++u) {
+                        const int c = tid + u * nthr, r = c / VC, col = (c % VC) * E;
+                        if (c < NB * VC) put(sv + r * C::VS + col, vx[u], r < nb, 0.f);
+                    }
+                    if (tid < NB) {
+                        sb[tid] = bsc;  // 0 for padded entries
+                        if constexpr (!CHAN) fa[tid] = asc;
+                    }
+                    if (qload) put(sq + tid * E, qx, true, 0.f);
+#pragma unroll
+                    for (int u = 0; u < CN; ++u) {
+                        const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
+                        if (idx < NB * NB && !(cur_here && ci == nl)) sx[ci * C::XS + cj] = cval[u];
+                    }
+                };
+                if (bf) stage(bf16{});
+                else stage(float{});
+                __syncthreads();
+
+                // 2. per key channel, in place: Khat_i = gamma_i o k_i, gamma,
+                // F_j = k_j o D(NB-1, j) (padded entries have a = 1, so D(NB-1, j) = D(nb-1, j)),
+                // stored at f_pos(c): a column of the same warp (f_pos keeps c's group of 16).
+                static_assert(DK <= nthr, "one key channel per thread");
+                for (int c = tid; c < DK; c += nthr) {
+                    float ac[NB], kc[NB];
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) {
+                        ac[i] = CHAN ? ff[i * C::WS + c] : fa[i];
+                        kc[i] = kh[C::kof(i, c)];
+                    }
+                    float gm = 1.f;
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) {
+                        gm *= ac[i];
+                        kh[C::kof(i, c)] = gm * kc[i];
+                    }
+                    gn[c] = gm;
+                    __syncwarp();  // the warp's lanes have read their decays before F lands over them
+                    const int fc = f_pos(c);
+                    float f = 1.f;
+#pragma unroll
+                    for (int j = NB - 1; j >= 0; --j) {
+                        ff[j * C::WS + fc] = kc[j] * f;
+                        f *= ac[j];
+                    }
+                }
+                cp_async_wait_all();  // this thread's share of the base tile has landed
+                __syncthreads();
+                if constexpr (Q8) {
+                    if (b0 == 0) {  // codes * scale into the float tile, 4 at a time
+                        constexpr int WPT = ROWS * DK / 4 / nthr;  // code words per thread
+                        static_assert(WPT * 4 * nthr == ROWS * DK, "whole words per thread");
+                        uint32_t wv[WPT];
+#pragma unroll
+                        // word u holds the codes of row u / (DK/4), from column 4 (u % (DK/4))
+                        for (int i = 0; i < WPT; ++i)
+                            wv[i] = *reinterpret_cast<const uint32_t *>(raw + 4 * (tid + i * nthr));
+                        __syncthreads();  // every code is in registers before the tile is written over them
+#pragma unroll
+                        for (int i = 0; i < WPT; ++i) {
+                            const int u = tid + i * nthr, r = u / (DK / 4), c4 = (u % (DK / 4)) * 4;
+                            const uint32_t w = wv[i];
+                            const float sc = scl[r];
+                            *reinterpret_cast<float4 *>(tile + TL::off(r, c4)) =
+                                make_float4((float)(int8_t)w * sc, (float)(int8_t)(w >> 8) * sc,
+                                            (float)(int8_t)(w >> 16) * sc, (float)(int8_t)(w >> 24) * sc);
+                        }
+                        __syncthreads();
+                    }
+                }
+                // The fused read's current entry is the block's last real one: F_nl = k_nl
+                // exactly (every later factor is a padded 1) and D(nl, j) is F_j's suffix
+                // product, so C(nl, j) = F_nl . F_j. Every warp forms that C row and the
+                // entry's X row itself, with no block barrier: lane-partial dots over its
+                // key channels, one transposing butterfly (lane l ends with C(nl, l >> SH)),
+                // then on lane j: X(nl, j) = -beta sum_{m=j..nl-1} C(nl, m) X(m, j),
+                // X(nl, nl) = beta, kept in the warp's own row sxw.
+                if (DELTA && cur_here) {
+                    constexpr int SH = NB == 16 ? 1 : 2;
+                    float fn[C::CW], pc[NB];
+#pragma unroll
+                    for (int e = 0; e < C::CW; ++e) fn[e] = ff[nl * C::WS + e * 32 + lane];
+#pragma unroll
+                    for (int j = 0; j < NB; ++j) {
+                        pc[j] = 0.f;
+#pragma unroll
+                        for (int e = 0; e < C::CW; ++e) pc[j] = fmaf(fn[e], ff[j * C::WS + e * 32 + lane], pc[j]);
+                    }
+                    multi_sum<NB>(pc, lane);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m < NB; ++m) {
+                        const float cnm = __shfl_sync(0xffffffffu, pc[0], m << SH);
+                        if (lane <= m && m < nl) acc = fmaf(cnm, sx[m * C::XS + lane], acc);
+                    }
+                    const float bn = sb[nl];
+                    if (lane < NB) sxw[warp * C::XS + lane] = lane < nl ? -bn * acc : (lane == nl ? bn : 0.f);
+                    __syncwarp();
+                }
+
+                // 3. this warp's 16 rows: delta in the A-operand layout (split hi + lo).
+                __syncwarp();  // a previous block's rows, written by this warp, are visible
+                const int rg = 16 * warp + g;
+                uint32_t xh[NT][4], xl[NT][4];
+                if constexpr (!DELTA) {
+                    // delta = V, read straight into the operand layout (entries 8nt + t, + 4).
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int i0 = 8 * nt + t;
+                        split_tf32(sv[i0 * C::VS + rg], xh[nt][0], xl[nt][0]);
+                        split_tf32(sv[i0 * C::VS + rg + 8], xh[nt][1], xl[nt][1]);
+                        split_tf32(sv[(i0 + 4) * C::VS + rg], xh[nt][2], xl[nt][2]);
+                        split_tf32(sv[(i0 + 4) * C::VS + rg + 8], xh[nt][3], xl[nt][3]);
+                    }
+                } else {
+                    // G = S Khat^T in the column order above: k-step 2j + h has the A
+                    // fragment a0 = S[g][c], a1 = S[g + 8][c], a2 = S[g][c + 1], a3 = S[g + 8][c + 1]
+                    // with c = 16j + 4t + 2h, and B fragment Khat[8nt + g][c], Khat[8nt + g][c + 1].
+                    // (two accumulator sets, even and odd k-steps, halve the dependent chains)
+                    float acc1[NT][4], acc2[NT][4];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) acc1[nt][x] = acc2[nt][x] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < DK / 16; ++j) {
+                        const float4 x0 = ld_tile4(tile + TL::off(tr + g, 16 * j + 4 * t));
+                        const float4 x1 = ld_tile4(tile + TL::off(tr + g + 8, 16 * j + 4 * t));
+                        uint32_t ah0[4], al0[4], ah1[4], al1[4];
+                        split_tf32(x0.x, ah0[0], al0[0]);
+                        split_tf32(x1.x, ah0[1], al0[1]);
+                        split_tf32(x0.y, ah0[2], al0[2]);
+                        split_tf32(x1.y, ah0[3], al0[3]);
+                        split_tf32(x0.z, ah1[0], al1[0]);
+                        split_tf32(x1.z, ah1[1], al1[1]);
+                        split_tf32(x0.w, ah1[2], al1[2]);
+                        split_tf32(x1.w, ah1[3], al1[3]);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const float4 kv =
+                                *reinterpret_cast<const float4 *>(kh + C::kof(8 * nt + g, 16 * j + 4 * t));
+                            mma3(acc1[nt], ah0, al0, kv.x, kv.y);
+                            mma3(acc2[nt], ah1, al1, kv.z, kv.w);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) acc1[nt][x] += acc2[nt][x];
+                    // E = V - G in the accumulator layout (rows g, g + 8; entries 8nt + 2t, +1).
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int i0 = 8 * nt + 2 * t;
+                        acc1[nt][0] = sv[i0 * C::VS + rg] - acc1[nt][0];
+                        acc1[nt][1] = sv[(i0 + 1) * C::VS + rg] - acc1[nt][1];
+                        acc1[nt][2] = sv[i0 * C::VS + rg + 8] - acc1[nt][2];
+                        acc1[nt][3] = sv[(i0 + 1) * C::VS + rg + 8] - acc1[nt][3];
+                    }
+                    // delta = E X^T (the triangular solve, one small product per warp; X is
+                    // lower triangular, so tiles above the diagonal are skipped).
+                    acc_to_operand<NT>(acc1, xh, xl, lane);
+                    float dl[NT][4];
+#pragma unroll
+                    for (int mt = 0; mt < NT; ++mt) {
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) dl[mt][x] = 0.f;
+                        const int xr = 8 * mt + g;  // the fused entry's row is the warp's own copy
+                        const float *xrow = (cur_here && xr == nl) ? sxw + warp * C::XS : sx + xr * C::XS;
+#pragma unroll
+                        for (int kt = 0; kt <= mt; ++kt) {
+                            const float *xp = xrow + 8 * kt + t;
+                            mma3(dl[mt], xh[kt], xl[kt], xp[0], xp[4]);
+                        }
+                    }
+                    acc_to_operand<NT>(dl, xh, xl, lane);
+                }
+                // S <- S o gamma + delta F, two 16 x 8 column tiles at a time: tiles 2j and
+                // 2j + 1 give lane (g, t) columns 16j + 4t .. + 3 of rows g and g + 8 (the
+                // column order above); from the tile, back to the tile for a following
+                // sub-merge (or, for an int8 base, for the rounding below), else straight
+                // to HBM.
+                float rmax0 = 0.f, rmax1 = 0.f;  // int8 base: |value| maxima of rows g, g + 8 (this lane's columns)
+#pragma unroll 2
+                for (int j = 0; j < DK / 16; ++j) {
+                    float d[2][4];  // tile 2j + h: rows g, g + 8 at columns 16j + 4t + 2h, + 1
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float dn[NT][4];  // one accumulator per entry tile: independent chains
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) dn[nt][x] = 0.f;
+                            const float *fp = ff + (8 * nt + t) * C::WS + 16 * j + 8 * h + g;
+                            mma3(dn[nt], xh[nt], xl[nt], fp[0], fp[4 * C::WS]);
+                        }
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            d[h][x] = dn[0][x];
+#pragma unroll
+                            for (int nt = 1; nt < NT; ++nt) d[h][x] += dn[nt][x];
+                        }
+                    }
+                    const int col = 16 * j + 4 * t;
+                    TT *p0 = tile + TL::off(tr + g, col), *p1 = tile + TL::off(tr + g + 8, col);
+                    const float4 r0 = ld_tile4(p0), r1 = ld_tile4(p1);
+                    const float4 gv = *reinterpret_cast<const float4 *>(gn + col);
+                    const float4 s0 = make_float4(fmaf(r0.x, gv.x, d[0][0]), fmaf(r0.y, gv.y, d[0][1]),
+                                                  fmaf(r0.z, gv.z, d[1][0]), fmaf(r0.w, gv.w, d[1][1]));
+                    const float4 s1 = make_float4(fmaf(r1.x, gv.x, d[0][2]), fmaf(r1.y, gv.y, d[0][3]),
+                                                  fmaf(r1.z, gv.z, d[1][2]), fmaf(r1.w, gv.w, d[1][3]));
+                    if (WITH_CUR && last) {
+                        const float4 qv = *reinterpret_cast<const float4 *>(sq + col);
+                        oacc[0] = fmaf(s0.x, qv.x, fmaf(s0.y, qv.y, fmaf(s0.z, qv.z, fmaf(s0.w, qv.w, oacc[0]))));
+                        oacc[1] = fmaf(s1.x, qv.x, fmaf(s1.y, qv.y, fmaf(s1.z, qv.z, fmaf(s1.w, qv.w, oacc[1]))));
+                    }
+                    if constexpr (Q8) {
+                        st_tile4(p0, s0);
+                        st_tile4(p1, s1);
+                        rmax0 = fmaxf(rmax0, fmaxf(fmaxf(fabsf(s0.x), fabsf(s0.y)), fmaxf(fabsf(s0.z), fabsf(s0.w))));
+                        rmax1 = fmaxf(rmax1, fmaxf(fmaxf(fabsf(s1.x), fabsf(s1.y)), fmaxf(fabsf(s1.z), fabsf(s1.w))));
+                    } else if (last) {
+                        st_state4(Sw + g * DK + col, s0);
+                        st_state4(Sw + (g + 8) * DK + col, s1);
+                    } else {
+                        st_tile4(p0, s0);
+                        st_tile4(p1, s1);
+                    }
+                }
+                if constexpr (Q8) {
+                    if (last) {  // round the warp's 16 rows to int8 (one scale per row) and store them
+#pragma unroll
+                        for (int off = 1; off <= 2; off <<= 1) {  // the quad holds a row's columns
+                            rmax0 = fmaxf(rmax0, __shfl_xor_sync(0xffffffffu, rmax0, off));
+                            rmax1 = fmaxf(rmax1, __shfl_xor_sync(0xffffffffu, rmax1, off));
+                        }
+                        if (t == 0) {
+                            wsc[warp * 16 + g] = i8_scale(rmax0);
+                            wsc[warp * 16 + g + 8] = i8_scale(rmax1);
+                        }
+                        __syncwarp();
+                        constexpr int CPR = DK / 16;  // 16-code chunks per row
+                        for (int i = lane; i < 16 * CPR; i += 32) {
+                            const int rl = i / CPR, c0 = (i % CPR) * 16;
+                            const float sc = wsc[warp * 16 + rl];
+                            uint32_t wd[4];
+#pragma unroll
+                            for (int qd = 0; qd < 4; ++qd) {
+                                const float4 x =
+                                    *reinterpret_cast<const float4 *>(tile + TL::off(tr + rl, c0 + 4 * qd));
+                                wd[qd] = (uint32_t)(i8_code(x.x, sc) & 0xff) |
+                                         ((uint32_t)(i8_code(x.y, sc) & 0xff) << 8) |
+                                         ((uint32_t)(i8_code(x.z, sc) & 0xff) << 16) |
+                                         ((uint32_t)(i8_code(x.w, sc) & 0xff) << 24);
+                            }
+                            st_stream(Sw + rl * DK + c0, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+                        }
+                        if (lane < 16) i8_scales[shead * DV + row0 + tr + lane] = wsc[warp * 16 + lane];
+                    }
+                }
+                __syncthreads();  // the next entry block reuses the shared buffers
+            }
+
+            if constexpr (WITH_CUR) {
+                oacc[0] = group_sum<4>(oacc[0]);
+                oacc[1] = group_sum<4>(oacc[1]);
+                if (t == 0) {
+                    o[head * DV + row0 + 16 * warp + g] = oacc[0];
+                    o[head * DV + row0 + 16 * warp + g + 8] = oacc[1];
+                }
+            }
+        }
+        if (!compact) break;
+        __syncthreads();  // thread 0's update of the walk is visible to all
     }
 }
 
@@ -577,7 +685,17 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
     const size_t smem = merge_smem_bytes<ST, DK, NB>();
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    const long long blocks = (long long)p.B * p.H * (p.dv / rows);
+    const long long units = (long long)p.B * p.H * (p.dv / rows);
+    long long blocks = units;
+    if (pool.slot && part == POOL_MERGE_FULL) {
+        // only the slots on their L-th entry merge: a compact grid of as many blocks
+        // as can be resident (4 per SM) walks all units and merges those
+        int dev = 0, sms = 0;
+        e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        blocks = std::min<long long>(units, 4LL * sms);
+    }
     // an int8 base's row scales follow its codes (all the state's heads: the pool's, or B*H)
     const long long state_heads = pool.slot ? (long long)pool.P * pool.H : (long long)p.B * p.H;
     float *i8_scales = std::is_same<ST, int8_t>::value
@@ -585,7 +703,7 @@ static cudaError_t launch_merge_t(const StepParams &p, const LogParams &lg, int 
                            : nullptr;
     kern<<<(unsigned)blocks, rows * 2, smem, st>>>(static_cast<ST *>(p.S), lg.k, lg.v, lg.beta, lg.a, lg.x, lg.L,
                                                    n_log, p.q, p.k, p.v, p.beta, p.a, p.o, p.dv,
-                                                   p.in_dt == DL_BF16, pool, part, i8_scales);
+                                                   p.in_dt == DL_BF16, pool, part, i8_scales, units);
     return cudaGetLastError();
 }
 
