@@ -130,11 +130,41 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
 
 
+def code_tokens(src: str) -> str:
+    """C/C++/CUDA source with its comments removed and whitespace runs folded
+    to one space: what the compiler sees, so that a comment edit does not
+    count as a kernel change. String and character literals are kept whole."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the dominant kernel's code (comments and layout excluded); the
+    profiled DRAM traffic is used only while the sources still hash to the
+    value recorded with it."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,8 +1,8 @@
 // Deferred step: append this step's factors to the log and read
 // o = S_n q from the unwritten base plus the log (DeltaLog page, Technical
-// Summary, "Append Phase", and "Kernel Implementation": key-side metadata
-// computed once per slot-head in a "ReplayPrep" stage and shared by the value
-// tiles, which then run in parallel "AppendDecode" stages).
+// Summary, "Append Phase", and "Kernel Implementation": the key-side work is
+// done once per (sequence, head) in a "ReplayPrep" stage, and its results serve
+// every value tile, each an "AppendDecode" stage running in parallel).
 //
 // With A_e = Diag(a_e)(I - beta_e k_e k_e^T), entries e = 0..n (n is this
 // step's, the newest), the logical state is S_bar A_0 ... A_n-style replayed

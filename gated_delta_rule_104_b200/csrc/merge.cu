@@ -1,7 +1,7 @@
-// Merge of the bounded log into the dense base (DeltaLog page, Technical
-// Summary, "Merge Phase": every M steps the accumulated logical state -- base
-// plus replayed log entries -- is materialised back into the base), and the
-// same merge fused with one step's read.
+// Merge of the bounded log into the dense base (DeltaLog page, "Core
+// Mechanism: Base + Log", the merge phase: at intervals the base absorbs every
+// update the log holds and the log starts empty again), and the same merge
+// fused with one step's read.
 //
 // Log-decay form. For log entries 0..n-1 (decays a_i, keys k_i, values v_i,
 // strengths beta_i) write D(i, j) = prod_{m=j+1..i} a_m (= exp(Lambda_i -
@@ -13,34 +13,37 @@
 // the merged row is s o gamma + sum_j delta_j F_j with F_j = k_j o D(n-1, j).
 // The triangular solve is the same for every row: delta = X (v_r - G) with
 // X = (I + Diag(beta) C)^{-1} Diag(beta), which the log keeps (each append
-// adds its row), so the merge is two thin products
+// adds its row), so per block of rows the merge is
 //   G = S Khat^T                 [rows x d_k] x [d_k x n]
-//   S <- S o gamma + (V - G) W,  W = X^T F     [rows x n] x [n x d_k]
-// with W formed once per head. That is 4 n d_k d_v FLOP against 2 d_k d_v
-// state elements moved: a small dense contraction. For a block of entries
-// [b, b + 16) of a longer log, X's diagonal block is the block's own X.
+//   delta = (V - G) X^T          [rows x n] x [n x n], X lower triangular
+//   S <- S o gamma + delta F     [rows x n] x [n x d_k]
+// That is about 4 n d_k d_v FLOP against 2 d_k d_v state elements moved: a
+// small dense contraction. For a block of entries [b, b + 16) of a longer log,
+// X's diagonal block is the block's own X.
 //
-// Both products run on the tensor cores (mma.sync m16n8k8, TF32 in fp32
+// All three products run on the tensor cores (mma.sync m16n8k8, TF32 in fp32
 // accumulators). Plain TF32 keeps 10 mantissa bits, too few for the fp32
 // state, so every operand is split as x = hi + lo (two TF32 values) and each
 // product is formed as hi*hi + hi*lo + lo*hi, which recovers ~fp32 accuracy.
 //
 // RWKV6 (no delta correction) is the case X = I and no G: delta = V.
 //
-// Kernel: one block per (head, tile of up to 128 rows); warp w owns rows
+// Kernel: one 4-warp block per unit (head, tile of 64 rows); warp w owns rows
 // 16w..16w+15 of the tile. The entries are merged in blocks of NB = 8 or 16
 // (a longer log is a chain of sub-merges; short blocks are padded with
-// neutral entries k = 0, a = 1, beta = 0, v = 0). Per block:
+// neutral entries k = 0, a = 1, beta = 0, v = 0). Per entry block:
 //  1. stage the block's keys, decays, beta, X rows and the tile's values in
-//     shared memory (all global loads issued before any shared store);
+//     shared memory (all global loads issued before any shared store; the
+//     first block also starts the base tile's cp.async);
 //  2. per key channel, running decay products give Khat, F and gamma; the
-//     fused read's current entry (the block's last) has C(n, j) = k_n . F_j,
-//     from which its X row follows;
-//  3. W = X^T F;
-//  4. per warp: G by tensor-core tiles, E = V - G moved from accumulator to
-//     operand layout with quad shuffles, S o gamma + E W by tensor-core
-//     tiles, the merged rows written back (and o = s_new . q for the fused
-//     read) straight from the accumulator layout.
+//     fused read's current entry (the block's last) has C(n, j) = F_n . F_j,
+//     from which each warp forms its X row;
+//  3. per warp: G by tensor-core tiles, E = V - G moved from accumulator to
+//     operand layout with quad shuffles, delta = E X^T (lower tiles only),
+//     then S o gamma + delta F by tensor-core tiles, the merged rows written
+//     back (and o = s_new . q for the fused read) straight from the
+//     accumulator layout.
+// A pool step's merge part runs the same body over a compact grid (below).
 #include "launch.h"
 
 namespace dl {

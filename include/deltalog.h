@@ -98,8 +98,8 @@ typedef enum {
  * the raw step factors, stored unchanged in `dtype` (lossless), their
  * log-decay metadata, and a small fp32 workspace the deferred read uses to
  * hand its per-head key-side results to the value tiles.
- * (The page's log keeps "compact update factors" plus log-decay metadata,
- * Technical Summary, "Core Mechanism: Base + Log"; here the decay products
+ * (The page's log holds each step's small update factors with log-decay
+ * metadata, Technical Summary, "Core Mechanism: Base + Log"; here the decay products
  * are recomputed from the stored decays where they are needed, and the
  * triangular solve they lead to is kept as x below.)
  *   k     [B, H, L, d_k]

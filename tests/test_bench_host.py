@@ -126,3 +126,15 @@ def test_max_over_ranks_gloo_world2(tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     for rank in (0, 1):  # every rank sees the max of the per-rank times
         assert (tmp_path / f"rank{rank}.txt").read_text() == "ok 11.0"
+
+
+def test_kernel_hash_ignores_comments_and_layout_only():
+    """The profiled traffic stays tied to the kernel's code: a comment or a
+    re-wrapped line keeps the hash, any change of code or literal moves it."""
+    src = 'int f(int x) {  // the count\n  /* scaled */ return x * 2 + "a//b"[0]; }\n'
+    same = 'int f(int x) {\n    return x * 2 + "a//b"[0];  /* other words */ }'
+    assert bench.code_tokens(src) == bench.code_tokens(same)
+    assert bench.code_tokens(src) != bench.code_tokens(src.replace("x * 2", "x * 3"))
+    assert bench.code_tokens(src) != bench.code_tokens(src.replace('"a//b"', '"a/ /b"'))
+    assert "/*" in bench.code_tokens('s = "/*"; t = 1;') and bench.code_tokens("a /* b */ c") == "a c"
+    assert bench.code_tokens("x = '\\'' ; // y") == "x = '\\'' ;"

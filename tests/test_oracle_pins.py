@@ -6,8 +6,9 @@ Technical Summary, "Kernel Implementation") is
 
     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
 
-and the deferred schedule must reproduce it exactly ("does not alter ... the
-mathematical recurrence", Technical Summary, "Methodology").
+and the deferred schedule must reproduce it exactly: the method changes only
+when the state is written back, never what it computes (Technical Summary,
+"Methodology").
 
 Pins:
   P0 hand-worked exact examples (tests/golden/hand_worked_steps.json);
