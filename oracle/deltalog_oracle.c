@@ -301,27 +301,36 @@ void oracle_deferred(long NH, int T, int dk, int dv, int kind, int L,
 
 /* Quantisation of a base held in int8 with one scale per state row (a value
  * channel): scale = max_c |row_c| / 127 and code_c = the nearest integer to
- * row_c / scale (ties to even), so that row_c becomes code_c * scale; an
- * all-zero row stays zero. (The low-precision base of the DAMP abstract,
- * "Decay-Aware Mixed-Precision Recurrent-State Quantization", which stores
- * recurrent states in INT8: with the deferred schedule the base is written,
- * and so rounded, only when a merge writes it.) */
+ * row_c / scale (ties to even, clamped to [-127, 127]), so that row_c becomes
+ * code_c * scale; a row whose largest magnitude is zero becomes zero. (The
+ * low-precision base of the DAMP abstract, "Decay-Aware Mixed-Precision
+ * Recurrent-State Quantization", which stores recurrent states in INT8: with
+ * the deferred schedule the base is written, and so rounded, only when a merge
+ * writes it.)
+ *
+ * The pages fix no precision for this rounding, so it is taken in fp32, the
+ * precision of the kernel that stores the base: the row is first taken to fp32,
+ * and the maximum, the scale, each quotient and each code * scale are single
+ * correctly rounded fp32 operations (this file is built with -ffp-contract=off,
+ * so none is fused). A value then takes the same code on both sides whenever
+ * both hold the same fp32 value. */
 static void quantize_rows_i8(double *S, int dv, int dk)
 {
     for (int r = 0; r < dv; ++r) {
         double *row = S + (long)r * dk;
-        double m = 0.0;
+        float m = 0.0f;
         for (int c = 0; c < dk; ++c)
-            if (fabs(row[c]) > m)
-                m = fabs(row[c]);
-        if (m == 0.0)
-            continue;
-        double scale = m / 127.0;
+            if (fabsf((float)row[c]) > m)
+                m = fabsf((float)row[c]);
+        const float scale = m / 127.0f;
         for (int c = 0; c < dk; ++c) {
-            double code = nearbyint(row[c] / scale);
-            if (code > 127.0) code = 127.0;
-            if (code < -127.0) code = -127.0;
-            row[c] = code * scale;
+            float code = 0.0f;
+            if (scale != 0.0f) {
+                code = nearbyintf((float)row[c] / scale);
+                if (code > 127.0f) code = 127.0f;
+                if (code < -127.0f) code = -127.0f;
+            }
+            row[c] = (double)(code * scale);
         }
     }
 }

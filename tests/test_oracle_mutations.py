@@ -44,8 +44,9 @@ MUTATIONS = {
     "rwkv6_merge_decays_own_value": ("delta[i] = lg->v[(long)(i - 1) * dv + r];",
                                      "delta[i] = lg->v[(long)(i - 1) * dv + r] * lg->a[(long)(i - 1) * dk];"),
     # int8 base
-    "i8_rounds_half_away": ("double code = nearbyint(row[c] / scale);", "double code = round(row[c] / scale);"),
-    "i8_scale_128": ("double scale = m / 127.0;", "double scale = m / 128.0;"),
+    "i8_rounds_half_away": ("code = nearbyintf((float)row[c] / scale);", "code = roundf((float)row[c] / scale);"),
+    "i8_scale_128": ("const float scale = m / 127.0f;", "const float scale = m / 128.0f;"),
+    "i8_decided_in_fp64": ("code = nearbyintf((float)row[c] / scale);", "code = (float)nearbyint(row[c] / scale);"),
     "i8_start_unrounded": ("        quantize_rows_i8(Sbar, dv, dk);\n        for (int t = 0; t < T; ++t) {",
                            "        for (int t = 0; t < T; ++t) {"),
     "i8_no_rounding_at_merges": ("                deferred_merge(Sbar, &lg);\n                quantize_rows_i8(Sbar, dv, dk);",

@@ -405,20 +405,34 @@ def test_p11_slot_pool_is_per_sequence_recurrence(oracle_mod):
 # ------------------------------------------------------------------ P12 (int8 base)
 
 def check_p12(impl):
-    # a hand-worked row: max 127 gives scale 1; 62.5 -> 62 and -3.5 -> -4 (ties to
-    # even), 0.4 -> 0; an all-zero row stays zero
-    S = np.array([[[127.0, 62.5, -3.5, 0.4], [0.0, 0.0, 0.0, 0.0], [-2.0, 1.0, 0.5, 0.25]]])
-    # third row: max 2, scale 2/127: codes -127, 63.5 -> 64 (even), 31.75 -> 32, 15.875 -> 16
-    exp = np.array([[[127.0, 62.0, -4.0, 0.0], [0.0, 0.0, 0.0, 0.0],
-                     [-2.0, 64 * 2 / 127, 32 * 2 / 127, 16 * 2 / 127]]])
+    # Hand-worked rows whose fp32 arithmetic is exact, so that the expected
+    # values can be checked by eye:
+    # - max 127, scale 1: 62.5 -> 62 and -3.5 -> -4 (ties to even), 0.4 -> 0;
+    # - an all-zero row stays zero;
+    # - max 63.5, scale 0.5: 31.75 / 0.5 = 63.5 -> 64 (even), 15.875 -> 31.75 -> 32,
+    #   0.25 -> 0.5 -> 0 (even);
+    # - the code is decided in fp32, the kernel's precision: 62.50000001 is
+    #   62.5 in fp32, a tie that goes to the even 62 (an fp64 decision gives 63).
+    S = np.array([[[127.0, 62.5, -3.5, 0.4], [0.0, 0.0, 0.0, 0.0], [-63.5, 31.75, 15.875, 0.25],
+                   [127.0, 62.50000001, 0.0, 0.0]]])
+    exp = np.array([[[127.0, 62.0, -4.0, 0.0], [0.0, 0.0, 0.0, 0.0], [-63.5, 32.0, 16.0, 0.0],
+                     [127.0, 62.0, 0.0, 0.0]]])
     got = impl.quantize_i8(S)
-    assert np.allclose(got, exp, rtol=0, atol=1e-15), got
+    assert np.array_equal(got, exp), got
     rng = np.random.default_rng(23)
     R = rng.standard_normal((3, 6, 8))
     once = impl.quantize_i8(R)
-    assert np.allclose(impl.quantize_i8(once), once, rtol=0, atol=1e-14)
-    codes = once / (np.abs(R).max(axis=-1, keepdims=True) / 127)
-    assert np.allclose(codes, np.round(codes), atol=1e-9) and np.abs(codes).max() <= 127 + 1e-9
+    # every value is code * scale with an integer code in [-127, 127] and the
+    # row's fp32 scale max|row| / 127
+    R32 = R.astype(np.float32)
+    scale = np.abs(R32).max(axis=-1, keepdims=True) / np.float32(127)
+    codes = once / scale.astype(np.float64)
+    assert np.allclose(codes, np.round(codes), rtol=0, atol=1e-4) and np.abs(np.round(codes)).max() <= 127
+    assert np.array_equal(once, (np.round(codes).astype(np.float32) * scale).astype(np.float64))
+    # and it is the nearest such value to each fp32 input (at most half a step away)
+    assert (np.abs(once - R32.astype(np.float64)) <= 0.5 * scale * (1 + 1e-6)).all()
+    # rounding again moves a value by at most an fp32 rounding of its scale
+    assert np.allclose(impl.quantize_i8(once), once, rtol=1e-6, atol=0)
     for chan, rw in ((False, False), (True, False), (True, True)):
         NH, T, dk, dv = 2, 9, 8, 6
         S0, q, k, v, beta, a = rand_case(rng, NH, T, dk, dv, chan or rw)
