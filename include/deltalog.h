@@ -80,7 +80,8 @@ typedef enum {
  * as for the other types, then B*H*d_v fp32 scales (dl_state_bytes) -- and an
  * element's value is code * scale. Every merge re-rounds the rows it writes:
  * scale = max|row| / 127, code = the nearest integer to value / scale, ties to
- * even (an all-zero row stays zero). (The low-precision base of the DAMP
+ * even, clamped to [-127, 127] (an all-zero row stays zero), each step one
+ * correctly rounded fp32 operation on the row's fp32 values. (The low-precision base of the DAMP
  * abstract, "Decay-Aware Mixed-Precision Recurrent-State Quantization": with
  * the deferred schedule the base is rounded once per merge, not every step.)
  * The eager steps take DL_F32 or DL_BF16 only (DL_I8 -> DL_ERR_UNSUPPORTED). */
