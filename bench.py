@@ -239,6 +239,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle leg
 
+REFERENCE_RUN_S = 120.0  # oracle seconds for all timed steps of `--impl reference`
+REFERENCE_MAX_HEADS = 2048  # bound on its sample (about 1 MB of inputs per head)
+
+
 def oracle_sample(w: W.Workload, L: int, budget_s: float, first_head: int = 0):
     """Time the fp64 oracle (deferred schedule, log capacity L) on heads of the
     workload until about ``budget_s`` seconds of CPU work; returns
@@ -257,7 +261,10 @@ def oracle_sample(w: W.Workload, L: int, budget_s: float, first_head: int = 0):
         secs += time.perf_counter() - t0
         heads_done += len(heads)
         h0 += len(heads)
-        chunk = min(chunk * 2, 4096)
+        # next chunk: double, but no more than the measured rate fits in what is
+        # left of the budget (a multiple of the threads, at least one round)
+        fit = int((budget_s - secs) / (secs / heads_done)) // threads * threads
+        chunk = max(threads, min(chunk * 2, 4096, fit))
     tokens = heads_done * w.T / w.H  # one token = one sequence step across its H heads
     return tokens / secs, heads_done, secs, threads
 
@@ -266,21 +273,35 @@ def run_reference(args, w, L):
     rank, _, ws = dist_env()
     if rank != 0:
         return 0
-    import oracle
+    import oracle  # the reference arm is the oracle itself
 
     oracle.build()
-    budget = args.cpu_seconds_per_step
+    threads = oracle.omp_threads()
+    # Each timed step runs the oracle's deferred schedule over one fixed sample
+    # of heads (all T steps of each), sized by a short probe so that a step is
+    # about `budget` seconds and the whole run about REFERENCE_RUN_S; the
+    # sample's inputs are generated once and reused by every step.
+    budget = min(args.cpu_seconds_per_step, max(1.0, REFERENCE_RUN_S / max(1, args.steps)))
+    n_probe = min(threads, w.heads)
+    probe = W.generate(w, heads=range(n_probe))
+    t0 = time.perf_counter()
+    oracle.run_workload_heads(w, probe, "deferred", L)
+    per_head = (time.perf_counter() - t0) / n_probe
+    nh = int(budget / per_head) // threads * threads
+    nh = max(n_probe, min(nh, w.heads, REFERENCE_MAX_HEADS))
+    stride = 997  # spread the sample over the batch (coprime with every B*H used)
+    x = W.generate(w, heads=[(i * stride) % w.heads for i in range(nh)])
     for _ in range(args.warmup):
-        oracle_sample(w, L, min(2.0, budget))
-    vals, secs_all, heads_all = [], 0.0, 0
-    for i in range(args.steps):
-        v, heads, secs, threads = oracle_sample(w, L, budget, first_head=i * 997)
-        vals.append(v)
-        secs_all += secs
-        heads_all += heads
+        oracle.run_workload_heads(w, probe, "deferred", L)
+    secs_all = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.run_workload_heads(w, x, "deferred", L)
+        secs_all += time.perf_counter() - t0
+    heads_all = nh * args.steps
     value = heads_all * w.T / w.H / secs_all
-    sample = (f"{heads_all} of {w.heads} (b,h) heads x all {w.T} steps over {args.steps} steps "
-              f"(about {budget:.0f} s of oracle work each), deferred schedule L={L}, fp64")
+    sample = (f"the same {nh} of {w.heads} (b,h) heads x all {w.T} steps in each of {args.steps} steps "
+              f"({secs_all / max(1, args.steps):.1f} s of oracle work each), deferred schedule L={L}, fp64")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * w.B * w.T / value, "higher_is_better": True, "scaling": "weak",

@@ -138,3 +138,21 @@ def test_kernel_hash_ignores_comments_and_layout_only():
     assert bench.code_tokens(src) != bench.code_tokens(src.replace('"a//b"', '"a/ /b"'))
     assert "/*" in bench.code_tokens('s = "/*"; t = 1;') and bench.code_tokens("a /* b */ c") == "a c"
     assert bench.code_tokens("x = '\\'' ; // y") == "x = '\\'' ;"
+
+
+def test_reference_arm_prints_one_oracle_line():
+    """`--impl reference` times the oracle on host cores and prints the
+    contract's line (smallest workload, so that it runs in seconds)."""
+    import json
+
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3",
+                          "--workload", "gdn_b1_h2_d64_t16"], cwd=os.path.dirname(bench.__file__),
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [x for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s" and d["steps"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "the same 2 of 2 (b,h) heads" in d["cpu_baseline"]["sample"]
