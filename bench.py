@@ -263,7 +263,7 @@ def oracle_sample(w: W.Workload, L: int, budget_s: float, first_head: int = 0):
         h0 += len(heads)
         # next chunk: double, but no more than the measured rate fits in what is
         # left of the budget (a multiple of the threads, at least one round)
-        fit = int((budget_s - secs) / (secs / heads_done)) // threads * threads
+        fit = int((budget_s - secs) / (max(secs, 1e-9) / heads_done)) // threads * threads
         chunk = max(threads, min(chunk * 2, 4096, fit))
     tokens = heads_done * w.T / w.H  # one token = one sequence step across its H heads
     return tokens / secs, heads_done, secs, threads
@@ -286,7 +286,7 @@ def run_reference(args, w, L):
     probe = W.generate(w, heads=range(n_probe))
     t0 = time.perf_counter()
     oracle.run_workload_heads(w, probe, "deferred", L)
-    per_head = (time.perf_counter() - t0) / n_probe
+    per_head = max(time.perf_counter() - t0, 1e-9) / n_probe
     nh = int(budget / per_head) // threads * threads
     nh = max(n_probe, min(nh, w.heads, REFERENCE_MAX_HEADS))
     stride = 997  # spread the sample over the batch (coprime with every B*H used)
