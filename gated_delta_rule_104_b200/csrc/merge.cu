@@ -154,11 +154,14 @@ struct BaseTile {
 //   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
 //   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
 //   sxw [4][XS] each warp's copy of the fused entry's X row
-//   xw [4] (after the int8 arrays, if any) a compact grid's unit ballots
+//   xw [5] (after the int8 arrays, if any) a compact grid's walk: four ballots
+//   and the batch index, XW_BYTES
 //   int8 base only: scl [ROWS] row scales, wsc [4][16] the new row scales of
 //   each warp's rows; the codes [ROWS][DK] land in the last ROWS * DK bytes of
 //   the float tile and are read out into registers before it is widened over
 //   them (no separate code buffer: four blocks per SM, as for a float base)
+constexpr size_t XW_BYTES = 32;  // the compact walk's five words, padded to 16-byte granules
+
 template <class ST, int DK, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
     using C = MergeShape<DK, NB>;
@@ -167,7 +170,7 @@ __host__ __device__ constexpr size_t merge_smem_bytes() {
     const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK +
                           (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS + 4 * (size_t)C::XS;
     const size_t q8 = Q8 ? (size_t)C::ROWS * 4 + 64 * 4 : 0;
-    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8 + 16;  // + 16: xw
+    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8 + XW_BYTES;
 }
 
 // Accumulator layout (rows g, g + 8; columns 8i + 2t, 8i + 2t + 1) to A-operand
