@@ -43,8 +43,9 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "kda_b256_h32_d128_t512"
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "append_read_kda_b256_h32_d128_L16.md")
-KERNEL_SOURCES = ["gated_delta_rule_104_b200/csrc/deferred_read.cu", "gated_delta_rule_104_b200/csrc/common.cuh"]
+# ncu DRAM traffic per launch, recorded per (kernel, workload, L) with a hash of
+# the kernel sources it was captured on (profiles/dram_traffic.json)
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 # ---------------------------------------------------------------- byte model
@@ -157,34 +158,34 @@ def code_tokens(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_source_hash() -> str:
-    """Hash of the dominant kernel's code (comments and layout excluded); the
-    profiled DRAM traffic is used only while the sources still hash to the
-    value recorded with it."""
+def kernel_source_hash(sources) -> str:
+    """Hash of a kernel's code (comments and layout excluded); a recorded DRAM
+    traffic figure is used only while its sources still hash to the value
+    recorded with it."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
             h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+def traffic_key(kind: str, workload: str, L: int) -> str:
+    return f"{kind}/{workload}/L{L}"
+
+
+def profiled_traffic(kind: str, workload: str, L: int, record: str = TRAFFIC_RECORD):
+    """DRAM bytes per launch of ``kind`` from the committed ncu record, if one
+    was taken for this workload and L on the current kernel sources (else None)."""
     try:
-        txt = open(PROFILE_SUMMARY).read()
-    except OSError:
+        with open(record, encoding="utf-8") as f:
+            rec = json.load(f).get(traffic_key(kind, workload, L))
+    except (OSError, ValueError):
         return None
-    vals = {}
-    for line in txt.splitlines():
-        if ":" in line and line.strip().startswith("- `"):
-            key, _, val = line.strip()[3:].partition("`:")
-            vals[key.strip()] = val.strip()
-    if vals.get("source_sha256_16") != kernel_source_hash():
+    if not rec or rec.get("source_sha256_16") != kernel_source_hash(rec.get("sources", [])):
         return None
     try:
-        return float(vals["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -566,6 +567,68 @@ def run_e2e(g, w, host, L, schedule, steps, warmup, stream):
     return ms, h2d_bytes, d2h_bytes
 
 
+def decode_bytes(w, plan):
+    """Algorithmic bytes of one whole decode (every launch of the plan)."""
+    return sum(alg_bytes(w, kind, n) for kind, n in plan)
+
+
+def run_sweep(args, w, Ls):
+    """Log-capacity sweep on one workload (the page's trade-off between replay
+    traffic and saved dense writes): per L, the fused deferred decode's
+    tokens/s, its read/merge time split and its bytes per token, beside the
+    eager decode's."""
+    workers = args.workers or W.default_workers()
+    x = W.generate(w, workers=workers)
+
+    import torch
+
+    import gated_delta_rule_104_b200 as g
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA library is the only compute path)")
+    torch.cuda.set_device(0)
+    g.load()
+    d = W.device_inputs(w, x)
+    del x
+    stream = torch.cuda.current_stream()
+    chan, rw = w.decay != W.HEAD, w.decay == W.RWKV6
+    o_all = torch.empty(w.T, w.B, w.H, w.d_v, dtype=torch.float32, device="cuda")
+    peak, peak_note = measured_peaks()
+    tokens = w.B * w.T
+    S_e = d["S0"].clone()
+    lau_e = Launcher(g, w, d, S_e, None, o_all, "eager", stream)
+    with ClockSampler(0) as smp:
+        ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup)
+    del S_e
+    eager_bpt = decode_bytes(w, lau_e.plan()) / tokens
+    eager_val = tokens / (ms_e / 1000.0)
+    print(json.dumps({"sweep": "eager", "workload": w.name, "value": eager_val, "unit": UNIT,
+                      "ms_per_step": round(ms_e, 3), "alg_bytes_per_token": round(eager_bpt),
+                      "roofline": roofline_for(w, kinds_e, "eager", peak, peak_note, None),
+                      "clocks": smp.summary()}), flush=True)
+    for L in Ls:
+        S = d["S0"].clone()
+        log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, d["q"].dtype, chan, rwkv6=rw)
+        lau = Launcher(g, w, d, S, log, o_all, "fused", stream)
+        with ClockSampler(0) as smp:
+            ms, kinds, launches = timed(lau, args.steps, args.warmup)
+        split = {k: round(sum(ms_ for _, ms_ in v) / args.steps, 3) for k, v in kinds.items()}
+        bpt = decode_bytes(w, lau.plan()) / tokens
+        value = tokens / (ms / 1000.0)
+        print(json.dumps({
+            "sweep": "L", "workload": w.name, "L": L, "value": value, "unit": UNIT, "ms_per_step": round(ms, 3),
+            "eager_value": eager_val, "deferred_over_eager": value / eager_val,
+            "ms_per_step_by_kernel": split,
+            "read_share": round(split.get("append_read", 0.0) / max(ms, 1e-9), 4),
+            "alg_bytes_per_token": round(bpt), "eager_alg_bytes_per_token": round(eager_bpt),
+            "eager_over_deferred_bytes": round(eager_bpt / bpt, 4),
+            "roofline": {k: roofline_for(w, kinds, k, peak, peak_note, profiled_traffic(k, w.name, L))
+                         for k in kinds},
+            "gpu_launches": launches, "clocks": smp.summary()}), flush=True)
+        del S, log
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -585,6 +648,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
                     help="decode only this many tokens per step (small profiling runs; default: the workload's T)")
+    ap.add_argument("--sweep-L", default="",
+                    help="comma list of log capacities: one JSON line per L (fused deferred schedule, with the "
+                         "read/merge split and bytes per token) after one eager line, inputs generated once")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -598,6 +664,8 @@ def main(argv=None):
 
     if args.impl == "reference":
         return run_reference(args, w, L)
+    if args.sweep_L:
+        return run_sweep(args, w, [int(x) for x in args.sweep_L.split(",") if x.strip()])
 
     # Inputs first (spawned generator processes start before any CUDA call).
     workers = args.workers or W.default_workers()
@@ -625,8 +693,6 @@ def main(argv=None):
     tdt = d["q"].dtype
     o_all = torch.empty(w.T, w.B, w.H, w.d_v, dtype=torch.float32, device="cuda")
     peak, peak_note = measured_peaks()
-    # the committed DRAM-traffic figure is for the KDA workload's append_read at L = 16
-    traffic = profiled_traffic() if (w.name == DEFAULT_WORKLOAD and L == 16) else None
 
     sampler = ClockSampler(local_rank)
     with sampler:
@@ -664,9 +730,13 @@ def main(argv=None):
     value = w.B * w.T / (ms_def / 1000.0) * ws
     main_kind = "pool" if args.schedule == "pool" else "append_read"
     wb = W.scaled(w, state_dtype="i8") if args.base_i8 else w
-    measured_traffic = traffic if (main_kind == "append_read" and not args.base_i8) else None
-    rf = roofline_for(wb, kinds_def, main_kind, peak, peak_note, measured_traffic)
-    other = {k: roofline_for(wb, kinds_def, k, peak, peak_note, None) for k in kinds_def if k != main_kind}
+    def traffic(kind):  # the ncu record is of the fp32/bf16 base on the fused schedule
+        if args.base_i8 or args.tokens or args.schedule == "unfused":
+            return None
+        return profiled_traffic(kind, w.name, L)
+
+    rf = roofline_for(wb, kinds_def, main_kind, peak, peak_note, traffic(main_kind))
+    other = {k: roofline_for(wb, kinds_def, k, peak, peak_note, traffic(k)) for k in kinds_def if k != main_kind}
     step_time = {k: round(sum(ms for _, ms in v) / args.steps, 3) for k, v in kinds_def.items()}
 
     e2e = None

@@ -39,8 +39,6 @@
 //                 shared memory, no block barrier). It may start while
 //                 replay_prep still runs: it issues its base loads first and
 //                 waits for the prep grid only before reading the workspace.
-#include <mutex>
-
 #include "launch.h"
 
 namespace dl {
@@ -465,26 +463,20 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
 // replay_prep writes every (x_0, w) value the decode kernel then reads.
 static __device__ __align__(256) float g_noalloc_work[DL_NOALLOC_WORK_BYTES / sizeof(float)];
 
-// Device address of g_noalloc_work on the current device. Host code may not
+// Device address of g_noalloc_work in the current context. Host code may not
 // hand the symbol itself to a kernel (on the host it names a host-side
-// stand-in), so the address is looked up with cudaGetSymbolAddress once per
-// device, with that device current, and cached.
+// stand-in), so the address is looked up with cudaGetSymbolAddress, with the
+// caller's device current. The lookup is made on every call rather than
+// cached: the array belongs to the module loaded in one context, and after a
+// device or primary-context reset (or under a context the caller made itself)
+// a cached address would point at memory the array no longer occupies. Once
+// the module is loaded in a context the lookup is a host-side table read; the
+// first call in a context may load the module.
 static cudaError_t noalloc_work_address(float **out) {
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static float *addr[kMaxDevices] = {};
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    float *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress((void **)&ptr, g_noalloc_work);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        float *ptr = nullptr;
-        e = cudaGetSymbolAddress((void **)&ptr, g_noalloc_work);
-        if (e != cudaSuccess) return e;
-        addr[dev] = ptr;
-    }
-    *out = addr[dev];
+    *out = ptr;
     return cudaSuccess;
 }
 

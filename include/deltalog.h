@@ -218,10 +218,13 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind,
  * the library, which every device that loads the library keeps until the
  * process exits.
  *   Limit      B * H * (d_k + d_v) * 4 <= DL_NOALLOC_WORK_BYTES (16 MiB, e.g.
- *              B * H = 8192 heads at d_k = d_v = 128); larger -> DL_ERR_UNSUPPORTED.
- *   Set-up     the first call on each device looks up the array's device
- *              address (cudaGetSymbolAddress) with that device current; make
- *              that first call before any stream capture.
+ *              B * H = 16384 heads at d_k = d_v = 128); larger -> DL_ERR_UNSUPPORTED.
+ *   Set-up     every call looks up the array's device address in the current
+ *              context (cudaGetSymbolAddress, with the caller's device
+ *              current), so the address stays right after a device reset or
+ *              under a context the caller made. The first call in a context
+ *              may load the library's module there; make that first call
+ *              before any stream capture.
  *   Sharing    every call uses the same array and leaves its contents behind;
  *              calls whose work overlaps on the GPU (other streams or host
  *              threads) race on it, so the caller must serialise them. No

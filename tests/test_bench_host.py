@@ -156,3 +156,48 @@ def test_reference_arm_prints_one_oracle_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert "the same 2 of 2 (b,h) heads" in d["cpu_baseline"]["sample"]
+
+
+def test_traffic_record_is_used_only_on_the_sources_it_was_taken_on(tmp_path):
+    """roofline.traffic comes from the committed JSON record of ncu DRAM bytes,
+    keyed by kernel, workload and L, and only while the kernel sources still
+    hash to the value recorded with them."""
+    import json
+
+    srcs = ["gated_delta_rule_104_b200/csrc/deferred_read.cu", "gated_delta_rule_104_b200/csrc/common.cuh"]
+    rec = {bench.traffic_key("append_read", "w", 16): {"dram_bytes_per_launch": 123.0, "sources": srcs,
+                                                      "source_sha256_16": bench.kernel_source_hash(srcs)},
+           bench.traffic_key("merge_read", "w", 16): {"dram_bytes_per_launch": 9.0, "sources": srcs,
+                                                     "source_sha256_16": "0" * 16}}
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(rec))
+    assert bench.profiled_traffic("append_read", "w", 16, str(p)) == 123.0
+    assert bench.profiled_traffic("merge_read", "w", 16, str(p)) is None  # stale hash
+    assert bench.profiled_traffic("append_read", "w", 8, str(p)) is None  # no record for this L
+    assert bench.profiled_traffic("append_read", "w", 16, str(tmp_path / "missing.json")) is None
+    # the committed record parses and names existing sources
+    committed = json.load(open(bench.TRAFFIC_RECORD))
+    for key, r in committed.items():
+        assert key.count("/") == 2 and r["dram_bytes_per_launch"] > 0
+        for s in r["sources"]:
+            assert os.path.exists(os.path.join(os.path.dirname(bench.__file__), s)), s
+
+
+def test_sweep_plan_bytes_per_token():
+    """The sweep's bytes per token: eager is 2 states + inputs per head-step;
+    the fused deferred plan at L = 1 is one merge-read per step (the same bytes
+    as eager); at larger L it is below eager."""
+    w = W.WORKLOADS["kda_b128_h16_d128_t2048"]
+    w = W.scaled(w, T=64)
+
+    def plan(schedule, L):
+        lau = bench.Launcher(None, w, None, None, None, None, schedule, None)
+        lau.L = L
+        return lau.plan()
+
+    eager = bench.decode_bytes(w, plan("eager", 0))
+    assert eager == w.T * bench.alg_bytes(w, "eager", 0)
+    assert bench.decode_bytes(w, plan("fused", 1)) == w.T * bench.alg_bytes(w, "merge_read", 0)
+    assert bench.alg_bytes(w, "merge_read", 0) == bench.alg_bytes(w, "eager", 0)
+    for L in (4, 8, 16):
+        assert bench.decode_bytes(w, plan("fused", L)) < eager
