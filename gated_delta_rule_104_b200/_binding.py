@@ -18,12 +18,12 @@ DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = ra
 DL_F32, DL_BF16, DL_I8 = 0, 1, 2
 DL_DECAY_HEAD, DL_DECAY_CHANNEL, DL_RWKV6 = 0, 1, 2
 DL_MAX_LOG = 64
-ABI_VERSION = 7
+ABI_VERSION = 8
 
 EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read", "dl_log_merge",
            "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_pool_step",
            "dl_pool_flush", "dl_state_bytes", "dl_state_to_i8", "dl_state_from_i8", "dl_status_string",
-           "dl_last_error", "dl_abi_version")
+           "dl_last_error", "dl_abi_version", "dl_device_faults")
 DL_NOALLOC_WORK_BYTES = 16 << 20
 
 
@@ -86,6 +86,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dl_log_work_bytes.restype = ctypes.c_size_t
     lib.dl_abi_version.argtypes = []
     lib.dl_abi_version.restype = ctypes.c_int
+    lib.dl_device_faults.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]
+    lib.dl_device_faults.restype = ctypes.c_int
     if lib.dl_abi_version() != ABI_VERSION:
         raise RuntimeError(f"libdeltalog.so ABI {lib.dl_abi_version()} != binding ABI {ABI_VERSION}: rebuild")
     if path is None:
@@ -324,6 +326,14 @@ def dl_log_merge(S_base, log: Log, n: int, stream=None) -> None:
     status = load().dl_log_merge(_state_ptr(S_base, "S_base"), _state_code(S_base), log.kind, ctypes.byref(ls),
                                  int(n), B, H, dk, dv, st)
     check("dl_log_merge", status)
+
+
+def dl_device_faults(clear: bool = False) -> int:
+    """The kernels' fault word on the current device (0: no bounded wait ran
+    out). Synchronises the device."""
+    w = ctypes.c_uint(0)
+    check("dl_device_faults", load().dl_device_faults(ctypes.byref(w), 1 if clear else 0))
+    return int(w.value)
 
 
 def dl_status_string(status: int) -> str:

@@ -381,4 +381,10 @@ size_t dl_log_work_bytes(int B, int H, int d_k, int d_v) {
 
 int dl_abi_version(void) { return DL_ABI_VERSION; }
 
+dl_status dl_device_faults(unsigned int *flags, int clear) {
+    if (!flags) return fail(DL_ERR_INVALID_ARG, "flags is a null pointer");
+    *flags = 0;
+    return cuda_status(dl::read_tc_faults(flags, clear != 0), "fault word read");
+}
+
 }  // extern "C"

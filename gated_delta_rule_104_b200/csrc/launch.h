@@ -99,6 +99,14 @@ cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg,
 // entry, and then o = S_new q) into the base.
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,
                          cudaStream_t st, const PoolIdx &pool = PoolIdx{}, int part = POOL_MERGE_FULL);
+// The same merge on the tcgen05 tensor cores (merge_tc.cu), for the cases
+// merge_tc_supported() accepts: an fp32 base, d_k = 128, d_v a multiple of
+// 128, 1..16 entries in all, no slot pool.
+bool merge_tc_supported(const StepParams &p, int n_log, bool with_cur, const PoolIdx &pool);
+cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st);
+// The tensor-core kernels' fault word (bit 0: a bounded wait ran out), read
+// synchronously; cleared afterwards when `clear`.
+cudaError_t read_tc_faults(unsigned int *out, bool clear);
 // State conversions to / from the int8 layout (rows = B*H*d_v rows of d_k).
 cudaError_t launch_to_i8(const void *S, dl_dtype s_dt, void *S_i8, long long rows, int dk, cudaStream_t st);
 cudaError_t launch_from_i8(const void *S_i8, void *S, dl_dtype s_dt, long long rows, int dk, cudaStream_t st);

@@ -1,0 +1,576 @@
+// Merge of the bounded log into an fp32 base on the 5th-generation tensor
+// cores (DeltaLog page, "Core Mechanism: Base + Log", the merge phase: the
+// base absorbs every update the log holds and the log starts empty again),
+// alone or fused with one step's read.
+//
+// The arithmetic is the log-decay form of merge.cu (same symbols): for a
+// block of n <= 16 entries with decays a_i, keys k_i, values v_i, strengths
+// beta_i, per 128-row tile S of one head
+//   G     = S Khat^T,          Khat_i = gamma_i o k_i, gamma_i = prod_{m<=i} a_m
+//   delta = X (V - G)          X = (I + Diag(beta) C)^{-1} Diag(beta), kept with the log
+//   S    <- S o gamma_{n-1} + delta F,   F_j = k_j o prod_{m=j+1..n-1} a_m
+// (RWKV6: delta = V, no G). The fused read's own entry is the block's last,
+// and its X row is formed here from C(n, j) = F_n . F_j.
+//
+// Both products run as tcgen05.mma kind::tf32 with fp32 accumulators in
+// tensor memory. A TF32 operand read keeps the top 19 bits of each fp32 word
+// (the rest are ignored), so every operand x is split as hi + lo with
+// hi = x with its low 13 mantissa bits cleared and lo = x - hi (exact), and
+// each product is formed from the three terms hi*hi + hi*lo + lo*hi (lo*lo
+// is below fp32 resolution; G also takes it, at no cost). The state tile,
+// as the TMA load leaves it in shared memory, is already its own hi part.
+//   G:        D_G[:, 0:16]  = S_hi Khat_hi^T + S_lo Khat_hi^T
+//             D_G[:, 16:32] = S_hi Khat_lo^T + S_lo Khat_lo^T    (N = 32)
+//             A = the state tile (shared memory) or S_lo (tensor memory),
+//             B = [Khat_hi; Khat_lo] (shared memory), 16 + 16 MMAs of K = 8
+//   write-back: D = delta_hi F_hi + delta_hi F_lo + delta_lo F_hi    (N = 128)
+//             A = [delta_hi | delta_lo] (tensor memory), B = [F_hi | F_lo]
+//             (shared memory), 6 MMAs of K = 8
+//
+// CTA: one per SM, persistent over units (unit = (head, 128-row tile)), in
+// these roles:
+//   warp 0    loads: the unit's state tile by TMA (four 32-column boxes,
+//             128-byte swizzle) and its raw log entries and X block
+//             (cp.async; the few scalars by plain loads issued first) into one
+//             of two stages; after the unit is merged, stores the tile back by
+//             TMA and refills the stage with the unit two ahead;
+//   warp 1, 2 issue the products of compute group 0, 1 (one thread each);
+//             warp 1 also allocates tensor memory;
+//   groups    NWG (two when their operand tiles fit the shared memory beside
+//             the stages, else one) groups of 4 warps; group w merges units
+//             w, w + NWG, ... with its own operand tiles and its own 256
+//             columns of tensor memory, so one group works while the other's
+//             products run. Thread t of a group owns state row
+//             r = 32 (warp % 4) + lane (its tensor-memory lane) and key
+//             channel c = r. Per unit: Khat, F and gamma from the raw entries
+//             (and the fused entry's X row), S_lo into tensor memory, then
+//             delta from G, then the write-back S o gamma + D into the tile
+//             (and o = S_new q for the fused read).
+// Every wait on an mbarrier is bounded; a wait that runs out sets a bit of
+// the module's fault word and the CTA drains and returns.
+#include "launch.h"
+#include "merge_tc_layout.h"
+#include "tc.cuh"
+
+namespace dl {
+
+// Fault word of the tensor-core kernels (bit 0: a bounded wait ran out).
+__device__ unsigned int g_tc_faults = 0;
+
+namespace {
+
+using namespace mtc;
+
+// ---------------------------------------------------------------- bounded waits
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for the phase of `bar` with parity `par`; gives up after about two
+// seconds, or at once once another role has given up (*abort set).
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t par, volatile int *abort) {
+    if (tc::mbar_try_wait(bar, par)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 0;; ++i) {
+        if (tc::mbar_try_wait(bar, par)) return true;
+        if ((i & 63u) == 63u) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > 2000000000ull) {
+                *abort = 1;
+                atomicOr(&g_tc_faults, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_async_bar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+
+// Unit index -> (batch head, first row of the tile).
+struct Unit {
+    long long head;
+    int row0;
+};
+__device__ __forceinline__ Unit unit_of(long long u, int tiles) { return {u / tiles, (int)(u % tiles) * ROWS}; }
+
+template <class IT>
+__device__ __forceinline__ float ld_in(const IT *p) {
+    return to_f(*p);
+}
+
+// ---------------------------------------------------------------- kernel
+
+// cp.async of 4 bytes (the X block's floats: rows of the log's [L, L] matrix
+// are only 4-byte aligned).
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+template <class IT, int KIND, bool WITH_CUR, int NWG>
+__global__ void __launch_bounds__(threads_for(NWG), 1)
+merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict__ log_k, const IT *__restrict__ log_v,
+                const IT *__restrict__ log_b, const IT *__restrict__ log_a, const float *__restrict__ log_x, int L,
+                int n_log, const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
+                const IT *__restrict__ beta, const IT *__restrict__ a, float *__restrict__ o, int DV,
+                long long units) {
+    constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
+    constexpr Layout LY{sizeof(IT), CHAN, NWG};
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + LY.off_bar());
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY.off_tslot());
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + LY.off_abort());
+    auto B_FULL = [&](int s) { return &bars[s]; };
+    auto B_FREE = [&](int s) { return &bars[NS + s]; };
+    auto B_LO = [&](int w) { return &bars[2 * NS + 4 * w + 0]; };
+    auto B_G = [&](int w) { return &bars[2 * NS + 4 * w + 1]; };
+    auto B_DELTA = [&](int w) { return &bars[2 * NS + 4 * w + 2]; };
+    auto B_D = [&](int w) { return &bars[2 * NS + 4 * w + 3]; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tiles = DV / ROWS;
+    const int nb = n_log + (WITH_CUR ? 1 : 0);  // entries merged (<= NB)
+    const int n_mine = units > blockIdx.x ? (int)((units - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            tc::mbar_init(B_FULL(s), 1 + 32);  // TMA bytes + the loader lanes' cp.async arrivals
+            tc::mbar_init(B_FREE(s), 1);
+        }
+        for (int w = 0; w < NWG; ++w) {
+            tc::mbar_init(B_LO(w), 1);
+            tc::mbar_init(B_G(w), 1);
+            tc::mbar_init(B_DELTA(w), 1);
+            tc::mbar_init(B_D(w), 1);
+        }
+        *abort = 0;
+        tc::mbar_init_fence();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tslot, tmem_cols_for(NWG));
+        tc::tmem_relinquish();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tbase = *tslot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ loads
+        if (lane == 0) tc::tma_prefetch_desc(&map_s);
+        for (int i = 0; i < n_mine; ++i) {
+            const int s = i % NS;
+            if (i >= NS && !wait_bar(B_FREE(s), (uint32_t)((i / NS - 1) & 1), abort)) break;
+            uint8_t *st = sm + LY.stage(s);
+            const Unit un = unit_of((long long)blockIdx.x + (long long)i * gridDim.x, tiles);
+            const long long lrow = un.head * L;
+            uint64_t *full = B_FULL(s);
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(full, (uint32_t)LY.tile());
+                for (int ch = 0; ch < NCHUNK; ++ch)
+                    tc::tma_load_2d(st + LY.off_tile() + ch * (ROWS * 128), &map_s, ch * CHUNK,
+                                    (int)(un.head * DV + un.row0), full);
+            }
+            // raw entries 0..nb-1: logged ones from the log, the fused read's own from the inputs
+            constexpr int E = 16 / (int)sizeof(IT);  // elements per 16-byte chunk
+            constexpr int KC = DK / E, VC = ROWS / E;
+            uint8_t *rk = st + LY.off_raw_k(), *ra = st + LY.off_raw_a(), *rv = st + LY.off_raw_v();
+            for (int u = lane; u < nb * KC; u += 32) {
+                const int e = u / KC, col = (u % KC) * E;
+                const IT *srck = e < n_log ? log_k + (lrow + e) * DK : k + un.head * DK;
+                cp_async16(rk + raw_k_off(e, col, sizeof(IT)), srck + col);
+                if constexpr (CHAN) {
+                    const IT *srca = e < n_log ? log_a + (lrow + e) * DK : a + un.head * DK;
+                    cp_async16(ra + raw_k_off(e, col, sizeof(IT)), srca + col);
+                }
+            }
+            for (int u = lane; u < nb * VC; u += 32) {
+                const int e = u / VC, col = (u % VC) * E;
+                const IT *srcv = e < n_log ? log_v + (lrow + e) * DV : v + un.head * DV;
+                cp_async16(rv + raw_v_off(e, col, sizeof(IT)), srcv + un.row0 + col);
+            }
+            if (WITH_CUR && lane < KC)
+                cp_async16(st + LY.off_raw_q() + raw_q_off(lane * E, sizeof(IT)), q + un.head * DK + lane * E);
+            if constexpr (DELTA) {  // the X block: X(j, e), e <= j < n_log
+                uint8_t *sc = st + LY.off_sc();
+                for (int u = lane; u < NB * NB; u += 32) {
+                    const int j = u / NB, e = u % NB;
+                    if (j < n_log && e <= j) cp_async4(sc + sc_x(j, e), log_x + (lrow + j) * L + e);
+                }
+            }
+            cp_async_bar_arrive(full);
+        }
+        cp_async_wait_all();
+    } else if (warp >= 1 && warp <= NWG) {
+        // ------------------------------------------------ products of group w (one thread)
+        const int w = warp - 1;
+        if (lane == 0) {
+            constexpr uint32_t ID_G = tc::instr_desc(tc::FMT_TF32, false, false, ROWS, 2 * NB);
+            constexpr uint32_t ID_W = tc::instr_desc(tc::FMT_TF32, false, false, ROWS, DK);
+            const uint32_t kf = tc::smem_u32(sm + LY.group(w) + LY.g_kf());
+            const uint32_t tw = tbase + (uint32_t)w * TMEM_COLS_PER_GROUP;
+            for (int j = 0, i = w; i < n_mine; ++j, i += NWG) {
+                const int s = i % NS;
+                const uint32_t par = (uint32_t)(j & 1);
+                if constexpr (DELTA) {
+                    if (!wait_bar(B_LO(w), par, abort)) break;
+                    tc::tc_fence_after();
+                    const uint32_t tile = tc::smem_u32(sm + LY.stage(s) + LY.off_tile());
+#pragma unroll
+                    for (int kk = 0; kk < DK / 8; ++kk) {
+                        const uint64_t ad = tc::smem_desc(tile + g_a_start(kk), 16, 1024, tc::SWZ_128);
+                        const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                        tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < DK / 8; ++kk) {
+                        const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                        tc::mma_ts_tf32(tw + COL_G, tw + COL_B + 8 * kk, bd, ID_G, true);
+                    }
+                    tc::mma_commit(B_G(w));
+                }
+                if (!wait_bar(B_DELTA(w), par, abort)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int m = 0; m < 6; ++m) {  // region B holds S o gamma: accumulate onto it
+                    const uint64_t bd = tc::smem_desc(kf + wb_b_start(m), 16, 1024, tc::SWZ_128);
+                    tc::mma_ts_tf32(tw + COL_B, tw + COL_DL + wb_a_col(m), bd, ID_W, true);
+                }
+                tc::mma_commit(B_D(w));
+            }
+        }
+        __syncwarp();
+    } else if (warp >= CTRL_WARPS) {
+        // ------------------------------------------------ compute group w (128 threads)
+        const int w = (warp - CTRL_WARPS) / 4;
+        const int ct = tid - 32 * CTRL_WARPS - 128 * w;  // 0..127
+        const int quad = warp & 3;                       // tensor-memory lane quadrant
+        const int r = 32 * quad + lane;                  // state row of this thread (and its key channel)
+        const int c = r;
+        const uint32_t trow = tbase + (uint32_t)w * TMEM_COLS_PER_GROUP + ((uint32_t)(32 * quad) << 16);
+        uint8_t *gp = sm + LY.group(w);
+        float *gam = reinterpret_cast<float *>(gp + LY.g_gam());
+        float *qf = reinterpret_cast<float *>(gp + LY.g_qf());
+        float *cn = reinterpret_cast<float *>(gp + LY.g_cn());
+        float *red = reinterpret_cast<float *>(gp + LY.g_red());
+        uint8_t *kf = gp + LY.g_kf();
+        uint8_t *out = gp + LY.g_out();
+        const int bar_id = 1 + w;
+        for (int j = 0, i = w; i < n_mine; ++j, i += NWG) {
+            const int s = i % NS;
+            const uint32_t par = (uint32_t)(j & 1);
+            uint8_t *st = sm + LY.stage(s);
+            uint8_t *tile = st + LY.off_tile();
+            const IT *rk = reinterpret_cast<const IT *>(st + LY.off_raw_k());
+            const IT *ra = reinterpret_cast<const IT *>(st + LY.off_raw_a());
+            const IT *rv = reinterpret_cast<const IT *>(st + LY.off_raw_v());
+            const IT *rq = reinterpret_cast<const IT *>(st + LY.off_raw_q());
+            uint8_t *sc = st + LY.off_sc();
+            auto scf = [&](size_t off) { return *reinterpret_cast<const float *>(sc + off); };
+            const Unit un = unit_of((long long)blockIdx.x + (long long)i * gridDim.x, tiles);
+            const long long lrow = un.head * L;
+            // the unit's scalars straight from global memory, before the wait:
+            // head-wise decays of every entry (each thread needs all of them) and
+            // the fused entry's beta
+            float adec[NB];
+#pragma unroll
+            for (int e = 0; e < NB; ++e) {
+                adec[e] = 1.f;
+                if (!CHAN && e < nb) adec[e] = e < n_log ? ld_in(log_a + lrow + e) : ld_in(a + un.head);
+            }
+            const float bcur = (DELTA && WITH_CUR) ? ld_in(beta + un.head) : 0.f;
+            if (!wait_bar(B_FULL(s), (uint32_t)((i / NS) & 1), abort)) break;
+
+            // 1. key side for channel c: Khat (hi and lo parts), F, gamma, q
+            float kc[NB], ac[NB];
+#pragma unroll
+            for (int e = 0; e < NB; ++e) {
+                const bool real = e < nb;
+                kc[e] = real ? to_f(rk[raw_k_off(e, c, 1)]) : 0.f;
+                ac[e] = real ? (CHAN ? to_f(ra[raw_k_off(e, c, 1)]) : adec[e]) : 1.f;
+            }
+            {
+                float g = 1.f;
+#pragma unroll
+                for (int e = 0; e < NB; ++e) {
+                    g *= ac[e];
+                    if constexpr (DELTA) {
+                        const float x = g * kc[e], hi = tc::tf32_trunc(x);
+                        *reinterpret_cast<float *>(kf + kh_off(e, c)) = hi;
+                        *reinterpret_cast<float *>(kf + kh_off(NB + e, c)) = x - hi;
+                    }
+                }
+                gam[c] = g;
+                if constexpr (WITH_CUR) qf[c] = to_f(rq[raw_q_off(c, 1)]);
+            }
+            float fv[NB];  // F_e[c] (kept until G has been read; then it replaces Khat)
+            {
+                float f = 1.f;
+#pragma unroll
+                for (int e = NB - 1; e >= 0; --e) {
+                    fv[e] = kc[e] * f;
+                    f *= ac[e];
+                }
+            }
+            // 2. S_lo = S - hi(S) into region B (row r); then G may start
+            if constexpr (DELTA) {
+#pragma unroll
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    uint32_t lo[32];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, ch * CHUNK + 4 * u));
+                        lo[4 * u + 0] = __float_as_uint(x.x - tc::tf32_trunc(x.x));
+                        lo[4 * u + 1] = __float_as_uint(x.y - tc::tf32_trunc(x.y));
+                        lo[4 * u + 2] = __float_as_uint(x.z - tc::tf32_trunc(x.z));
+                        lo[4 * u + 3] = __float_as_uint(x.w - tc::tf32_trunc(x.w));
+                    }
+                    tc::tmem_st32(trow + COL_B + ch * CHUNK, lo);
+                }
+                tc::tmem_wait_st();
+                tc::fence_async_smem();  // Khat is read by the tensor cores
+                tc::tc_fence_before();
+                tc::named_sync(bar_id, 128);
+                if (ct == 0) tc::mbar_arrive(B_LO(w));
+            } else {
+                tc::named_sync(bar_id, 128);  // gamma and q of every channel are in place
+            }
+            // 3. while G runs: the fused read's entry (index nb - 1) gets its X row
+            //    from C(nb-1, e) = F_{nb-1} . F_e
+            if (DELTA && WITH_CUR) {
+                const int nl = nb - 1;
+                const float fn = to_f(rk[raw_k_off(nl, c, 1)]);  // F_{nb-1} = k_{nb-1}: every later factor is a padded 1
+                float p[NB];
+#pragma unroll
+                for (int e = 0; e < NB; ++e) p[e] = e < nl ? fn * fv[e] : 0.f;
+                multi_sum<NB>(p, lane);  // lane l: this warp's sum for entry l >> 1
+                if ((lane & 1) == 0) red[quad * NB + (lane >> 1)] = p[0];
+                tc::named_sync(bar_id, 128);
+                if (ct < NB) cn[ct] = red[ct] + red[NB + ct] + red[2 * NB + ct] + red[3 * NB + ct];
+                tc::named_sync(bar_id, 128);
+                if (ct <= nl) {
+                    // X(nl, ct) = -beta_nl sum_{m = ct..nl-1} C(nl, m) X(m, ct); X(nl, nl) = beta_nl
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m < NB; ++m)
+                        if (m >= ct && m < nl) acc = fmaf(cn[m], scf(sc_x(m, ct)), acc);
+                    *reinterpret_cast<float *>(sc + sc_x(nl, ct)) = ct == nl ? bcur : -bcur * acc;
+                }
+                tc::named_sync(bar_id, 128);
+            }
+            float vr[NB];
+#pragma unroll
+            for (int e = 0; e < NB; ++e) vr[e] = e < nb ? to_f(rv[raw_v_off(e, r, 1)]) : 0.f;
+
+            // 4. delta = X (V - G) for row r (RWKV6: delta = V) into A[32, 64)
+            float dl[NB];
+            if constexpr (DELTA) {
+                if (!wait_bar(B_G(w), par, abort)) break;
+                tc::tc_fence_after();
+                uint32_t gr[32];
+                tc::tmem_ld32(trow + COL_G, gr);
+                tc::tmem_wait_ld();
+                float ev[NB];
+#pragma unroll
+                for (int e = 0; e < NB; ++e) ev[e] = vr[e] - (__uint_as_float(gr[e]) + __uint_as_float(gr[NB + e]));
+#pragma unroll
+                for (int e = 0; e < NB; ++e) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m <= e; ++m) acc = fmaf(scf(sc_x(e, m)), ev[m], acc);
+                    dl[e] = e < nb ? acc : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < NB; ++e) dl[e] = vr[e];
+            }
+            {
+                uint32_t wd[32];
+#pragma unroll
+                for (int e = 0; e < NB; ++e) {
+                    const float hi = tc::tf32_trunc(dl[e]);
+                    wd[e] = __float_as_uint(hi);
+                    wd[NB + e] = __float_as_uint(dl[e] - hi);
+                }
+                tc::tmem_st32(trow + COL_DL, wd);
+            }
+            // 5. S o gamma into region B (S_lo there has been read by G), F over Khat
+#pragma unroll
+            for (int ch = 0; ch < NCHUNK; ++ch) {
+                uint32_t y[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int col = ch * CHUNK + 4 * u;
+                    const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, col));
+                    const float4 gv = *reinterpret_cast<const float4 *>(gam + col);
+                    y[4 * u + 0] = __float_as_uint(x.x * gv.x);
+                    y[4 * u + 1] = __float_as_uint(x.y * gv.y);
+                    y[4 * u + 2] = __float_as_uint(x.z * gv.z);
+                    y[4 * u + 3] = __float_as_uint(x.w * gv.w);
+                }
+                tc::tmem_st32(trow + COL_B + ch * CHUNK, y);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {  // 16-byte pieces: hi of entries 4u.. (u < 4), lo (u >= 4)
+                float4 wv;
+                float *wp = reinterpret_cast<float *>(&wv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x = fv[(4 * u + e) % NB], hi = tc::tf32_trunc(x);
+                    wp[e] = u < 4 ? hi : x - hi;
+                }
+                *reinterpret_cast<float4 *>(kf + ff_off(c, 4 * u)) = wv;
+            }
+            tc::tmem_wait_st();
+            tc::fence_async_smem();  // F is read by the tensor cores
+            tc::tc_fence_before();
+            tc::named_sync(bar_id, 128);
+            if (ct == 0) {
+                tc::mbar_arrive(B_DELTA(w));
+                tc::mbar_arrive(B_FREE(s));  // the unit reads nothing more of its stage
+            }
+
+            // 6. S_new = region B after the write-back: o = S_new q for the fused
+            //    read, and the rows to HBM by TMA, one 32-column chunk at a time
+            //    through the group's staging tile
+            if (!wait_bar(B_D(w), par, abort)) break;
+            tc::tc_fence_after();
+            float oacc = 0.f;
+#pragma unroll 1
+            for (int ch = 0; ch < NCHUNK; ++ch) {
+                uint32_t d[32];
+                tc::tmem_ld32(trow + COL_B + ch * CHUNK, d);
+                if (ct == 0) tc::bulk_wait_read<0>();  // the staging tile's previous store has read it
+                tc::tmem_wait_ld();
+                tc::named_sync(bar_id, 128);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int col = ch * CHUNK + 4 * u;
+                    const float4 y = make_float4(__uint_as_float(d[4 * u + 0]), __uint_as_float(d[4 * u + 1]),
+                                                 __uint_as_float(d[4 * u + 2]), __uint_as_float(d[4 * u + 3]));
+                    *reinterpret_cast<float4 *>(out + tile_off(r, 4 * u)) = y;
+                    if constexpr (WITH_CUR) {
+                        const float4 qv = *reinterpret_cast<const float4 *>(qf + col);
+                        oacc = fmaf(y.x, qv.x, fmaf(y.y, qv.y, fmaf(y.z, qv.z, fmaf(y.w, qv.w, oacc))));
+                    }
+                }
+                tc::fence_async_smem();  // the staging tile is read by the TMA store
+                tc::named_sync(bar_id, 128);
+                if (ct == 0) {
+                    tc::tma_store_2d(&map_s, ch * CHUNK, (int)(un.head * DV + un.row0), out);
+                    tc::bulk_commit();
+                }
+            }
+            if constexpr (WITH_CUR) o[un.head * DV + un.row0 + r] = oacc;
+            tc::tc_fence_before();  // region B is rewritten by the group's next unit
+        }
+        if (ct == 0) tc::bulk_wait_all();  // the group's last stores have landed
+    }
+    // drain: every role has left its loop; products in flight have completed
+    // (the compute warps waited for the last one, or the CTA gave up)
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tbase, tmem_cols_for(NWG));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); looked up once.
+EncodeTiledFn encoder() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// The fp32 state [rows, 128] as a tensor map of 32-column x 128-row boxes,
+// 128-byte swizzle.
+cudaError_t state_map(CUtensorMap *m, void *S, unsigned long long rows) {
+    EncodeTiledFn fn = encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)DK, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)DK * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)CHUNK, (cuuint32_t)ROWS};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, S, dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <class IT, int KD, bool WC>
+cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
+    constexpr int NWG = groups_for(sizeof(IT), Rule<KD>::CHAN);
+    constexpr Layout LY{sizeof(IT), Rule<KD>::CHAN, NWG};
+    static_assert(LY.request() <= SMEM_LIMIT, "layout fits the shared memory a block may request");
+    auto kern = merge_tc_kernel<IT, KD, WC, NWG>;
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), LY.request());
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long heads = (long long)p.B * p.H;
+    CUtensorMap map;
+    e = state_map(&map, p.S, (unsigned long long)heads * p.dv);
+    if (e != cudaSuccess) return e;
+    const long long units = heads * (p.dv / ROWS);
+    const unsigned grid = (unsigned)std::min<long long>(units, sms);
+    kern<<<grid, threads_for(NWG), LY.request(), st>>>(
+        map, static_cast<const IT *>(lg.k), static_cast<const IT *>(lg.v), static_cast<const IT *>(lg.beta),
+        static_cast<const IT *>(lg.a), lg.x, lg.L, n_log, static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
+        static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), p.o, p.dv,
+        units);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool merge_tc_supported(const StepParams &p, int n_log, bool with_cur, const PoolIdx &pool) {
+    const long long rows = (long long)p.B * p.H * p.dv;
+    return pool.slot == nullptr && p.s_dt == DL_F32 && p.dk == DK && p.dv % ROWS == 0 &&
+           n_log + (with_cur ? 1 : 0) <= NB && n_log + (with_cur ? 1 : 0) >= 1 && rows < (1LL << 31) &&
+           encoder() != nullptr;
+}
+
+cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st) {
+    auto with_kind = [&](auto it_t, auto kd_c) -> cudaError_t {
+        using IT = decltype(it_t);
+        constexpr int KD = decltype(kd_c)::value;
+        if (with_cur) return launch_tc_t<IT, KD, true>(p, lg, n_log, st);
+        return launch_tc_t<IT, KD, false>(p, lg, n_log, st);
+    };
+    auto with_it = [&](auto it_t) -> cudaError_t {
+        if (p.kind == DL_RWKV6) return with_kind(it_t, std::integral_constant<int, DL_RWKV6>{});
+        if (p.kind == DL_DECAY_CHANNEL) return with_kind(it_t, std::integral_constant<int, DL_DECAY_CHANNEL>{});
+        return with_kind(it_t, std::integral_constant<int, DL_DECAY_HEAD>{});
+    };
+    if (p.in_dt == DL_BF16) return with_it(bf16{});
+    return with_it(float{});
+}
+
+cudaError_t read_tc_faults(unsigned int *out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_faults, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_tc_faults, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace dl

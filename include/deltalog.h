@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 7
+#define DL_ABI_VERSION 8
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -312,6 +312,16 @@ const char *dl_last_error(void);
 
 /* DL_ABI_VERSION of the built library. */
 int dl_abi_version(void);
+
+/* Fault word of the library's kernels on the current device. The kernels that
+ * wait on on-chip barriers (the tcgen05 merge of dl_log_merge and
+ * dl_log_merge_read) bound every such wait; a wait that runs out (about two
+ * seconds; it means a bug, not a slow GPU) sets bit 0 here, abandons its work
+ * (the state it was merging is then unspecified) and returns, so the device
+ * stays usable. *flags receives the word; clear != 0 resets it to 0.
+ * Synchronous: it waits for the device's pending work (cudaMemcpyFromSymbol).
+ * No counterpart on the pages: it is a health check of this library. */
+dl_status dl_device_faults(unsigned int *flags, int clear);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,309 @@
+// Host replay of every shared-memory, tensor-memory and global address the
+// tensor-core merge kernel (gated_delta_rule_104_b200/csrc/merge_tc.cu)
+// forms, for every instantiation (input element size, channel or head decay,
+// delta rule or RWKV6, fused read or not) and every entry count it accepts.
+// It uses the same layout functions as the kernel (merge_tc_layout.h) and
+// walks the kernel's loops with their bounds, checking that each access lies
+// inside its region, is aligned for its width, that regions do not overlap,
+// that the swizzled layouts are one-to-one, that the operand tiles the
+// threads write are the ones the descriptors make the tensor cores read, and
+// that the whole layout fits the requested dynamic shared memory.
+//
+// Usage: merge_tc_replay [shrink <region> <bytes>]
+//   shrink: the bounds table believes <region> is <bytes> shorter than the
+//   layout says (a planted overrun: the replay must then fail).
+// Exit status 0: every check passed; 1: a check failed (printed).
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <set>
+#include <string>
+#include <vector>
+
+#include "merge_tc_layout.h"
+
+using namespace dl::mtc;
+
+namespace {
+
+int failures = 0;
+std::map<std::string, long> shrink;
+
+void fail(const char *what, const std::string &ctx) {
+    if (failures < 20) std::printf("FAIL %s: %s\n", what, ctx.c_str());
+    ++failures;
+}
+
+struct Region {
+    std::string name;
+    size_t off, bytes;
+};
+
+struct Replay {
+    size_t in_size;
+    bool chan, delta, with_cur;
+    Layout ly;
+    std::vector<Region> regions;
+
+    Replay(size_t in, bool ch, bool de, bool wc)
+        : in_size(in), chan(ch), delta(de), with_cur(wc), ly{in, ch, groups_for(in, ch)} {
+        for (int s = 0; s < NS; ++s) {
+            const std::string p = "stage" + std::to_string(s) + ".";
+            add(p + "tile", ly.stage(s) + ly.off_tile(), ly.tile());
+            add(p + "raw_k", ly.stage(s) + ly.off_raw_k(), ly.raw_k());
+            if (chan) add(p + "raw_a", ly.stage(s) + ly.off_raw_a(), ly.raw_a());
+            add(p + "raw_v", ly.stage(s) + ly.off_raw_v(), ly.raw_v());
+            add(p + "raw_q", ly.stage(s) + ly.off_raw_q(), ly.raw_q());
+            add(p + "sc", ly.stage(s) + ly.off_sc(), ly.sc_floats() * 4);
+        }
+        for (int w = 0; w < ly.nwg; ++w) {
+            const std::string p = "group" + std::to_string(w) + ".";
+            add(p + "kf", ly.group(w) + ly.g_kf(), ly.kf_bytes());
+            add(p + "out", ly.group(w) + ly.g_out(), ly.out_bytes());
+            add(p + "gam", ly.group(w) + ly.g_gam(), DK * 4);
+            add(p + "qf", ly.group(w) + ly.g_qf(), DK * 4);
+            add(p + "cn", ly.group(w) + ly.g_cn(), NB * 4);
+            add(p + "red", ly.group(w) + ly.g_red(), 4 * NB * 4);
+        }
+        add("bar", ly.off_bar(), (size_t)ly.nbar() * 8);
+        add("tslot", ly.off_tslot(), 4);
+        add("abort", ly.off_abort(), 4);
+    }
+    std::string tag() const {
+        char b[96];
+        std::snprintf(b, sizeof b, "in%zu %s %s %s", in_size, chan ? "chan" : "head", delta ? "delta" : "rwkv6",
+                      with_cur ? "fused" : "merge");
+        return b;
+    }
+    void add(const std::string &name, size_t off, size_t bytes) {
+        // a planted shrink applies to every stage's region of that name
+        for (auto &kv : shrink) {
+            const std::string &n = kv.first;
+            if (name == n || (name.size() > n.size() && name.compare(name.size() - n.size(), n.size(), n) == 0 &&
+                              name[name.size() - n.size() - 1] == '.'))
+                bytes = bytes > (size_t)kv.second ? bytes - kv.second : 0;
+        }
+        regions.push_back({name, off, bytes});
+    }
+    const Region &region(const std::string &name) const {
+        for (auto &r : regions)
+            if (r.name == name) return r;
+        std::printf("no region %s\n", name.c_str());
+        std::exit(2);
+    }
+    // an access of `bytes` at `off` (from the region's start) of width-aligned data
+    void acc(const std::string &name, size_t off, size_t bytes, size_t align, const char *what) {
+        const Region &r = region(name);
+        if (off + bytes > r.bytes) fail("out of region", tag() + " " + name + " " + what + " off " + std::to_string(off));
+        if ((r.off + off) % align) fail("misaligned", tag() + " " + name + " " + what);
+    }
+
+    void layout_checks() {
+        if (ly.request() > SMEM_LIMIT) fail("request above 227 KiB", tag());
+        if (ly.end() + 1023 > ly.request()) fail("no room for the 1024-byte base alignment", tag());
+        if (ly.stage_bytes() % 1024) fail("stage not 1024-aligned", tag());
+        for (int w = 0; w < ly.nwg; ++w)
+            if ((ly.group(w) + ly.g_kf()) % 1024 || (ly.group(w) + ly.g_out()) % 1024)
+                fail("operand region not 1024-aligned", tag());
+        if (ly.nwg < 1 || ly.nwg > 2 || (int)tmem_cols_for(ly.nwg) < ly.nwg * (int)TMEM_COLS_PER_GROUP)
+            fail("tensor memory for the groups", tag());
+        for (size_t i = 0; i < regions.size(); ++i) {
+            if (regions[i].off + regions[i].bytes > ly.end()) fail("region beyond the layout", regions[i].name);
+            for (size_t j = i + 1; j < regions.size(); ++j) {
+                const Region &a = regions[i], &b = regions[j];
+                if (a.bytes && b.bytes && a.off < b.off + b.bytes && b.off < a.off + a.bytes)
+                    fail("overlapping regions", a.name + " / " + b.name);
+            }
+        }
+        for (int s = 0; s < NS; ++s)
+            for (int ch = 0; ch < NCHUNK; ++ch)
+                if ((ly.stage(s) + ly.off_tile() + ch * ROWS * 128) % 1024) fail("TMA box not 1024-aligned", tag());
+    }
+
+    // warp 0: TMA boxes, cp.async of the raw entries, scalars and the X block
+    void producer(int n_log, int L) {
+        const int nb = n_log + (with_cur ? 1 : 0);
+        const int E = 16 / (int)in_size, KC = DK / E, VC = ROWS / E;
+        for (int s = 0; s < NS; ++s) {
+            const std::string p = "stage" + std::to_string(s) + ".";
+            for (int ch = 0; ch < NCHUNK; ++ch) acc(p + "tile", ch * ROWS * 128, ROWS * 128, 1024, "TMA box");
+            for (int lane = 0; lane < 32; ++lane) {
+                for (int u = lane; u < nb * KC; u += 32) {
+                    const int e = u / KC, col = (u % KC) * E;
+                    acc(p + "raw_k", raw_k_off(e, col, in_size), 16, 16, "cp.async k");
+                    if (chan) acc(p + "raw_a", raw_k_off(e, col, in_size), 16, 16, "cp.async a");
+                }
+                for (int u = lane; u < nb * VC; u += 32) {
+                    const int e = u / VC, col = (u % VC) * E;
+                    acc(p + "raw_v", raw_v_off(e, col, in_size), 16, 16, "cp.async v");
+                }
+                if (with_cur && lane < KC) acc(p + "raw_q", raw_q_off(lane * E, in_size), 16, 16, "cp.async q");
+                if (delta)
+                    for (int u = lane; u < NB * NB; u += 32) {
+                        const int j = u / NB, e = u % NB;
+                        if (j < n_log && e <= j) {
+                            acc(p + "sc", sc_x(j, e), 4, 4, "X block");
+                            // the global element read: row j < n_log <= L of the head's [L, L] block
+                            if (j >= L || e >= L) fail("X read outside the head's block", tag());
+                        }
+                    }
+            }
+        }
+    }
+
+    // compute group w: key side, fused X row, S_lo, delta, write-back (128 threads)
+    void compute(int n_log, int w) {
+        const int nb = n_log + (with_cur ? 1 : 0);
+        const std::string p = "stage" + std::to_string(w % NS) + ".";
+        const std::string gp = "group" + std::to_string(w) + ".";
+        std::set<uint32_t> khs, ffs, tiles;
+        for (int ct = 0; ct < 128; ++ct) {
+            const int warp = CTRL_WARPS + 4 * w + ct / 32, lane = ct % 32, quad = warp & 3, r = 32 * quad + lane,
+                      c = r;
+            if (warp >= threads_for(ly.nwg) / 32) fail("warp outside the block", tag());
+            if (r < 0 || r >= ROWS) fail("row outside the tile", tag());
+            for (int j = 0; j < NB; ++j) {
+                if (j < nb) {
+                    acc(p + "raw_k", raw_k_off(j, c, in_size), in_size, in_size, "k read");
+                    if (chan) acc(p + "raw_a", raw_k_off(j, c, in_size), in_size, in_size, "a read");
+                    acc(p + "raw_v", raw_v_off(j, r, in_size), in_size, in_size, "v read");
+                }
+                if (delta) {
+                    acc(gp + "kf", kh_off(j, c), 4, 4, "Khat hi");
+                    acc(gp + "kf", kh_off(NB + j, c), 4, 4, "Khat lo");
+                    khs.insert(kh_off(j, c));
+                    khs.insert(kh_off(NB + j, c));
+                    for (int m = 0; m <= j; ++m) acc(p + "sc", sc_x(j, m), 4, 4, "X read");
+                }
+            }
+            acc(gp + "gam", c * 4, 4, 4, "gamma");
+            if (with_cur) {
+                acc(gp + "qf", c * 4, 4, 4, "q widened");
+                acc(p + "raw_q", raw_q_off(c, in_size), in_size, in_size, "q raw read");
+            }
+            for (int u = 0; u < 8; ++u) {
+                acc(gp + "kf", ff_off(c, 4 * u), 16, 16, "F piece");
+                for (int e = 0; e < 4; ++e) {
+                    if (ff_off(c, 4 * u + e) != ff_off(c, 4 * u) + 4u * e) fail("F piece not contiguous", tag());
+                    ffs.insert(ff_off(c, 4 * u + e));
+                }
+            }
+            if (delta && with_cur) {
+                const int nl = nb - 1;
+                acc(p + "raw_k", raw_k_off(nl, c, in_size), in_size, in_size, "fused key");
+                if ((lane & 1) == 0) acc(gp + "red", (quad * NB + (lane >> 1)) * 4, 4, 4, "red write");
+                if (ct < NB) {
+                    for (int w = 0; w < 4; ++w) acc(gp + "red", (w * NB + ct) * 4, 4, 4, "red read");
+                    acc(gp + "cn", ct * 4, 4, 4, "cn write");
+                }
+                if (ct <= nl) {
+                    for (int m = ct; m < nl; ++m) {
+                        acc(gp + "cn", m * 4, 4, 4, "cn read");
+                        acc(p + "sc", sc_x(m, ct), 4, 4, "X read (fused row)");
+                    }
+                    acc(p + "sc", sc_x(nl, ct), 4, 4, "fused X row write");
+                }
+            }
+            for (int col = 0; col < DK; col += 4) {
+                acc(p + "tile", tile_off(r, col), 16, 16, "tile piece");
+                if (col < CHUNK) {
+                    acc(gp + "out", tile_off(r, col), 16, 16, "staging piece");
+                    if (tile_off(r, col) >= ly.out_bytes()) fail("staging piece outside the chunk", tag());
+                }
+                acc(gp + "gam", col * 4, 16, 16, "gamma piece");
+                if (with_cur) acc(gp + "qf", col * 4, 16, 16, "q piece");
+                for (int e = 0; e < 4; ++e) {
+                    if (tile_off(r, col + e) != tile_off(r, col) + 4u * e) fail("tile piece not contiguous", tag());
+                    tiles.insert(tile_off(r, col + e));
+                    (void)e;
+                }
+            }
+            // tensor memory: region B (S_lo, then S o gamma and the write-back), 4 chunks
+            for (int ch = 0; ch < NCHUNK; ++ch)
+                if (COL_B + ch * CHUNK + 32 > (int)TMEM_COLS_PER_GROUP) fail("region B columns out of range", tag());
+        }
+        if (delta && khs.size() != (size_t)2 * NB * DK) fail("Khat layout not one-to-one", tag());
+        if (ffs.size() != (size_t)DK * 2 * NB) fail("F layout not one-to-one", tag());
+        if (tiles.size() != (size_t)ROWS * DK) fail("tile layout not one-to-one", tag());
+    }
+
+    // what the descriptors make the tensor cores read: K-major, 128-byte
+    // swizzle, 8-row groups 1024 bytes apart, 32 bytes of K per step. The
+    // element (row, k) a step reads must be the one the threads wrote there.
+    static uint32_t desc_elem(uint32_t start, int row, int k) {
+        // start = group-aligned base + byte offset of the step within the 128-byte row
+        const uint32_t base = start & ~127u, within = start & 127u;
+        return base + (uint32_t)(row / 8) * 1024 + swz128((uint32_t)((row % 8) * 128) + within + 4u * k);
+    }
+    void descriptors() {
+        // G, A = the state tile: step kk reads rows 0..127, channels 8kk..8kk+7
+        for (int kk = 0; kk < DK / 8; ++kk)
+            for (int row = 0; row < ROWS; ++row)
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = desc_elem(g_a_start(kk), row, k);
+                    if (a != tile_off(row, 8 * kk + k)) fail("G's A operand is not the tile element", tag());
+                    if (delta) {
+                        if (row < 2 * NB) {
+                            const uint32_t b = desc_elem(g_b_start(kk), row, k);
+                            if (b != kh_off(row, 8 * kk + k)) fail("G's B operand is not the Khat element", tag());
+                            if (b + 4 > ly.kf_bytes()) fail("G's B read outside Khat", tag());
+                        }
+                    }
+                    if (a + 4 > ly.tile()) fail("G's A read outside the tile", tag());
+                }
+        // write-back, B = F: step m reads rows (channels) 0..127, entries of its 8-column slice
+        for (int m = 0; m < 6; ++m) {
+            const int jbase = (m < 4 ? m : m - 4) * 8;  // column of F in [hi 0..15 | lo 16..31]
+            for (int row = 0; row < DK; ++row)
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t b = desc_elem(wb_b_start(m), row, k);
+                    if (b != ff_off(row, jbase + k)) fail("write-back's B operand is not the F element", tag());
+                    if (b + 4 > ly.kf_bytes()) fail("write-back's B read outside F", tag());
+                }
+            // A in tensor memory: delta columns of the same entries (hi for m < 4, lo after)
+            const int acol = COL_DL + wb_a_col(m);
+            const int entry0 = (m % 2) * 8, part = m < 4 ? 0 : 1;  // which half of [hi | lo]
+            if (acol != COL_DL + part * NB + entry0) fail("write-back's A columns", tag());
+            const bool b_lo = (m == 2 || m == 3);
+            if ((b_lo ? NB : 0) + entry0 != jbase) fail("write-back pairs the wrong F half", tag());
+            if (acol + 8 > (int)TMEM_COLS_PER_GROUP) fail("tensor-memory column out of range", tag());
+        }
+        // G's second product: A = S_lo in region B, columns COL_B + 8kk
+        for (int kk = 0; kk < DK / 8; ++kk)
+            if (COL_B + 8 * kk + 8 > (int)TMEM_COLS_PER_GROUP) fail("S_lo A columns out of range", tag());
+        // region A: G [COL_G, +32) and delta [COL_DL, +32) apart and below region B
+        if (COL_G + 2 * NB > COL_DL || COL_DL + 2 * NB > COL_B || COL_B + DK > (int)TMEM_COLS_PER_GROUP)
+            fail("tensor-memory regions overlap or overflow", tag());
+    }
+};
+
+}  // namespace
+
+int main(int argc, char **argv) {
+    for (int i = 1; i < argc; ++i) {
+        if (std::strcmp(argv[i], "shrink") == 0 && i + 2 < argc) {
+            shrink[argv[i + 1]] = std::atol(argv[i + 2]);
+            i += 2;
+        }
+    }
+    int cases = 0;
+    for (size_t in : {2, 4})
+        for (int chan = 0; chan < 2; ++chan)
+            for (int delta = 0; delta < 2; ++delta)
+                for (int wc = 0; wc < 2; ++wc) {
+                    if (!delta && !chan) continue;  // RWKV6 has channel decay
+                    Replay rp(in, chan, delta, wc);
+                    rp.layout_checks();
+                    rp.descriptors();
+                    for (int n_log = wc ? 0 : 1; n_log + wc <= NB; ++n_log) {
+                        // L: the log capacity; fused reads need n_log < L, merges n_log <= L
+                        const int L = wc ? n_log + 1 : n_log;
+                        rp.producer(n_log, L);
+                        for (int w = 0; w < rp.ly.nwg; ++w) rp.compute(n_log, w);
+                        ++cases;
+                    }
+                }
+    std::printf("%d cases, %d failures\n", cases, failures);
+    return failures ? 1 : 0;
+}
