@@ -112,9 +112,10 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) 
 
 template <class IT, int KIND, bool WITH_CUR, int NWG>
 __global__ void __launch_bounds__(threads_for(NWG), 1)
-merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict__ log_k, const IT *__restrict__ log_v,
-                const IT *__restrict__ log_b, const IT *__restrict__ log_a, const float *__restrict__ log_x, int L,
-                int n_log, const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
+merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_st,
+                const IT *__restrict__ log_k, const IT *__restrict__ log_v, const IT *__restrict__ log_b,
+                const IT *__restrict__ log_a, const float *__restrict__ log_x, int L, int n_log,
+                const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                 const IT *__restrict__ beta, const IT *__restrict__ a, float *__restrict__ o, int DV,
                 long long units) {
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
@@ -126,10 +127,12 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
     volatile int *abort = reinterpret_cast<volatile int *>(sm + LY.off_abort());
     auto B_FULL = [&](int s) { return &bars[s]; };
     auto B_FREE = [&](int s) { return &bars[NS + s]; };
-    auto B_LO = [&](int w) { return &bars[2 * NS + 4 * w + 0]; };
-    auto B_G = [&](int w) { return &bars[2 * NS + 4 * w + 1]; };
-    auto B_DELTA = [&](int w) { return &bars[2 * NS + 4 * w + 2]; };
-    auto B_D = [&](int w) { return &bars[2 * NS + 4 * w + 3]; };
+    auto B_KH = [&](int w) { return &bars[2 * NS + 6 * w + 0]; };
+    auto B_LO = [&](int w) { return &bars[2 * NS + 6 * w + 1]; };      // completes twice per unit
+    auto B_LOFREE = [&](int w) { return &bars[2 * NS + 6 * w + 2]; };
+    auto B_G = [&](int w) { return &bars[2 * NS + 6 * w + 3]; };
+    auto B_DELTA = [&](int w) { return &bars[2 * NS + 6 * w + 4]; };
+    auto B_D = [&](int w) { return &bars[2 * NS + 6 * w + 5]; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tiles = DV / ROWS;
@@ -138,15 +141,11 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
-            tc::mbar_init(B_FULL(s), 1 + 32);  // TMA bytes + the loader lanes' cp.async arrivals
+            tc::mbar_init(B_FULL(s), 1 + 32);  // the loader's byte count + its lanes' cp.async arrivals
             tc::mbar_init(B_FREE(s), 1);
         }
-        for (int w = 0; w < NWG; ++w) {
-            tc::mbar_init(B_LO(w), 1);
-            tc::mbar_init(B_G(w), 1);
-            tc::mbar_init(B_DELTA(w), 1);
-            tc::mbar_init(B_D(w), 1);
-        }
+        for (int w = 0; w < NWG; ++w)
+            for (int b = 0; b < 6; ++b) tc::mbar_init(&bars[2 * NS + 6 * w + b], 1);
         *abort = 0;
         tc::mbar_init_fence();
     }
@@ -160,7 +159,12 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
 
     if (warp == 0) {
         // ------------------------------------------------ loads
-        if (lane == 0) tc::tma_prefetch_desc(&map_s);
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&map_s);
+            tc::tma_prefetch_desc(&map_st);
+        }
+        constexpr uint32_t KB = DK * sizeof(IT), VB = ROWS * sizeof(IT);  // one entry's key / value-tile bytes
+        const uint32_t tx = (uint32_t)LY.tile() + (uint32_t)nb * (KB * (CHAN ? 2 : 1) + VB) + (WITH_CUR ? KB : 0);
         for (int i = 0; i < n_mine; ++i) {
             const int s = i % NS;
             if (i >= NS && !wait_bar(B_FREE(s), (uint32_t)((i / NS - 1) & 1), abort)) break;
@@ -168,32 +172,28 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
             const Unit un = unit_of((long long)blockIdx.x + (long long)i * gridDim.x, tiles);
             const long long lrow = un.head * L;
             uint64_t *full = B_FULL(s);
-            if (lane == 0) {
-                tc::mbar_arrive_expect_tx(full, (uint32_t)LY.tile());
-                for (int ch = 0; ch < NCHUNK; ++ch)
-                    tc::tma_load_2d(st + LY.off_tile() + ch * (ROWS * 128), &map_s, ch * CHUNK,
-                                    (int)(un.head * DV + un.row0), full);
-            }
-            // raw entries 0..nb-1: logged ones from the log, the fused read's own from the inputs
-            constexpr int E = 16 / (int)sizeof(IT);  // elements per 16-byte chunk
-            constexpr int KC = DK / E, VC = ROWS / E;
+            // the state tile by TMA; the raw entries by bulk copies spread over
+            // the lanes: logged ones from the log (contiguous per head), the
+            // fused read's own from this step's inputs
+            if (lane == 0) tc::mbar_arrive_expect_tx(full, tx);
+            __syncwarp();
             uint8_t *rk = st + LY.off_raw_k(), *ra = st + LY.off_raw_a(), *rv = st + LY.off_raw_v();
-            for (int u = lane; u < nb * KC; u += 32) {
-                const int e = u / KC, col = (u % KC) * E;
-                const IT *srck = e < n_log ? log_k + (lrow + e) * DK : k + un.head * DK;
-                cp_async16(rk + raw_k_off(e, col, sizeof(IT)), srck + col);
-                if constexpr (CHAN) {
-                    const IT *srca = e < n_log ? log_a + (lrow + e) * DK : a + un.head * DK;
-                    cp_async16(ra + raw_k_off(e, col, sizeof(IT)), srca + col);
-                }
+            if (lane < NCHUNK)
+                tc::tma_load_2d(st + LY.off_tile() + lane * (ROWS * 128), &map_s, lane * CHUNK,
+                                (int)(un.head * DV + un.row0), full);
+            if (lane == NCHUNK && n_log > 0) tc::bulk_load(rk, log_k + lrow * DK, (uint32_t)n_log * KB, full);
+            if (CHAN && lane == NCHUNK + 1 && n_log > 0)
+                tc::bulk_load(ra, log_a + lrow * DK, (uint32_t)n_log * KB, full);
+            if (WITH_CUR && lane == NCHUNK + 2) {
+                tc::bulk_load(rk + raw_k_off(n_log, 0, sizeof(IT)), k + un.head * DK, KB, full);
+                if constexpr (CHAN) tc::bulk_load(ra + raw_k_off(n_log, 0, sizeof(IT)), a + un.head * DK, KB, full);
+                tc::bulk_load(st + LY.off_raw_q(), q + un.head * DK, KB, full);
             }
-            for (int u = lane; u < nb * VC; u += 32) {
-                const int e = u / VC, col = (u % VC) * E;
-                const IT *srcv = e < n_log ? log_v + (lrow + e) * DV : v + un.head * DV;
-                cp_async16(rv + raw_v_off(e, col, sizeof(IT)), srcv + un.row0 + col);
+            if (lane >= 16 && lane - 16 < nb) {  // value tiles: lane 16 + e copies entry e's
+                const int e = lane - 16;
+                const IT *src = e < n_log ? log_v + (lrow + e) * DV + un.row0 : v + un.head * DV + un.row0;
+                tc::bulk_load(rv + raw_v_off(e, 0, sizeof(IT)), src, VB, full);
             }
-            if (WITH_CUR && lane < KC)
-                cp_async16(st + LY.off_raw_q() + raw_q_off(lane * E, sizeof(IT)), q + un.head * DK + lane * E);
             if constexpr (DELTA) {  // the X block: X(j, e), e <= j < n_log
                 uint8_t *sc = st + LY.off_sc();
                 for (int u = lane; u < NB * NB; u += 32) {
@@ -216,7 +216,9 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                 const int s = i % NS;
                 const uint32_t par = (uint32_t)(j & 1);
                 if constexpr (DELTA) {
-                    if (!wait_bar(B_LO(w), par, abort)) break;
+                    // G: the tile part as soon as Khat is in place, then the S_lo
+                    // part in two halves of the key columns as the group writes them
+                    if (!wait_bar(B_KH(w), par, abort)) break;
                     tc::tc_fence_after();
                     const uint32_t tile = tc::smem_u32(sm + LY.stage(s) + LY.off_tile());
 #pragma unroll
@@ -225,19 +227,30 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                         const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
                         tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
                     }
+                    bool ok = true;
 #pragma unroll
-                    for (int kk = 0; kk < DK / 8; ++kk) {
-                        const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
-                        tc::mma_ts_tf32(tw + COL_G, tw + COL_B + 8 * kk, bd, ID_G, true);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (!wait_bar(B_LO(w), (uint32_t)h, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+#pragma unroll
+                        for (int kq = 0; kq < DK / 16; ++kq) {
+                            const int kk = h * (DK / 16) + kq;
+                            const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                            tc::mma_ts_tf32(tw + COL_G, tw + COL_LO + 8 * kq, bd, ID_G, true);
+                        }
+                        tc::mma_commit(h == 0 ? B_LOFREE(w) : B_G(w));
                     }
-                    tc::mma_commit(B_G(w));
+                    if (!ok) break;
                 }
                 if (!wait_bar(B_DELTA(w), par, abort)) break;
                 tc::tc_fence_after();
 #pragma unroll
-                for (int m = 0; m < 6; ++m) {  // region B holds S o gamma: accumulate onto it
+                for (int m = 0; m < 6; ++m) {  // onto S o gamma
                     const uint64_t bd = tc::smem_desc(kf + wb_b_start(m), 16, 1024, tc::SWZ_128);
-                    tc::mma_ts_tf32(tw + COL_B, tw + COL_DL + wb_a_col(m), bd, ID_W, true);
+                    tc::mma_ts_tf32(tw + COL_SG, tw + COL_DL + wb_a_col(m), bd, ID_W, true);
                 }
                 tc::mma_commit(B_D(w));
             }
@@ -257,7 +270,6 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
         float *cn = reinterpret_cast<float *>(gp + LY.g_cn());
         float *red = reinterpret_cast<float *>(gp + LY.g_red());
         uint8_t *kf = gp + LY.g_kf();
-        uint8_t *out = gp + LY.g_out();
         const int bar_id = 1 + w;
         for (int j = 0, i = w; i < n_mine; ++j, i += NWG) {
             const int s = i % NS;
@@ -283,6 +295,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
             }
             const float bcur = (DELTA && WITH_CUR) ? ld_in(beta + un.head) : 0.f;
             if (!wait_bar(B_FULL(s), (uint32_t)((i / NS) & 1), abort)) break;
+            if (j > 0) tc::named_sync(bar_id, 128);  // every warp's last stores have read the operand tile
 
             // 1. key side for channel c: Khat (hi and lo parts), F, gamma, q
             float kc[NB], ac[NB];
@@ -315,43 +328,88 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                     f *= ac[e];
                 }
             }
-            // 2. S_lo = S - hi(S) into region B (row r); then G may start
-            if constexpr (DELTA) {
+            if constexpr (DELTA) tc::fence_async_smem();  // Khat is read by the tensor cores
+            tc::named_sync(bar_id, 128);                   // Khat, gamma and q of every channel are in place
+            if (DELTA && ct == 0) tc::mbar_arrive(B_KH(w));
+
+            // 2. one pass over the tile row: S o gamma into [COL_SG, +128), and
+            //    S_lo = S - hi(S) into [COL_LO, +64) one half of the columns at a
+            //    time (the second half once G has read the first); for the fused
+            //    read also (S o gamma) . q
+            float oacc = 0.f;
+            auto row_chunk = [&](int ch, uint32_t (&lo)[32]) {
+                uint32_t y[32];
 #pragma unroll
-                for (int ch = 0; ch < NCHUNK; ++ch) {
-                    uint32_t lo[32];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, ch * CHUNK + 4 * u));
+                for (int u = 0; u < 8; ++u) {
+                    const int col = ch * CHUNK + 4 * u;
+                    const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, col));
+                    const float4 gv = *reinterpret_cast<const float4 *>(gam + col);
+                    const float4 sg = make_float4(x.x * gv.x, x.y * gv.y, x.z * gv.z, x.w * gv.w);
+                    y[4 * u + 0] = __float_as_uint(sg.x);
+                    y[4 * u + 1] = __float_as_uint(sg.y);
+                    y[4 * u + 2] = __float_as_uint(sg.z);
+                    y[4 * u + 3] = __float_as_uint(sg.w);
+                    if constexpr (DELTA) {
                         lo[4 * u + 0] = __float_as_uint(x.x - tc::tf32_trunc(x.x));
                         lo[4 * u + 1] = __float_as_uint(x.y - tc::tf32_trunc(x.y));
                         lo[4 * u + 2] = __float_as_uint(x.z - tc::tf32_trunc(x.z));
                         lo[4 * u + 3] = __float_as_uint(x.w - tc::tf32_trunc(x.w));
                     }
-                    tc::tmem_st32(trow + COL_B + ch * CHUNK, lo);
+                    if constexpr (WITH_CUR) {
+                        const float4 qv = *reinterpret_cast<const float4 *>(qf + col);
+                        oacc = fmaf(sg.x, qv.x, fmaf(sg.y, qv.y, fmaf(sg.z, qv.z, fmaf(sg.w, qv.w, oacc))));
+                    }
                 }
-                tc::tmem_wait_st();
-                tc::fence_async_smem();  // Khat is read by the tensor cores
-                tc::tc_fence_before();
-                tc::named_sync(bar_id, 128);
-                if (ct == 0) tc::mbar_arrive(B_LO(w));
-            } else {
-                tc::named_sync(bar_id, 128);  // gamma and q of every channel are in place
+                tc::tmem_st32(trow + COL_SG + ch * CHUNK, y);
+            };
+            {
+                uint32_t lo[32];
+                row_chunk(0, lo);
+                if constexpr (DELTA) tc::tmem_st32(trow + COL_LO, lo);
+                row_chunk(1, lo);
+                if constexpr (DELTA) {
+                    tc::tmem_st32(trow + COL_LO + CHUNK, lo);
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
+                    tc::named_sync(bar_id, 128);
+                    if (ct == 0) tc::mbar_arrive(B_LO(w));  // first half
+                }
+                row_chunk(2, lo);
+                if constexpr (DELTA) {
+                    if (!wait_bar(B_LOFREE(w), par, abort)) break;  // G has read the first half
+                    tc::tc_fence_after();
+                    tc::tmem_st32(trow + COL_LO, lo);
+                }
+                row_chunk(3, lo);
+                if constexpr (DELTA) {
+                    tc::tmem_st32(trow + COL_LO + CHUNK, lo);
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
+                    tc::named_sync(bar_id, 128);
+                    if (ct == 0) tc::mbar_arrive(B_LO(w));  // second half
+                }
             }
-            // 3. while G runs: the fused read's entry (index nb - 1) gets its X row
-            //    from C(nb-1, e) = F_{nb-1} . F_e
-            if (DELTA && WITH_CUR) {
+            // 3. while G runs, for the fused read: the sums over key channels that
+            //    its entry's X row and its output need, C(nb-1, e) = F_{nb-1} . F_e
+            //    (every factor after the entry is a padded 1, so F_{nb-1} = k_{nb-1})
+            //    and (F q)_e; then the entry's X row
+            if constexpr (WITH_CUR) {
                 const int nl = nb - 1;
-                const float fn = to_f(rk[raw_k_off(nl, c, 1)]);  // F_{nb-1} = k_{nb-1}: every later factor is a padded 1
-                float p[NB];
+                const float fn = to_f(rk[raw_k_off(nl, c, 1)]);
+                const float qc = qf[c];
+                float p[2 * NB];
 #pragma unroll
-                for (int e = 0; e < NB; ++e) p[e] = e < nl ? fn * fv[e] : 0.f;
-                multi_sum<NB>(p, lane);  // lane l: this warp's sum for entry l >> 1
-                if ((lane & 1) == 0) red[quad * NB + (lane >> 1)] = p[0];
+                for (int e = 0; e < NB; ++e) {
+                    p[e] = (DELTA && e < nl) ? fn * fv[e] : 0.f;
+                    p[NB + e] = fv[e] * qc;
+                }
+                multi_sum<2 * NB>(p, lane);  // lane l: this warp's sum of item l
+                red[quad * 2 * NB + lane] = p[0];
                 tc::named_sync(bar_id, 128);
-                if (ct < NB) cn[ct] = red[ct] + red[NB + ct] + red[2 * NB + ct] + red[3 * NB + ct];
+                if (ct < 2 * NB)
+                    cn[ct] = red[ct] + red[2 * NB + ct] + red[4 * NB + ct] + red[6 * NB + ct];
                 tc::named_sync(bar_id, 128);
-                if (ct <= nl) {
+                if (DELTA && ct <= nl) {
                     // X(nl, ct) = -beta_nl sum_{m = ct..nl-1} C(nl, m) X(m, ct); X(nl, nl) = beta_nl
                     float acc = 0.f;
 #pragma unroll
@@ -359,13 +417,14 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                         if (m >= ct && m < nl) acc = fmaf(cn[m], scf(sc_x(m, ct)), acc);
                     *reinterpret_cast<float *>(sc + sc_x(nl, ct)) = ct == nl ? bcur : -bcur * acc;
                 }
-                tc::named_sync(bar_id, 128);
+                if constexpr (DELTA) tc::named_sync(bar_id, 128);
             }
             float vr[NB];
 #pragma unroll
             for (int e = 0; e < NB; ++e) vr[e] = e < nb ? to_f(rv[raw_v_off(e, r, 1)]) : 0.f;
 
-            // 4. delta = X (V - G) for row r (RWKV6: delta = V) into A[32, 64)
+            // 4. delta = X (V - G) for row r (RWKV6: delta = V) into [COL_DL, +32);
+            //    F over Khat (G has read it)
             float dl[NB];
             if constexpr (DELTA) {
                 if (!wait_bar(B_G(w), par, abort)) break;
@@ -378,9 +437,18 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                 for (int e = 0; e < NB; ++e) ev[e] = vr[e] - (__uint_as_float(gr[e]) + __uint_as_float(gr[NB + e]));
 #pragma unroll
                 for (int e = 0; e < NB; ++e) {
+                    float xr[NB];  // row e of X (entries past the diagonal are not read)
+#pragma unroll
+                    for (int m4 = 0; m4 <= e / 4; ++m4) {
+                        const float4 x4 = *reinterpret_cast<const float4 *>(sc + sc_x(e, 4 * m4));
+                        xr[4 * m4 + 0] = x4.x;
+                        xr[4 * m4 + 1] = x4.y;
+                        xr[4 * m4 + 2] = x4.z;
+                        xr[4 * m4 + 3] = x4.w;
+                    }
                     float acc = 0.f;
 #pragma unroll
-                    for (int m = 0; m <= e; ++m) acc = fmaf(scf(sc_x(e, m)), ev[m], acc);
+                    for (int m = 0; m <= e; ++m) acc = fmaf(xr[m], ev[m], acc);
                     dl[e] = e < nb ? acc : 0.f;
                 }
             } else {
@@ -396,22 +464,6 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                     wd[NB + e] = __float_as_uint(dl[e] - hi);
                 }
                 tc::tmem_st32(trow + COL_DL, wd);
-            }
-            // 5. S o gamma into region B (S_lo there has been read by G), F over Khat
-#pragma unroll
-            for (int ch = 0; ch < NCHUNK; ++ch) {
-                uint32_t y[32];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int col = ch * CHUNK + 4 * u;
-                    const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, col));
-                    const float4 gv = *reinterpret_cast<const float4 *>(gam + col);
-                    y[4 * u + 0] = __float_as_uint(x.x * gv.x);
-                    y[4 * u + 1] = __float_as_uint(x.y * gv.y);
-                    y[4 * u + 2] = __float_as_uint(x.z * gv.z);
-                    y[4 * u + 3] = __float_as_uint(x.w * gv.w);
-                }
-                tc::tmem_st32(trow + COL_B + ch * CHUNK, y);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {  // 16-byte pieces: hi of entries 4u.. (u < 4), lo (u >= 4)
@@ -432,42 +484,44 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const IT *__restrict_
                 tc::mbar_arrive(B_DELTA(w));
                 tc::mbar_arrive(B_FREE(s));  // the unit reads nothing more of its stage
             }
+            if constexpr (WITH_CUR) {  // o = (S o gamma) . q + delta . (F q)
+#pragma unroll
+                for (int e = 0; e < NB; ++e) oacc = fmaf(dl[e], cn[NB + e], oacc);
+                o[un.head * DV + un.row0 + r] = oacc;
+            }
 
-            // 6. S_new = region B after the write-back: o = S_new q for the fused
-            //    read, and the rows to HBM by TMA, one 32-column chunk at a time
-            //    through the group's staging tile
+            // 5. S_new = [COL_SG, +128) after the write-back: each warp's 32 rows
+            //    to HBM by TMA, 32 columns at a time, through two staging tiles
+            //    used in turn (the first is the warp's quarter of the operand
+            //    tile, which the write-back has finished reading)
             if (!wait_bar(B_D(w), par, abort)) break;
             tc::tc_fence_after();
-            float oacc = 0.f;
 #pragma unroll 1
             for (int ch = 0; ch < NCHUNK; ++ch) {
                 uint32_t d[32];
-                tc::tmem_ld32(trow + COL_B + ch * CHUNK, d);
-                if (ct == 0) tc::bulk_wait_read<0>();  // the staging tile's previous store has read it
+                tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
+                uint8_t *buf = sm + LY.group(w) + LY.out_buf(quad, ch & 1);
+                if (ch >= 2 && lane == 0) tc::bulk_wait_read<1>();  // the store that last used this tile has read it
+                __syncwarp();
                 tc::tmem_wait_ld();
-                tc::named_sync(bar_id, 128);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int col = ch * CHUNK + 4 * u;
-                    const float4 y = make_float4(__uint_as_float(d[4 * u + 0]), __uint_as_float(d[4 * u + 1]),
-                                                 __uint_as_float(d[4 * u + 2]), __uint_as_float(d[4 * u + 3]));
-                    *reinterpret_cast<float4 *>(out + tile_off(r, 4 * u)) = y;
-                    if constexpr (WITH_CUR) {
-                        const float4 qv = *reinterpret_cast<const float4 *>(qf + col);
-                        oacc = fmaf(y.x, qv.x, fmaf(y.y, qv.y, fmaf(y.z, qv.z, fmaf(y.w, qv.w, oacc))));
-                    }
-                }
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<uint4 *>(buf + tile_off(lane, 4 * u)) =
+                        make_uint4(d[4 * u + 0], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
                 tc::fence_async_smem();  // the staging tile is read by the TMA store
-                tc::named_sync(bar_id, 128);
-                if (ct == 0) {
-                    tc::tma_store_2d(&map_s, ch * CHUNK, (int)(un.head * DV + un.row0), out);
+                __syncwarp();
+                if (lane == 0) {
+                    tc::tma_store_2d(&map_st, ch * CHUNK, (int)(un.head * DV + un.row0 + 32 * quad), buf);
                     tc::bulk_commit();
                 }
             }
-            if constexpr (WITH_CUR) o[un.head * DV + un.row0 + r] = oacc;
-            tc::tc_fence_before();  // region B is rewritten by the group's next unit
+            // the operand tile is rewritten by the next unit's key side: this
+            // warp's stores from it (and from its other staging tile) have read them
+            if (lane == 0) tc::bulk_wait_read<0>();
+            __syncwarp();
+            tc::tc_fence_before();  // [COL_SG, +128) is rewritten by the group's next unit
         }
-        if (ct == 0) tc::bulk_wait_all();  // the group's last stores have landed
+        if (lane == 0) tc::bulk_wait_all();  // the warp's last stores have landed
     }
     // drain: every role has left its loop; products in flight have completed
     // (the compute warps waited for the last one, or the CTA gave up)
@@ -498,17 +552,20 @@ EncodeTiledFn encoder() {
     return fn;
 }
 
-// The fp32 state [rows, 128] as a tensor map of 32-column x 128-row boxes,
-// 128-byte swizzle.
-cudaError_t state_map(CUtensorMap *m, void *S, unsigned long long rows) {
+// The fp32 state [rows, 128] as a tensor map of box_cols x box_rows boxes
+// (box_cols x 4 bytes = the swizzle span: 32 columns with 128-byte swizzle,
+// 16 with 64-byte).
+cudaError_t state_map(CUtensorMap *m, void *S, unsigned long long rows, unsigned box_cols, unsigned box_rows) {
     EncodeTiledFn fn = encoder();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {(cuuint64_t)DK, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)DK * 4};
-    const cuuint32_t box[2] = {(cuuint32_t)CHUNK, (cuuint32_t)ROWS};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     const cuuint32_t es[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, S, dims, strides, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -526,13 +583,14 @@ cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cud
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const long long heads = (long long)p.B * p.H;
-    CUtensorMap map;
-    e = state_map(&map, p.S, (unsigned long long)heads * p.dv);
+    CUtensorMap map, map_st;  // loads: 32 x 128 boxes; each warp's stores: 32 x 32 boxes
+    e = state_map(&map, p.S, (unsigned long long)heads * p.dv, CHUNK, ROWS);
+    if (e == cudaSuccess) e = state_map(&map_st, p.S, (unsigned long long)heads * p.dv, CHUNK, 32);
     if (e != cudaSuccess) return e;
     const long long units = heads * (p.dv / ROWS);
     const unsigned grid = (unsigned)std::min<long long>(units, sms);
     kern<<<grid, threads_for(NWG), LY.request(), st>>>(
-        map, static_cast<const IT *>(lg.k), static_cast<const IT *>(lg.v), static_cast<const IT *>(lg.beta),
+        map, map_st, static_cast<const IT *>(lg.k), static_cast<const IT *>(lg.v), static_cast<const IT *>(lg.beta),
         static_cast<const IT *>(lg.a), lg.x, lg.L, n_log, static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
         static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), p.o, p.dv,
         units);

@@ -35,14 +35,17 @@ constexpr int CHUNK = 32;     // fp32 columns per 128-byte swizzle row
 constexpr int NCHUNK = DK / CHUNK;
 constexpr int CTRL_WARPS = 4; // warp 0 loads, warps 1 and 2 issue products (group 0, 1), warp 3 idle
 constexpr uint32_t TMEM_COLS_PER_GROUP = 256;
-// A group's tensor memory: region A = columns [0, 128), region B = [128, 256).
-//   B  <- S_lo (the low part of the state tile: the A operand of G's second half)
-//   A[0, 32)  <- G = S Khat^T (hi half of Khat, then lo half)
-//   A[32, 64) <- delta hi (16 columns) | delta lo (16 columns)
-//   B  <- S o gamma, once G is read; then += delta F (the write-back) = S_new
-constexpr int COL_G = 0;
-constexpr int COL_DL = 32;
-constexpr int COL_B = 128;
+// A group's tensor memory (columns from the group's base):
+//   [0, 128)   S o gamma, written while the tile is read for S_lo; the
+//              write-back accumulates delta F onto it, giving S_new
+//   [128, 192) S_lo for one half of the key columns at a time (the A operand
+//              of G's second half, two rounds of 8 K-steps)
+//   [192, 224) G = S Khat^T (hi half of Khat, then lo half)
+//   [224, 256) delta hi (16 columns) | delta lo (16 columns)
+constexpr int COL_SG = 0;
+constexpr int COL_LO = 128;
+constexpr int COL_G = 192;
+constexpr int COL_DL = 224;
 constexpr size_t SMEM_LIMIT = 232448;  // dynamic shared memory a block may request (227 KiB)
 
 DL_HD constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -80,21 +83,29 @@ struct Layout {
     // K-major, 128-byte swizzle).
     DL_HD constexpr size_t g_kf() const { return 0; }
     DL_HD constexpr size_t kf_bytes() const { return (size_t)2 * NB * DK * 4; }
-    // the staging tile of the result's TMA store: one 32-column chunk
-    // [128 rows x 128 B], 128-byte swizzle
+    // the staging tiles of the result's TMA stores, two per warp of the group
+    // (used in turn): warp quad q (rows 32q..32q+31) stages one 32-column
+    // chunk of its rows, [32 rows x 128 B] with 128-byte swizzle. Tile 0 is
+    // the warp's quarter of the operand tile (free once the write-back has
+    // read F), tile 1 its quarter of this region.
     DL_HD constexpr size_t g_out() const { return g_kf() + kf_bytes(); }
     DL_HD constexpr size_t out_bytes() const { return (size_t)ROWS * 128; }
+    DL_HD constexpr size_t out_buf(int quad, int b) const {
+        return (b == 0 ? g_kf() : g_out()) + (size_t)quad * 32 * 128;
+    }
     DL_HD constexpr size_t g_gam() const { return g_out() + out_bytes(); }  // gamma [128] floats
     DL_HD constexpr size_t g_qf() const { return g_gam() + DK * 4; }        // q widened [128] floats
-    DL_HD constexpr size_t g_cn() const { return g_qf() + DK * 4; }         // C row of the step's entry [16]
-    DL_HD constexpr size_t g_red() const { return g_cn() + NB * 4; }        // [4 warps][16] partial sums
-    DL_HD constexpr size_t group_bytes() const { return round_up(g_red() + 4 * NB * 4, 1024); }
+    // the fused read's sums over key channels: C(n, e) (16) then (F q)_e (16)
+    DL_HD constexpr size_t g_cn() const { return g_qf() + DK * 4; }
+    DL_HD constexpr size_t g_red() const { return g_cn() + 2 * NB * 4; }    // [4 warps][32] partial sums
+    DL_HD constexpr size_t group_bytes() const { return round_up(g_red() + 4 * 2 * NB * 4, 1024); }
     DL_HD constexpr size_t group(int w) const { return stage(NS) + (size_t)w * group_bytes(); }
 
     // ---- barriers and words
     DL_HD constexpr size_t off_bar() const { return group(nwg); }
-    // full[NS], free[NS], then per group: lo_ready, g_done, delta_ready, d_done
-    DL_HD constexpr int nbar() const { return 2 * NS + 4 * nwg; }
+    // full[NS], free[NS], then per group: kh_ready, lo_ready (twice per unit),
+    // lo_free, g_done, delta_ready, d_done
+    DL_HD constexpr int nbar() const { return 2 * NS + 6 * nwg; }
     DL_HD constexpr size_t off_tslot() const { return off_bar() + (size_t)nbar() * 8; }
     DL_HD constexpr size_t off_abort() const { return off_tslot() + 4; }
     DL_HD constexpr size_t end() const { return off_abort() + 4; }
@@ -137,7 +148,6 @@ DL_HD constexpr uint32_t kh_off(int n, int c) {
 }
 // F element (channel c, column j in 0..31) inside the operand tile.
 DL_HD constexpr uint32_t ff_off(int c, int j) { return swz128((uint32_t)(c * 128 + j * 4)); }
-
 // Groups the launch can afford: two when their operand tiles fit beside the
 // two stages, else one.
 DL_HD constexpr int groups_for(size_t in_size, bool chan) {

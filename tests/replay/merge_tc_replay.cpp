@@ -63,8 +63,8 @@ struct Replay {
             add(p + "out", ly.group(w) + ly.g_out(), ly.out_bytes());
             add(p + "gam", ly.group(w) + ly.g_gam(), DK * 4);
             add(p + "qf", ly.group(w) + ly.g_qf(), DK * 4);
-            add(p + "cn", ly.group(w) + ly.g_cn(), NB * 4);
-            add(p + "red", ly.group(w) + ly.g_red(), 4 * NB * 4);
+            add(p + "cn", ly.group(w) + ly.g_cn(), 2 * NB * 4);        // C(n, e) then (F q)_e
+            add(p + "red", ly.group(w) + ly.g_red(), 4 * 2 * NB * 4);  // [4 warps][32]
         }
         add("bar", ly.off_bar(), (size_t)ly.nbar() * 8);
         add("tslot", ly.off_tslot(), 4);
@@ -121,24 +121,40 @@ struct Replay {
                 if ((ly.stage(s) + ly.off_tile() + ch * ROWS * 128) % 1024) fail("TMA box not 1024-aligned", tag());
     }
 
-    // warp 0: TMA boxes, cp.async of the raw entries, scalars and the X block
+    // warp 0: TMA boxes and bulk copies of the raw entries (lane 0), cp.async of the X block
     void producer(int n_log, int L) {
         const int nb = n_log + (with_cur ? 1 : 0);
-        const int E = 16 / (int)in_size, KC = DK / E, VC = ROWS / E;
+        const size_t KB = DK * in_size, VB = ROWS * in_size;
         for (int s = 0; s < NS; ++s) {
             const std::string p = "stage" + std::to_string(s) + ".";
-            for (int ch = 0; ch < NCHUNK; ++ch) acc(p + "tile", ch * ROWS * 128, ROWS * 128, 1024, "TMA box");
-            for (int lane = 0; lane < 32; ++lane) {
-                for (int u = lane; u < nb * KC; u += 32) {
-                    const int e = u / KC, col = (u % KC) * E;
-                    acc(p + "raw_k", raw_k_off(e, col, in_size), 16, 16, "cp.async k");
-                    if (chan) acc(p + "raw_a", raw_k_off(e, col, in_size), 16, 16, "cp.async a");
-                }
-                for (int u = lane; u < nb * VC; u += 32) {
-                    const int e = u / VC, col = (u % VC) * E;
-                    acc(p + "raw_v", raw_v_off(e, col, in_size), 16, 16, "cp.async v");
-                }
-                if (with_cur && lane < KC) acc(p + "raw_q", raw_q_off(lane * E, in_size), 16, 16, "cp.async q");
+            size_t tx = 0;
+            for (int ch = 0; ch < NCHUNK; ++ch) {
+                acc(p + "tile", ch * ROWS * 128, ROWS * 128, 1024, "TMA box");
+                tx += ROWS * 128;
+            }
+            // (lanes 16 + e copy entry e's value tile: every entry has a lane)
+            if (nb > 16) fail("more entries than value-copy lanes", tag());
+            auto bulk = [&](const std::string &reg, size_t off, size_t bytes, const char *what) {
+                if (bytes % 16) fail("bulk copy size not a multiple of 16", tag() + " " + what);
+                acc(reg, off, bytes, 16, what);
+                tx += bytes;
+            };
+            if (n_log > 0) {
+                bulk(p + "raw_k", raw_k_off(0, 0, in_size), n_log * KB, "log keys");
+                if (chan) bulk(p + "raw_a", raw_k_off(0, 0, in_size), n_log * KB, "log decays");
+            }
+            for (int e = 0; e < n_log; ++e) bulk(p + "raw_v", raw_v_off(e, 0, in_size), VB, "log values");
+            if (with_cur) {
+                bulk(p + "raw_k", raw_k_off(n_log, 0, in_size), KB, "step key");
+                if (chan) bulk(p + "raw_a", raw_k_off(n_log, 0, in_size), KB, "step decays");
+                bulk(p + "raw_v", raw_v_off(n_log, 0, in_size), VB, "step values");
+                bulk(p + "raw_q", raw_q_off(0, in_size), KB, "step query");
+            }
+            // the byte count the loader expects (merge_tc.cu: tx)
+            const size_t expect = ly.tile() + (size_t)nb * (KB * (chan ? 2 : 1) + VB) + (with_cur ? KB : 0);
+            if (tx != expect) fail("expected bytes differ from the bytes copied", tag());
+            if (tx >= (1u << 20)) fail("transaction count beyond the mbarrier's range", tag());
+            for (int lane = 0; lane < 32; ++lane)
                 if (delta)
                     for (int u = lane; u < NB * NB; u += 32) {
                         const int j = u / NB, e = u % NB;
@@ -148,7 +164,6 @@ struct Replay {
                             if (j >= L || e >= L) fail("X read outside the head's block", tag());
                         }
                     }
-            }
         }
     }
 
@@ -174,7 +189,7 @@ struct Replay {
                     acc(gp + "kf", kh_off(NB + j, c), 4, 4, "Khat lo");
                     khs.insert(kh_off(j, c));
                     khs.insert(kh_off(NB + j, c));
-                    for (int m = 0; m <= j; ++m) acc(p + "sc", sc_x(j, m), 4, 4, "X read");
+                    for (int m4 = 0; m4 <= j / 4; ++m4) acc(p + "sc", sc_x(j, 4 * m4), 16, 16, "X row piece");
                 }
             }
             acc(gp + "gam", c * 4, 4, 4, "gamma");
@@ -189,28 +204,35 @@ struct Replay {
                     ffs.insert(ff_off(c, 4 * u + e));
                 }
             }
-            if (delta && with_cur) {
+            if (with_cur) {  // the fused read's sums over key channels and its entry's X row
                 const int nl = nb - 1;
                 acc(p + "raw_k", raw_k_off(nl, c, in_size), in_size, in_size, "fused key");
-                if ((lane & 1) == 0) acc(gp + "red", (quad * NB + (lane >> 1)) * 4, 4, 4, "red write");
-                if (ct < NB) {
-                    for (int w = 0; w < 4; ++w) acc(gp + "red", (w * NB + ct) * 4, 4, 4, "red read");
+                acc(p + "raw_q", raw_q_off(c, in_size), in_size, in_size, "fused q");
+                acc(gp + "red", (quad * 2 * NB + lane) * 4, 4, 4, "red write");
+                if (ct < 2 * NB) {
+                    for (int q4 = 0; q4 < 4; ++q4) acc(gp + "red", (q4 * 2 * NB + ct) * 4, 4, 4, "red read");
                     acc(gp + "cn", ct * 4, 4, 4, "cn write");
                 }
-                if (ct <= nl) {
+                if (delta && ct <= nl) {
                     for (int m = ct; m < nl; ++m) {
                         acc(gp + "cn", m * 4, 4, 4, "cn read");
                         acc(p + "sc", sc_x(m, ct), 4, 4, "X read (fused row)");
                     }
                     acc(p + "sc", sc_x(nl, ct), 4, 4, "fused X row write");
                 }
+                for (int e = 0; e < NB; ++e) acc(gp + "cn", (NB + e) * 4, 4, 4, "F q read");
             }
             for (int col = 0; col < DK; col += 4) {
                 acc(p + "tile", tile_off(r, col), 16, 16, "tile piece");
-                if (col < CHUNK) {
-                    acc(gp + "out", tile_off(r, col), 16, 16, "staging piece");
-                    if (tile_off(r, col) >= ly.out_bytes()) fail("staging piece outside the chunk", tag());
-                }
+                if (col < CHUNK)  // the warp's two staging tiles: its 32 rows of one 32-column chunk
+                    for (int b = 0; b < 2; ++b) {
+                        const char *reg = b == 0 ? "kf" : "out";
+                        const size_t base = b == 0 ? ly.g_kf() : ly.g_out();
+                        const size_t o = ly.out_buf(quad, b) - base + tile_off(lane, col);
+                        acc(gp + reg, o, 16, 16, "staging piece");
+                        if (tile_off(lane, col) >= 32 * 128) fail("staging piece outside its tile", tag());
+                        if ((ly.group(w) + ly.out_buf(quad, b)) % 1024) fail("staging tile not 1024-aligned", tag());
+                    }
                 acc(gp + "gam", col * 4, 16, 16, "gamma piece");
                 if (with_cur) acc(gp + "qf", col * 4, 16, 16, "q piece");
                 for (int e = 0; e < 4; ++e) {
@@ -219,9 +241,13 @@ struct Replay {
                     (void)e;
                 }
             }
-            // tensor memory: region B (S_lo, then S o gamma and the write-back), 4 chunks
+            // tensor memory: S o gamma chunks, the two S_lo halves, G, delta, the write-back's 16-column reads
             for (int ch = 0; ch < NCHUNK; ++ch)
-                if (COL_B + ch * CHUNK + 32 > (int)TMEM_COLS_PER_GROUP) fail("region B columns out of range", tag());
+                if (COL_SG + ch * CHUNK + 32 > COL_LO) fail("S o gamma columns run into S_lo", tag());
+            for (int h = 0; h < 2; ++h)
+                if (COL_LO + h * CHUNK + 32 > COL_G) fail("S_lo columns run into G", tag());
+            for (int c16 = 0; c16 < DK / 16; ++c16)
+                if (COL_SG + 16 * c16 + 16 > COL_LO) fail("write-back read past S_new", tag());
         }
         if (delta && khs.size() != (size_t)2 * NB * DK) fail("Khat layout not one-to-one", tag());
         if (ffs.size() != (size_t)DK * 2 * NB) fail("F layout not one-to-one", tag());
@@ -269,11 +295,12 @@ struct Replay {
             if ((b_lo ? NB : 0) + entry0 != jbase) fail("write-back pairs the wrong F half", tag());
             if (acol + 8 > (int)TMEM_COLS_PER_GROUP) fail("tensor-memory column out of range", tag());
         }
-        // G's second product: A = S_lo in region B, columns COL_B + 8kk
-        for (int kk = 0; kk < DK / 8; ++kk)
-            if (COL_B + 8 * kk + 8 > (int)TMEM_COLS_PER_GROUP) fail("S_lo A columns out of range", tag());
-        // region A: G [COL_G, +32) and delta [COL_DL, +32) apart and below region B
-        if (COL_G + 2 * NB > COL_DL || COL_DL + 2 * NB > COL_B || COL_B + DK > (int)TMEM_COLS_PER_GROUP)
+        // G's second product: A = S_lo, columns COL_LO + 8 kq for the 8 K-steps of each half
+        for (int kq = 0; kq < DK / 16; ++kq)
+            if (COL_LO + 8 * kq + 8 > COL_G) fail("S_lo A columns out of range", tag());
+        // S o gamma [0, 128) | S_lo [128, 192) | G [192, 224) | delta [224, 256)
+        if (COL_SG + DK > COL_LO || COL_LO + DK / 2 > COL_G || COL_G + 2 * NB > COL_DL ||
+            COL_DL + 2 * NB > (int)TMEM_COLS_PER_GROUP)
             fail("tensor-memory regions overlap or overflow", tag());
     }
 };
