@@ -325,6 +325,10 @@ def config_block(w, L, args):
                          "unfused": "DeltaLog deferred, separate merge every L steps",
                          "pool": "slot pool, staggered log fills (each step 1/L of the rows merge)"}[args.schedule],
             "global_batch": w.B * max(1, dist_env()[2]), "seq_len": w.T,
+            "timing": ("launches issued directly, CUDA events around the decode"
+                       if getattr(args, "no_graph", False) or getattr(args, "impl", "ours") == "reference"
+                       else "one decode captured as a CUDA graph, replayed once per step between CUDA events; "
+                            "per-kernel split from one more decode with events around each launch"),
             "l2": "inputs larger than L2 (state %d MiB per GPU), no flush" % (w.state_bytes() >> 20)}
 
 
@@ -423,8 +427,16 @@ class Launcher:
         return e
 
 
-def timed(launcher, steps, warmup):
-    """Returns (ms per step (max over ranks), per-kind {durations}, launches)."""
+def timed(launcher, steps, warmup, use_graph=True):
+    """Returns (ms per step (max over ranks), per-kind {durations}, launches).
+
+    The step time: with ``use_graph`` one decode (all T steps' launches) is
+    captured once in a CUDA graph after the warm-up and replayed ``steps``
+    times between CUDA events, so that host launch overhead does not enter
+    (a serving loop replays its decode graph the same way); otherwise the
+    launches are issued directly. The per-kind split always comes from one
+    more decode issued directly with events around every launch (for short
+    kernels those times include launch gaps: an upper bound)."""
     import torch
     import torch.distributed as dist
 
@@ -435,19 +447,54 @@ def timed(launcher, steps, warmup):
         dist.barrier()
     torch.cuda.synchronize()
     plan = launcher.plan()
-    all_events = []
-    for _ in range(steps):
+    graph = None
+    if use_graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        home = launcher.stream
+        launcher.stream = side
+        try:
+            with torch.cuda.graph(graph, stream=side):
+                launcher.run()
+        finally:
+            launcher.stream = home
+        torch.cuda.synchronize()
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if dist.is_initialized():
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(launcher.stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(launcher.stream)
+        torch.cuda.synchronize()
+        if dist.is_initialized():
+            dist.barrier()
+        total_ms = e0.elapsed_time(e1)
         ev = []
-        launcher.run(ev)
-        all_events.append(ev)
-    torch.cuda.synchronize()
-    if dist.is_initialized():
-        dist.barrier()
-    total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in all_events)
+        launcher.run(ev)  # the per-kind split
+        torch.cuda.synchronize()
+        all_events = [ev]
+    else:
+        all_events = []
+        for _ in range(steps):
+            ev = []
+            launcher.run(ev)
+            all_events.append(ev)
+        torch.cuda.synchronize()
+        if dist.is_initialized():
+            dist.barrier()
+        total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in all_events)
     per_kind = {}
     for ev in all_events:
         for i, (kind, n) in enumerate(plan):
             per_kind.setdefault(kind, []).append((n, ev[i].elapsed_time(ev[i + 1])))
+    del graph
     ms = reduce_max(total_ms / steps)
     return ms, per_kind, steps * sum(KERNELS_PER_CALL[kind] for kind, _ in plan)
 
@@ -598,7 +645,7 @@ def run_sweep(args, w, Ls):
     S_e = d["S0"].clone()
     lau_e = Launcher(g, w, d, S_e, None, o_all, "eager", stream)
     with ClockSampler(0) as smp:
-        ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup)
+        ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup, not args.no_graph)
     del S_e
     eager_bpt = decode_bytes(w, lau_e.plan()) / tokens
     eager_val = tokens / (ms_e / 1000.0)
@@ -611,8 +658,8 @@ def run_sweep(args, w, Ls):
         log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, d["q"].dtype, chan, rwkv6=rw)
         lau = Launcher(g, w, d, S, log, o_all, "fused", stream)
         with ClockSampler(0) as smp:
-            ms, kinds, launches = timed(lau, args.steps, args.warmup)
-        split = {k: round(sum(ms_ for _, ms_ in v) / args.steps, 3) for k, v in kinds.items()}
+            ms, kinds, launches = timed(lau, args.steps, args.warmup, not args.no_graph)
+        split = {k: round(sum(ms_ for _, ms_ in v) / (args.steps if args.no_graph else 1), 3) for k, v in kinds.items()}
         bpt = decode_bytes(w, lau.plan()) / tokens
         value = tokens / (ms / 1000.0)
         print(json.dumps({
@@ -648,6 +695,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
                     help="decode only this many tokens per step (small profiling runs; default: the workload's T)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="issue every launch directly in the timed steps (default: replay a CUDA graph of one decode)")
     ap.add_argument("--sweep-L", default="",
                     help="comma list of log capacities: one JSON line per L (fused deferred schedule, with the "
                          "read/merge split and bytes per token) after one eager line, inputs generated once")
@@ -715,12 +764,12 @@ def main(argv=None):
             S_def = d["S0"].clone()
             log = g.Log.allocate(w.B, w.H, w.d_k, w.d_v, L, tdt, chan, rwkv6=rw)
             lau = Launcher(g, w, d, S_def, log, o_all, args.schedule, stream)
-        ms_def, kinds_def, launches = timed(lau, args.steps, args.warmup)
+        ms_def, kinds_def, launches = timed(lau, args.steps, args.warmup, not args.no_graph)
         eager = None
         if not args.no_eager:
             S_e = d["S0"].clone()
             lau_e = Launcher(g, w, d, S_e, None, o_all, "eager", stream)
-            ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup)
+            ms_e, kinds_e, _ = timed(lau_e, args.steps, args.warmup, not args.no_graph)
             eager = {"value": w.B * w.T / (ms_e / 1000.0) * ws, "unit": UNIT, "ms_per_step": round(ms_e, 3),
                      "state_updates_per_s": w.heads * w.T / (ms_e / 1000.0) * ws,
                      "roofline": roofline_for(w, kinds_e, "eager", peak, peak_note, None)}
@@ -737,7 +786,8 @@ def main(argv=None):
 
     rf = roofline_for(wb, kinds_def, main_kind, peak, peak_note, traffic(main_kind))
     other = {k: roofline_for(wb, kinds_def, k, peak, peak_note, traffic(k)) for k in kinds_def if k != main_kind}
-    step_time = {k: round(sum(ms for _, ms in v) / args.steps, 3) for k, v in kinds_def.items()}
+    split_steps = 1 if not args.no_graph else args.steps
+    step_time = {k: round(sum(ms for _, ms in v) / split_steps, 3) for k, v in kinds_def.items()}
 
     e2e = None
     if not args.no_e2e and args.schedule != "pool" and not args.base_i8:

@@ -47,22 +47,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// A bounded wait for the phase with the given parity to complete. Each
-// try_wait suspends the thread for a hardware-chosen time; after `limit`
-// tries (seconds, far beyond any legitimate wait) the wait gives up, sets
-// bit `code` of *err and returns false. Once *err is set by any thread the
-// later waits of the block give up at once, so that a block that lost a
-// phase drains instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code,
-                                          uint32_t limit = 1u << 26) {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *(volatile int *)err != 0) return false;
-    }
-    atomicOr(err, 1 << code);
-    return false;
-}
-
 // ------------------------------------------------------------------ fences
 
 // Generic-proxy writes to shared memory become visible to the async proxy
