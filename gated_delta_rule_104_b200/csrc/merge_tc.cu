@@ -210,7 +210,8 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
         if (lane == 0) {
             constexpr uint32_t ID_G = tc::instr_desc(tc::FMT_TF32, false, false, ROWS, 2 * NB);
             constexpr uint32_t ID_W = tc::instr_desc(tc::FMT_TF32, false, false, ROWS, DK);
-            const uint32_t kf = tc::smem_u32(sm + LY.group(w) + LY.g_kf());
+            const uint32_t kh = tc::smem_u32(sm + LY.group(w) + LY.g_kh());
+            const uint32_t ff = tc::smem_u32(sm + LY.group(w) + LY.g_ff());
             const uint32_t tw = tbase + (uint32_t)w * TMEM_COLS_PER_GROUP;
             for (int j = 0, i = w; i < n_mine; ++j, i += NWG) {
                 const int s = i % NS;
@@ -224,7 +225,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 #pragma unroll
                     for (int kk = 0; kk < DK / 8; ++kk) {
                         const uint64_t ad = tc::smem_desc(tile + g_a_start(kk), 16, 1024, tc::SWZ_128);
-                        const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                        const uint64_t bd = tc::smem_desc(kh + g_b_start(kk), 16, 1024, tc::SWZ_128);
                         tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
                     }
                     bool ok = true;
@@ -238,7 +239,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 #pragma unroll
                         for (int kq = 0; kq < DK / 16; ++kq) {
                             const int kk = h * (DK / 16) + kq;
-                            const uint64_t bd = tc::smem_desc(kf + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                            const uint64_t bd = tc::smem_desc(kh + g_b_start(kk), 16, 1024, tc::SWZ_128);
                             tc::mma_ts_tf32(tw + COL_G, tw + COL_LO + 8 * kq, bd, ID_G, true);
                         }
                         tc::mma_commit(h == 0 ? B_LOFREE(w) : B_G(w));
@@ -249,7 +250,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                 tc::tc_fence_after();
 #pragma unroll
                 for (int m = 0; m < 6; ++m) {  // onto S o gamma
-                    const uint64_t bd = tc::smem_desc(kf + wb_b_start(m), 16, 1024, tc::SWZ_128);
+                    const uint64_t bd = tc::smem_desc(ff + wb_b_start(m), 16, 1024, tc::SWZ_128);
                     tc::mma_ts_tf32(tw + COL_SG, tw + COL_DL + wb_a_col(m), bd, ID_W, true);
                 }
                 tc::mma_commit(B_D(w));
@@ -269,8 +270,25 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
         float *qf = reinterpret_cast<float *>(gp + LY.g_qf());
         float *cn = reinterpret_cast<float *>(gp + LY.g_cn());
         float *red = reinterpret_cast<float *>(gp + LY.g_red());
-        uint8_t *kf = gp + LY.g_kf();
+        uint8_t *kh = gp + LY.g_kh();
+        uint8_t *ff = gp + LY.g_ff();
         const int bar_id = 1 + w;
+        // the unit's scalars from global memory (head-wise decays of every
+        // entry, which each thread needs all of, and the fused entry's beta),
+        // fetched one unit of the group ahead: behind the stages' bulk loads a
+        // plain load takes about as long as a unit
+        float adec_n[NB], bcur_n = 0.f;
+        auto fetch = [&](int i) {
+            const long long head = ((long long)blockIdx.x + (long long)i * gridDim.x) / tiles;
+#pragma unroll
+            for (int e = 0; e < NB; ++e) {
+                adec_n[e] = 1.f;
+                if (!CHAN && e < nb && i < n_mine)
+                    adec_n[e] = e < n_log ? ld_in(log_a + head * L + e) : ld_in(a + head);
+            }
+            if (DELTA && WITH_CUR && i < n_mine) bcur_n = ld_in(beta + head);
+        };
+        fetch(w);
         for (int j = 0, i = w; i < n_mine; ++j, i += NWG) {
             const int s = i % NS;
             const uint32_t par = (uint32_t)(j & 1);
@@ -283,19 +301,13 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
             uint8_t *sc = st + LY.off_sc();
             auto scf = [&](size_t off) { return *reinterpret_cast<const float *>(sc + off); };
             const Unit un = unit_of((long long)blockIdx.x + (long long)i * gridDim.x, tiles);
-            const long long lrow = un.head * L;
-            // the unit's scalars straight from global memory, before the wait:
-            // head-wise decays of every entry (each thread needs all of them) and
-            // the fused entry's beta
             float adec[NB];
 #pragma unroll
-            for (int e = 0; e < NB; ++e) {
-                adec[e] = 1.f;
-                if (!CHAN && e < nb) adec[e] = e < n_log ? ld_in(log_a + lrow + e) : ld_in(a + un.head);
-            }
-            const float bcur = (DELTA && WITH_CUR) ? ld_in(beta + un.head) : 0.f;
+            for (int e = 0; e < NB; ++e) adec[e] = adec_n[e];
+            const float bcur = bcur_n;
+            fetch(i + NWG);
             if (!wait_bar(B_FULL(s), (uint32_t)((i / NS) & 1), abort)) break;
-            if (j > 0) tc::named_sync(bar_id, 128);  // every warp's last stores have read the operand tile
+            if (j > 0) tc::named_sync(bar_id, 128);  // every warp's last stores have read its quarter of Khat
 
             // 1. key side for channel c: Khat (hi and lo parts), F, gamma, q
             float kc[NB], ac[NB];
@@ -312,14 +324,14 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     g *= ac[e];
                     if constexpr (DELTA) {
                         const float x = g * kc[e], hi = tc::tf32_trunc(x);
-                        *reinterpret_cast<float *>(kf + kh_off(e, c)) = hi;
-                        *reinterpret_cast<float *>(kf + kh_off(NB + e, c)) = x - hi;
+                        *reinterpret_cast<float *>(kh + kh_off(e, c)) = hi;
+                        *reinterpret_cast<float *>(kh + kh_off(NB + e, c)) = x - hi;
                     }
                 }
                 gam[c] = g;
                 if constexpr (WITH_CUR) qf[c] = to_f(rq[raw_q_off(c, 1)]);
             }
-            float fv[NB];  // F_e[c] (kept until G has been read; then it replaces Khat)
+            float fv[NB];  // F_e[c], into row c of F (this warp's quarter of F, which its last stores have read)
             {
                 float f = 1.f;
 #pragma unroll
@@ -327,9 +339,22 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     fv[e] = kc[e] * f;
                     f *= ac[e];
                 }
+                if (lane == 0) tc::bulk_wait_read<0>();
+                __syncwarp();
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {  // 16-byte pieces: hi of entries 4u.. (u < 4), lo (u >= 4)
+                    float4 wv;
+                    float *wp = reinterpret_cast<float *>(&wv);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x = fv[(4 * u + e) % NB], hi = tc::tf32_trunc(x);
+                        wp[e] = u < 4 ? hi : x - hi;
+                    }
+                    *reinterpret_cast<float4 *>(ff + ff_off(c, 4 * u)) = wv;
+                }
             }
-            if constexpr (DELTA) tc::fence_async_smem();  // Khat is read by the tensor cores
-            tc::named_sync(bar_id, 128);                   // Khat, gamma and q of every channel are in place
+            tc::fence_async_smem();       // Khat and F are read by the tensor cores
+            tc::named_sync(bar_id, 128);  // Khat, gamma and q of every channel are in place
             if (DELTA && ct == 0) tc::mbar_arrive(B_KH(w));
 
             // 2. one pass over the tile row: S o gamma into [COL_SG, +128), and
@@ -423,8 +448,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 #pragma unroll
             for (int e = 0; e < NB; ++e) vr[e] = e < nb ? to_f(rv[raw_v_off(e, r, 1)]) : 0.f;
 
-            // 4. delta = X (V - G) for row r (RWKV6: delta = V) into [COL_DL, +32);
-            //    F over Khat (G has read it)
+            // 4. delta = X (V - G) for row r (RWKV6: delta = V) into [COL_DL, +32)
             float dl[NB];
             if constexpr (DELTA) {
                 if (!wait_bar(B_G(w), par, abort)) break;
@@ -465,19 +489,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                 }
                 tc::tmem_st32(trow + COL_DL, wd);
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {  // 16-byte pieces: hi of entries 4u.. (u < 4), lo (u >= 4)
-                float4 wv;
-                float *wp = reinterpret_cast<float *>(&wv);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x = fv[(4 * u + e) % NB], hi = tc::tf32_trunc(x);
-                    wp[e] = u < 4 ? hi : x - hi;
-                }
-                *reinterpret_cast<float4 *>(kf + ff_off(c, 4 * u)) = wv;
-            }
             tc::tmem_wait_st();
-            tc::fence_async_smem();  // F is read by the tensor cores
             tc::tc_fence_before();
             tc::named_sync(bar_id, 128);
             if (ct == 0) {
@@ -492,8 +504,11 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 
             // 5. S_new = [COL_SG, +128) after the write-back: each warp's 32 rows
             //    to HBM by TMA, 32 columns at a time, through two staging tiles
-            //    used in turn (the first is the warp's quarter of the operand
-            //    tile, which the write-back has finished reading)
+            //    used in turn: the warp's quarters of Khat (which G has finished
+            //    reading) and of F (which the write-back has). Before a tile is
+            //    rewritten, the store that last used it has read it: stores
+            //    complete their reads in order, so waiting until at most one is
+            //    still reading suffices, at the next chunk and at the unit's end.
             if (!wait_bar(B_D(w), par, abort)) break;
             tc::tc_fence_after();
 #pragma unroll 1
@@ -501,7 +516,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                 uint32_t d[32];
                 tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
                 uint8_t *buf = sm + LY.group(w) + LY.out_buf(quad, ch & 1);
-                if (ch >= 2 && lane == 0) tc::bulk_wait_read<1>();  // the store that last used this tile has read it
+                if (ch >= 1 && lane == 0) tc::bulk_wait_read<1>();
                 __syncwarp();
                 tc::tmem_wait_ld();
 #pragma unroll
@@ -515,9 +530,10 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     tc::bulk_commit();
                 }
             }
-            // the operand tile is rewritten by the next unit's key side: this
-            // warp's stores from it (and from its other staging tile) have read them
-            if (lane == 0) tc::bulk_wait_read<0>();
+            // the warp's quarter of Khat, rewritten by the next unit's key side,
+            // is free once the third store has read it; the fourth may still be
+            // reading the warp's quarter of F, which the next F write waits for
+            if (lane == 0) tc::bulk_wait_read<1>();
             __syncwarp();
             tc::tc_fence_before();  // [COL_SG, +128) is rewritten by the group's next unit
         }

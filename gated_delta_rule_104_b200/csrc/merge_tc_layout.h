@@ -8,9 +8,9 @@
 // leaves it) and the raw log entries its merge needs; a stage is released as
 // soon as its unit no longer reads it (before the write-back), not when the
 // unit's result has been stored. NWG compute groups (1 or 2) each keep their
-// own operand tile (Khat, later F), a few vectors and a staging tile for the
-// TMA store of the result, and their own 256 columns of tensor memory; group w
-// merges the units i = w, w + NWG, ... of the CTA.
+// own operand tiles (Khat and F, which double as staging tiles for the TMA
+// stores of the result), a few vectors, and their own 256 columns of tensor
+// memory; group w merges the units i = w, w + NWG, ... of the CTA.
 #pragma once
 
 #include <stddef.h>
@@ -75,25 +75,25 @@ struct Layout {
     DL_HD constexpr size_t stage(int s) const { return (size_t)s * stage_bytes(); }
 
     // ---- one compute group's regions (from the group's base)
-    // The operand tile: first Khat, the B operand of G (32 rows: entries' hi
-    // parts 0..15, lo parts 16..31, x 128 key channels, K-major, 128-byte
-    // swizzle; column chunk c = channels 32c..32c+31 is a [32 x 128 B] block at
-    // 4 KiB c); once G has been read, F, the B operand of the write-back (128
-    // rows = key channels x 32: entries' hi parts 0..15, lo parts 16..31,
-    // K-major, 128-byte swizzle).
-    DL_HD constexpr size_t g_kf() const { return 0; }
-    DL_HD constexpr size_t kf_bytes() const { return (size_t)2 * NB * DK * 4; }
+    // Khat, the B operand of G: 32 rows (entries' hi parts 0..15, lo parts
+    // 16..31) x 128 key channels, K-major, 128-byte swizzle; column chunk c =
+    // channels 32c..32c+31 is a [32 x 128 B] block at 4 KiB c.
+    DL_HD constexpr size_t g_kh() const { return 0; }
+    DL_HD constexpr size_t kh_bytes() const { return (size_t)2 * NB * DK * 4; }
+    // F, the B operand of the write-back: 128 rows (key channels) x 32
+    // (entries' hi parts 0..15, lo parts 16..31), K-major, 128-byte swizzle;
+    // rows 32q..32q+31 are the quarter q (4 KiB).
+    DL_HD constexpr size_t g_ff() const { return g_kh() + kh_bytes(); }
+    DL_HD constexpr size_t ff_bytes() const { return (size_t)DK * 2 * NB * 4; }
     // the staging tiles of the result's TMA stores, two per warp of the group
     // (used in turn): warp quad q (rows 32q..32q+31) stages one 32-column
     // chunk of its rows, [32 rows x 128 B] with 128-byte swizzle. Tile 0 is
-    // the warp's quarter of the operand tile (free once the write-back has
-    // read F), tile 1 its quarter of this region.
-    DL_HD constexpr size_t g_out() const { return g_kf() + kf_bytes(); }
-    DL_HD constexpr size_t out_bytes() const { return (size_t)ROWS * 128; }
+    // the warp's quarter of Khat (free once G has read it), tile 1 its quarter
+    // of F (free once the write-back has read it).
     DL_HD constexpr size_t out_buf(int quad, int b) const {
-        return (b == 0 ? g_kf() : g_out()) + (size_t)quad * 32 * 128;
+        return (b == 0 ? g_kh() : g_ff()) + (size_t)quad * 32 * 128;
     }
-    DL_HD constexpr size_t g_gam() const { return g_out() + out_bytes(); }  // gamma [128] floats
+    DL_HD constexpr size_t g_gam() const { return g_ff() + ff_bytes(); }    // gamma [128] floats
     DL_HD constexpr size_t g_qf() const { return g_gam() + DK * 4; }        // q widened [128] floats
     // the fused read's sums over key channels: C(n, e) (16) then (F q)_e (16)
     DL_HD constexpr size_t g_cn() const { return g_qf() + DK * 4; }
@@ -142,13 +142,13 @@ DL_HD constexpr uint32_t swz128(uint32_t off) { return off ^ ((off & 0x380u) >> 
 DL_HD constexpr uint32_t tile_off(int r, int c) {
     return (uint32_t)((c / CHUNK) * (ROWS * 128)) + swz128((uint32_t)(r * 128 + (c % CHUNK) * 4));
 }
-// Khat element (row n in 0..31, channel c) inside the operand tile.
+// Khat element (row n in 0..31, channel c) inside Khat.
 DL_HD constexpr uint32_t kh_off(int n, int c) {
     return (uint32_t)((c / CHUNK) * (2 * NB * 128)) + swz128((uint32_t)(n * 128 + (c % CHUNK) * 4));
 }
-// F element (channel c, column j in 0..31) inside the operand tile.
+// F element (channel c, column j in 0..31) inside F.
 DL_HD constexpr uint32_t ff_off(int c, int j) { return swz128((uint32_t)(c * 128 + j * 4)); }
-// Groups the launch can afford: two when their operand tiles fit beside the
+// Groups the launch can afford: two when their regions fit beside the
 // two stages, else one.
 DL_HD constexpr int groups_for(size_t in_size, bool chan) {
     return Layout{in_size, chan, 2}.request() <= SMEM_LIMIT ? 2 : 1;

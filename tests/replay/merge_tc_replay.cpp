@@ -59,8 +59,8 @@ struct Replay {
         }
         for (int w = 0; w < ly.nwg; ++w) {
             const std::string p = "group" + std::to_string(w) + ".";
-            add(p + "kf", ly.group(w) + ly.g_kf(), ly.kf_bytes());
-            add(p + "out", ly.group(w) + ly.g_out(), ly.out_bytes());
+            add(p + "kh", ly.group(w) + ly.g_kh(), ly.kh_bytes());
+            add(p + "ff", ly.group(w) + ly.g_ff(), ly.ff_bytes());
             add(p + "gam", ly.group(w) + ly.g_gam(), DK * 4);
             add(p + "qf", ly.group(w) + ly.g_qf(), DK * 4);
             add(p + "cn", ly.group(w) + ly.g_cn(), 2 * NB * 4);        // C(n, e) then (F q)_e
@@ -104,7 +104,7 @@ struct Replay {
         if (ly.end() + 1023 > ly.request()) fail("no room for the 1024-byte base alignment", tag());
         if (ly.stage_bytes() % 1024) fail("stage not 1024-aligned", tag());
         for (int w = 0; w < ly.nwg; ++w)
-            if ((ly.group(w) + ly.g_kf()) % 1024 || (ly.group(w) + ly.g_out()) % 1024)
+            if ((ly.group(w) + ly.g_kh()) % 1024 || (ly.group(w) + ly.g_ff()) % 1024)
                 fail("operand region not 1024-aligned", tag());
         if (ly.nwg < 1 || ly.nwg > 2 || (int)tmem_cols_for(ly.nwg) < ly.nwg * (int)TMEM_COLS_PER_GROUP)
             fail("tensor memory for the groups", tag());
@@ -185,8 +185,8 @@ struct Replay {
                     acc(p + "raw_v", raw_v_off(j, r, in_size), in_size, in_size, "v read");
                 }
                 if (delta) {
-                    acc(gp + "kf", kh_off(j, c), 4, 4, "Khat hi");
-                    acc(gp + "kf", kh_off(NB + j, c), 4, 4, "Khat lo");
+                    acc(gp + "kh", kh_off(j, c), 4, 4, "Khat hi");
+                    acc(gp + "kh", kh_off(NB + j, c), 4, 4, "Khat lo");
                     khs.insert(kh_off(j, c));
                     khs.insert(kh_off(NB + j, c));
                     for (int m4 = 0; m4 <= j / 4; ++m4) acc(p + "sc", sc_x(j, 4 * m4), 16, 16, "X row piece");
@@ -198,7 +198,11 @@ struct Replay {
                 acc(p + "raw_q", raw_q_off(c, in_size), in_size, in_size, "q raw read");
             }
             for (int u = 0; u < 8; ++u) {
-                acc(gp + "kf", ff_off(c, 4 * u), 16, 16, "F piece");
+                acc(gp + "ff", ff_off(c, 4 * u), 16, 16, "F piece");
+                // F row c lies in the warp's own quarter of F (its staging tile 1)
+                const size_t q1 = ly.out_buf(quad, 1) - ly.g_ff();
+                if (ff_off(c, 4 * u) < q1 || ff_off(c, 4 * u) + 16 > q1 + 32 * 128)
+                    fail("F piece outside the warp's own quarter", tag());
                 for (int e = 0; e < 4; ++e) {
                     if (ff_off(c, 4 * u + e) != ff_off(c, 4 * u) + 4u * e) fail("F piece not contiguous", tag());
                     ffs.insert(ff_off(c, 4 * u + e));
@@ -226,8 +230,8 @@ struct Replay {
                 acc(p + "tile", tile_off(r, col), 16, 16, "tile piece");
                 if (col < CHUNK)  // the warp's two staging tiles: its 32 rows of one 32-column chunk
                     for (int b = 0; b < 2; ++b) {
-                        const char *reg = b == 0 ? "kf" : "out";
-                        const size_t base = b == 0 ? ly.g_kf() : ly.g_out();
+                        const char *reg = b == 0 ? "kh" : "ff";
+                        const size_t base = b == 0 ? ly.g_kh() : ly.g_ff();
                         const size_t o = ly.out_buf(quad, b) - base + tile_off(lane, col);
                         acc(gp + reg, o, 16, 16, "staging piece");
                         if (tile_off(lane, col) >= 32 * 128) fail("staging piece outside its tile", tag());
@@ -273,7 +277,7 @@ struct Replay {
                         if (row < 2 * NB) {
                             const uint32_t b = desc_elem(g_b_start(kk), row, k);
                             if (b != kh_off(row, 8 * kk + k)) fail("G's B operand is not the Khat element", tag());
-                            if (b + 4 > ly.kf_bytes()) fail("G's B read outside Khat", tag());
+                            if (b + 4 > ly.kh_bytes()) fail("G's B read outside Khat", tag());
                         }
                     }
                     if (a + 4 > ly.tile()) fail("G's A read outside the tile", tag());
@@ -285,7 +289,7 @@ struct Replay {
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t b = desc_elem(wb_b_start(m), row, k);
                     if (b != ff_off(row, jbase + k)) fail("write-back's B operand is not the F element", tag());
-                    if (b + 4 > ly.kf_bytes()) fail("write-back's B read outside F", tag());
+                    if (b + 4 > ly.ff_bytes()) fail("write-back's B read outside F", tag());
                 }
             // A in tensor memory: delta columns of the same entries (hi for m < 4, lo after)
             const int acol = COL_DL + wb_a_col(m);

@@ -41,7 +41,7 @@ def test_every_access_in_bounds_and_aligned(replay):
     assert "192 cases, 0 failures" in r.stdout
 
 
-@pytest.mark.parametrize("region", ["sc", "kf", "out", "raw_v", "raw_q", "red", "qf", "gam", "tile"])
+@pytest.mark.parametrize("region", ["sc", "kh", "ff", "raw_k", "raw_v", "raw_q", "red", "qf", "gam", "tile"])
 def test_a_planted_four_byte_overrun_is_caught(replay, region):
     r = run(replay, "shrink", region, "4")
     assert r.returncode == 1, r.stdout[-2000:]
