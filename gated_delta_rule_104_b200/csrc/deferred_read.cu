@@ -40,21 +40,11 @@
 //                 replay_prep still runs: it issues its base loads first and
 //                 waits for the prep grid only before reading the workspace.
 #include "launch.h"
+#include "prep_layout.h"
 
 namespace dl {
 
 // ------------------------------------------------------------------ prep
-
-template <class IT, int DK, int EMAX, bool CHAN>
-struct PrepSmem {  // one warp's staging area
-    static constexpr int ROWB = DK * (int)sizeof(IT);           // bytes of one key row
-    static constexpr int K_OFF = 0;
-    static constexpr int A_OFF = K_OFF + EMAX * ROWB;           // channel decays (raw)
-    static constexpr int F_OFF = A_OFF + (CHAN ? EMAX * ROWB : 0);
-    // floats from F_OFF: as[EMAX], beta[EMAX], d[EMAX], cn[EMAX], sv[EMAX], xrow[EMAX][EMAX]
-    static constexpr int FLOATS = 5 * EMAX + EMAX * EMAX;
-    static constexpr int BYTES = F_OFF + FLOATS * 4;
-};
 
 template <class IT, int DK, int DV, int KIND, int EMAX>
 __global__ void __launch_bounds__(128)
@@ -65,7 +55,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
                    PoolIdx pool) {
     pdl_launch_dependents();
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
-    using P = PrepSmem<IT, DK, EMAX, CHAN>;
+    using P = PrepSmem<(int)sizeof(IT), DK, EMAX, CHAN>;
     constexpr int CW = DK / 32;            // key columns per lane (contiguous)
     constexpr int RV = DV / 32;            // value rows per lane
     constexpr int CH = EMAX < 32 ? EMAX : 32;  // entries per butterfly
@@ -75,8 +65,9 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     unsigned char *base = reinterpret_cast<unsigned char *>(smem_raw) + (size_t)warp * P::BYTES;
     IT *sk = reinterpret_cast<IT *>(base + P::K_OFF);
     IT *sa = reinterpret_cast<IT *>(base + P::A_OFF);
-    float *fas = reinterpret_cast<float *>(base + P::F_OFF);
-    float *fbeta = fas + EMAX, *fd = fbeta + EMAX, *fcn = fd + EMAX, *fs = fcn + EMAX, *xrow = fs + EMAX;
+    float *fl = reinterpret_cast<float *>(base + P::F_OFF);
+    float *fas = fl + P::AS, *fbeta = fl + P::BETA, *fd = fl + P::D, *fcn = fl + P::CN, *fs = fl + P::S,
+          *xrow = fl + P::XROW;
 
     // A pool step launches this kernel as a programmatic dependent of its merge
     // part (which works on other slots), so the two overlap; every warp waits
@@ -408,8 +399,8 @@ static cudaError_t launch_decode(const StepParams &p, const float *work, cudaStr
 template <class IT, int DK, int DV, int KD, int EMAX>
 static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
                                const PoolIdx &pool) {
-    using P = PrepSmem<IT, DK, EMAX, Rule<KD>::CHAN>;
-    constexpr int WARPS = EMAX <= 32 ? 4 : 2;
+    using P = PrepSmem<(int)sizeof(IT), DK, EMAX, Rule<KD>::CHAN>;
+    constexpr int WARPS = prep_warps(EMAX);
     auto kern = replay_prep_kernel<IT, DK, DV, KD, EMAX>;
     const size_t smem = (size_t)WARPS * P::BYTES;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), smem);
@@ -440,8 +431,9 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
         constexpr int DV = decltype(dv_c)::value;
         constexpr int KD = decltype(ch_c)::value;
         cudaError_t e;
-        if (lg.L <= 16) e = launch_prep<IT, DK, DV, KD, 16>(p, lg, n, work, st, pool);
-        else if (lg.L <= 32) e = launch_prep<IT, DK, DV, KD, 32>(p, lg, n, work, st, pool);
+        const int emax = prep_emax(lg.L);
+        if (emax == 16) e = launch_prep<IT, DK, DV, KD, 16>(p, lg, n, work, st, pool);
+        else if (emax == 32) e = launch_prep<IT, DK, DV, KD, 32>(p, lg, n, work, st, pool);
         else e = launch_prep<IT, DK, DV, KD, 64>(p, lg, n, work, st, pool);
         if (e != cudaSuccess) return e;
         if (p.s_dt == DL_I8) e = launch_decode<int8_t, DK, DV>(p, work, st, pool);

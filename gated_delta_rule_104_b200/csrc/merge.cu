@@ -45,6 +45,7 @@
 //     accumulator layout.
 // A pool step's merge part runs the same body over a compact grid (below).
 #include "launch.h"
+#include "merge_layout.h"
 
 namespace dl {
 
@@ -102,75 +103,12 @@ __device__ __forceinline__ void st_state4(bf16 *p, float4 x) {
 //    16j + 4 (n / 2) + 2h + n mod 2.
 // Either way lane (g, t) holds columns 16j + 4t .. 16j + 4t + 3 of its rows, so
 // the base tile, Khat, gamma, q and the merged rows move 16 bytes per access.
-// F is stored in the order the update's B fragments read it: column c at
-// position f_pos(c) = 16j + 8h + n of its group.
-__device__ __forceinline__ int f_pos(int c) {
-    return (c & ~15) | (((c >> 1) & 1) << 3) | (((c >> 2) & 3) << 1) | (c & 1);
-}
-
-// ------------------------------------------------------------------ layout
-
-__host__ __device__ constexpr size_t round4(size_t x) { return (x + 3) & ~(size_t)3; }
-
-template <int DK, int NB>
-struct MergeShape {
-    static constexpr int ROWS = 64;     // base rows per block: 4 warps of 16
-    static constexpr int KH = DK;       // Khat row stride (no padding: the rows are swizzled, kof)
-    static constexpr int WS = DK + 8;   // F row stride (conflict-free B-fragment reads)
-    static constexpr int XS = NB + 4;   // X row stride (conflict-free B-fragment reads)
-    static constexpr int VS = ROWS + 4; // value row stride (conflict-free accumulator-layout reads)
-    static constexpr int CW = DK / 32;  // key channels per lane (warp-wide dots)
-    // Khat element (i, c): the 16-byte chunks of row i XOR-swizzled by 4 (i mod 2),
-    // so that a 16-byte B-fragment read (rows 2m and 2m + 1 in one 8-lane phase)
-    // hits every bank; a pair of chunks 2u, 2u + 1 stays adjacent.
-    __device__ static __forceinline__ int kof(int i, int c) {
-        return i * KH + ((((c >> 2) ^ ((i & 1) << 2)) << 2) | (c & 3));
-    }
-};
-
-// The block's base rows in shared memory: ROWS x DK elements of the tile
-// type, row-major, with the 16-byte chunks of row r XOR-swizzled by f(r). Every
-// access is lane (g, t) moving columns 16j + 4t .. + 3 of row g (or g + 8):
-//  - fp32: one 128-byte phase is 8 lanes, rows r, r + 1 with 4 chunks each;
-//    f(r) = 4 (r mod 2) puts the two rows in opposite halves of the banks;
-//  - bf16: one phase is 16 lanes of 8 bytes, rows r .. r + 3 with a chunk pair
-//    each; f(r) = 2 (r mod 4) puts the four pairs on distinct banks.
-// No padding.
-template <class ST, int DK>
-struct BaseTile {
-    static constexpr int CE = 16 / (int)sizeof(ST);  // elements per 16-byte chunk
-    static_assert(DK / CE >= 8, "swizzle spans 8 chunks");
-    __device__ static __forceinline__ int off(int r, int c) {
-        const int f = CE == 4 ? (r & 1) << 2 : (r & 3) << 1;
-        return r * DK + (((c / CE) ^ f) * CE) + (c % CE);
-    }
-};
-
-// Shared memory (bytes) of one block for NB-entry sub-merges:
-//   tile [ROWS][DK] of the tile type (swizzled base rows: float for an int8
-//   base, else the state type), then floats:
-//   kh [NB][KH] keys, turned into Khat in place
-//   ff [NB][WS] F (channel decay: holds the decays until F replaces them)
-//   fa [NB] head decays (padded to 4)   gn [DK] gamma   sq [DK] q
-//   sx [NB][XS] X   sb [NB] beta   sv [NB][VS] the tile's values
-//   sxw [4][XS] each warp's copy of the fused entry's X row
-//   xw [5] (after the int8 arrays, if any) a compact grid's walk: four ballots
-//   and the batch index, XW_BYTES
-//   int8 base only: scl [ROWS] row scales, wsc [4][16] the new row scales of
-//   each warp's rows; the codes [ROWS][DK] land in the last ROWS * DK bytes of
-//   the float tile and are read out into registers before it is widened over
-//   them (no separate code buffer: four blocks per SM, as for a float base)
-constexpr size_t XW_BYTES = 32;  // the compact walk's five words, padded to 16-byte granules
+// F is stored in the order the update's B fragments read it (f_pos, in
+// merge_layout.h, with the block's shared-memory layout).
 
 template <class ST, int DK, int NB>
 __host__ __device__ constexpr size_t merge_smem_bytes() {
-    using C = MergeShape<DK, NB>;
-    constexpr bool Q8 = std::is_same<ST, int8_t>::value;
-    using TT = typename std::conditional<Q8, float, ST>::type;
-    const size_t floats = (size_t)NB * C::KH + (size_t)NB * C::WS + round4(NB) + DK + DK +
-                          (size_t)NB * C::XS + round4(NB) + (size_t)NB * C::VS + 4 * (size_t)C::XS;
-    const size_t q8 = Q8 ? (size_t)C::ROWS * 4 + 64 * 4 : 0;
-    return (size_t)C::ROWS * DK * sizeof(TT) + floats * sizeof(float) + q8 + XW_BYTES;
+    return MergeRegions<(int)sizeof(ST), std::is_same<ST, int8_t>::value, DK, NB>::bytes;
 }
 
 // Accumulator layout (rows g, g + 8; columns 8i + 2t, 8i + 2t + 1) to A-operand
@@ -208,27 +146,29 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     // as a float base, and its rows rounded back to int8 when they are stored.
     constexpr bool Q8 = std::is_same<ST, int8_t>::value;
     using TT = typename std::conditional<Q8, float, ST>::type;
-    using TL = BaseTile<TT, DK>;
+    using TL = BaseTile<(int)sizeof(TT), DK>;
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
     constexpr int NT = NB / 8;   // entry tiles
     constexpr int ROWS = C::ROWS;
     constexpr int nthr = 2 * ROWS;  // 4 warps, 16 rows each
 
+    using RG = MergeRegions<(int)sizeof(ST), Q8, DK, NB>;
     extern __shared__ float4 smem_raw[];
     TT *tile = reinterpret_cast<TT *>(smem_raw);
-    float *kh = reinterpret_cast<float *>(tile + ROWS * DK);
-    float *ff = kh + NB * C::KH;
-    float *fa = ff + NB * C::WS;
-    float *gn = fa + round4(NB);
-    float *sq = gn + DK;
-    float *sx = sq + DK;
-    float *sb = sx + NB * C::XS;
-    float *sv = sb + round4(NB);
-    float *sxw = sv + NB * C::VS;
+    float *fl = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_raw) + RG::tile_bytes);
+    float *kh = fl + RG::kh;
+    float *ff = fl + RG::ff;
+    float *fa = fl + RG::fa;
+    float *gn = fl + RG::gn;
+    float *sq = fl + RG::sq;
+    float *sx = fl + RG::sx;
+    float *sb = fl + RG::sb;
+    float *sv = fl + RG::sv;
+    float *sxw = fl + RG::sxw;
     // int8 base only: the codes at the end of the (float) tile, the scales after sxw
-    int8_t *raw = reinterpret_cast<int8_t *>(tile) + (size_t)ROWS * DK * (sizeof(TT) - 1);
-    float *scl = sxw + 4 * C::XS;
-    float *wsc = scl + ROWS;
+    int8_t *raw = reinterpret_cast<int8_t *>(smem_raw) + RG::raw_bytes_off;
+    float *scl = fl + RG::scl;
+    float *wsc = fl + RG::wsc;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;  // fragment coordinates
@@ -243,7 +183,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     // them one after another. The walk's state lives in shared memory, so that
     // nothing of it stays in registers across a merge.
     const bool compact = units != (long long)gridDim.x;
-    uint32_t *xw = reinterpret_cast<uint32_t *>(Q8 ? wsc + 64 : sxw + 4 * C::XS);
+    uint32_t *xw = reinterpret_cast<uint32_t *>(fl + RG::xw);
     if (compact) {
         if (tid < 4) xw[tid] = 0u;
         if (tid == 0) xw[4] = 0xffffffffu;  // batch -1: none checked yet
