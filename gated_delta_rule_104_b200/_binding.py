@@ -12,18 +12,21 @@ import os
 from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libdeltalog.so")
+# the library a process loads: libdeltalog.so, or the file DELTALOG_LIBRARY
+# names (e.g. the index-guard debug build, libdeltalog_guard.so)
+LIB_PATH = os.environ.get("DELTALOG_LIBRARY") or os.path.join(HERE, "libdeltalog.so")
+GUARD_LIB_PATH = os.path.join(HERE, "libdeltalog_guard.so")
 
 DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_LOG_FULL, DL_ERR_CUDA = range(5)
 DL_F32, DL_BF16, DL_I8 = 0, 1, 2
 DL_DECAY_HEAD, DL_DECAY_CHANNEL, DL_RWKV6 = 0, 1, 2
 DL_MAX_LOG = 64
-ABI_VERSION = 8
+ABI_VERSION = 9
 
 EXPORTS = ("dl_gdn_decode_step", "dl_kda_decode_step", "dl_rwkv6_decode_step", "dl_log_append_read", "dl_log_merge",
            "dl_log_merge_read", "dl_log_work_bytes", "dl_log_append_read_noalloc", "dl_pool_step",
            "dl_pool_flush", "dl_state_bytes", "dl_state_to_i8", "dl_state_from_i8", "dl_status_string",
-           "dl_last_error", "dl_abi_version", "dl_device_faults")
+           "dl_last_error", "dl_abi_version", "dl_device_faults", "dl_index_guard_build")
 DL_NOALLOC_WORK_BYTES = 16 << 20
 
 
@@ -88,6 +91,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dl_abi_version.restype = ctypes.c_int
     lib.dl_device_faults.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]
     lib.dl_device_faults.restype = ctypes.c_int
+    lib.dl_index_guard_build.argtypes = []
+    lib.dl_index_guard_build.restype = ctypes.c_int
     if lib.dl_abi_version() != ABI_VERSION:
         raise RuntimeError(f"libdeltalog.so ABI {lib.dl_abi_version()} != binding ABI {ABI_VERSION}: rebuild")
     if path is None:
@@ -330,10 +335,16 @@ def dl_log_merge(S_base, log: Log, n: int, stream=None) -> None:
 
 def dl_device_faults(clear: bool = False) -> int:
     """The kernels' fault word on the current device (0: no bounded wait ran
-    out). Synchronises the device."""
+    out and, in the index-guard build, no shared-memory write was out of
+    bounds). Synchronises the device."""
     w = ctypes.c_uint(0)
     check("dl_device_faults", load().dl_device_faults(ctypes.byref(w), 1 if clear else 0))
     return int(w.value)
+
+
+def dl_index_guard_build() -> bool:
+    """Whether the loaded library is the index-guard debug build."""
+    return bool(load().dl_index_guard_build())
 
 
 def dl_status_string(status: int) -> str:

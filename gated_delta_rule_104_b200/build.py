@@ -5,7 +5,12 @@ arch=compute_100a,code=sm_100a``), with line info, into one shared library
 that exports the C ABI declared in ``include/deltalog.h``. The CUDA runtime
 is linked statically, so the library depends only on the driver.
 
-Usage: ``python -m gated_delta_rule_104_b200.build [--force] [-v]``
+``--guard`` builds the index-guard debug library instead,
+``libdeltalog_guard.so`` (the same sources with ``-DDL_INDEX_GUARD``: every
+shared-memory write of the kernels checks its bounds and alignment, skips
+and records a write that fails; see ``csrc/guard.cuh``).
+
+Usage: ``python -m gated_delta_rule_104_b200.build [--force] [--guard] [-v]``
 """
 from __future__ import annotations
 
@@ -21,6 +26,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdeltalog.so")
+GUARD_LIB = os.path.join(HERE, "libdeltalog_guard.so")
 OBJDIR = os.path.join(HERE, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -44,22 +50,26 @@ def _deps():
         [os.path.join(INCLUDE, "deltalog.h"), __file__]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, jobs: int = 0, guard: bool = False) -> str:
+    lib = GUARD_LIB if guard else LIB
+    if not force and up_to_date(lib):
+        return lib
+    objdir = OBJDIR + ("_guard" if guard else "")
+    os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     objs, procs = [], []
     extra = ["-Xptxas", "-v"] if verbose else []
+    if guard:
+        extra.append("-DDL_INDEX_GUARD")
     for src in sources():
-        obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         cmd = [cc, *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -72,15 +82,16 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
             failed.append(" ".join(cmd))
     if failed:
         raise RuntimeError("nvcc failed:\n" + "\n".join(failed))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     subprocess.run([cc, *ARCH, "-shared", "-o", tmp, *objs], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--guard", action="store_true", help="the index-guard debug library")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, guard=a.guard))

@@ -384,7 +384,35 @@ int dl_abi_version(void) { return DL_ABI_VERSION; }
 dl_status dl_device_faults(unsigned int *flags, int clear) {
     if (!flags) return fail(DL_ERR_INVALID_ARG, "flags is a null pointer");
     *flags = 0;
-    return cuda_status(dl::read_tc_faults(flags, clear != 0), "fault word read");
+    unsigned int w = 0;
+    dl_status st = cuda_status(dl::read_tc_faults(&w, clear != 0), "fault word read");
+    if (st != DL_OK) return st;
+    *flags = w;
+    struct {
+        const char *file;
+        cudaError_t (*read)(unsigned int *, unsigned int *, bool);
+    } const units[] = {{"merge.cu", dl::read_guard_merge},
+                       {"deferred_read.cu", dl::read_guard_read},
+                       {"merge_tc.cu", dl::read_guard_merge_tc}};
+    for (const auto &u : units) {
+        unsigned int g = 0, line = 0;
+        st = cuda_status(u.read(&g, &line, clear != 0), "guard word read");
+        if (st != DL_OK) return st;
+        if (g) {
+            *flags |= g;
+            snprintf(g_err, sizeof g_err, "index guard: an out-of-bounds shared-memory write was skipped (%s:%u)",
+                          u.file, line);
+        }
+    }
+    return DL_OK;
+}
+
+int dl_index_guard_build(void) {
+#ifdef DL_INDEX_GUARD
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 }  // extern "C"

@@ -40,6 +40,7 @@
 //                 replay_prep still runs: it issues its base loads first and
 //                 waits for the prep grid only before reading the workspace.
 #include "launch.h"
+#include "guard.cuh"
 #include "prep_layout.h"
 
 namespace dl {
@@ -90,11 +91,15 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     for (int u = lane; u < (n + 1) * (DK / E); u += 32) {
         const int e = u / (DK / E), col = (u % (DK / E)) * E;
         if (e < n) {
-            cp_async16(sk + e * DK + col, log_k + (lrow + e) * DK + col);
-            if constexpr (CHAN) cp_async16(sa + e * DK + col, log_a + (lrow + e) * DK + col);
+            DL_GUARD(sk + e * DK + col, 16) cp_async16(sk + e * DK + col, log_k + (lrow + e) * DK + col);
+            if constexpr (CHAN) {
+                DL_GUARD(sa + e * DK + col, 16) cp_async16(sa + e * DK + col, log_a + (lrow + e) * DK + col);
+            }
         } else {
-            cp_async16(sk + e * DK + col, k + head * DK + col);
-            if constexpr (CHAN) cp_async16(sa + e * DK + col, a + head * DK + col);
+            DL_GUARD(sk + e * DK + col, 16) cp_async16(sk + e * DK + col, k + head * DK + col);
+            if constexpr (CHAN) {
+                DL_GUARD(sa + e * DK + col, 16) cp_async16(sa + e * DK + col, a + head * DK + col);
+            }
         }
     }
     cp_async_commit();
@@ -136,7 +141,9 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll
         for (int i = 0; i < XB; ++i) {
             const int u = base + i * 32 + lane, j = u / EMAX, e = u % EMAX;
-            if (DELTA && u < n * EMAX && e <= j) xrow[j * EMAX + e] = xx[i];
+            if (DELTA && u < n * EMAX && e <= j) {
+                DL_GUARD(xrow + j * EMAX + e, 4) xrow[j * EMAX + e] = xx[i];
+            }
         }
     };
     x_load(0);
@@ -156,11 +163,11 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
             float t1[1];
             if constexpr (DELTA) {
                 bx[i].widen(t1);
-                fbeta[e] = t1[0];
+                DL_GUARD(fbeta + e, 4) fbeta[e] = t1[0];
             }
             if constexpr (!CHAN) {
                 ax[i].widen(t1);
-                fas[e] = t1[0];
+                DL_GUARD(fas + e, 4) fas[e] = t1[0];
             }
         }
     }
@@ -221,8 +228,8 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         constexpr int shift = CH == 32 ? 0 : CH == 16 ? 1 : CH == 8 ? 2 : 3;
         const int e = top - (lane >> shift);
         if ((lane & ((1 << shift) - 1)) == 0 && e >= 0) {
-            fd[e] = pd[0];
-            fcn[e] = pc[0];  // (C(n, n) is not used)
+            DL_GUARD(fd + e, 4) fd[e] = pd[0];
+            DL_GUARD(fcn + e, 4) fcn[e] = pc[0];  // (C(n, n) is not used)
         }
     }
     __syncwarp();
@@ -233,7 +240,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll 4
         for (int m = j; m < n; ++m) acc = fmaf(fcn[m], xrow[m * EMAX + j], acc);
         const float xnj = j == n ? bn : -bn * acc;
-        xrow[n * EMAX + j] = xnj;
+        DL_GUARD(xrow + n * EMAX + j, 4) xrow[n * EMAX + j] = xnj;
         st_hint(log_x + (lrow + n) * L + j, __float_as_uint(xnj), keep);
     }
     __syncwarp();
@@ -246,7 +253,7 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         } else {
             acc = fd[e];
         }
-        fs[e] = acc;
+        DL_GUARD(fs + e, 4) fs[e] = acc;
     }
     __syncwarp();
 
@@ -477,6 +484,11 @@ cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg,
     cudaError_t e = noalloc_work_address(&work);
     if (e != cudaSuccess) return e;
     return launch_append_read(p, lg, n, work, st);
+}
+
+// The guard word of this file's kernels (index-guard build; 0 otherwise).
+cudaError_t read_guard_read(unsigned int *flags, unsigned int *line, bool clear) {
+    return read_guard_word(flags, line, clear);
 }
 
 }  // namespace dl

@@ -107,6 +107,11 @@ cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log,
 // The tensor-core kernels' fault word (bit 0: a bounded wait ran out), read
 // synchronously; cleared afterwards when `clear`.
 cudaError_t read_tc_faults(unsigned int *out, bool clear);
+// index-guard words of the kernels' files (bit 1: a shared-memory write out of
+// bounds was skipped; line: the source line of the first); 0 in the ordinary build
+cudaError_t read_guard_merge(unsigned int *flags, unsigned int *line, bool clear);
+cudaError_t read_guard_read(unsigned int *flags, unsigned int *line, bool clear);
+cudaError_t read_guard_merge_tc(unsigned int *flags, unsigned int *line, bool clear);
 // State conversions to / from the int8 layout (rows = B*H*d_v rows of d_k).
 cudaError_t launch_to_i8(const void *S, dl_dtype s_dt, void *S_i8, long long rows, int dk, cudaStream_t st);
 cudaError_t launch_from_i8(const void *S_i8, void *S, dl_dtype s_dt, long long rows, int dk, cudaStream_t st);

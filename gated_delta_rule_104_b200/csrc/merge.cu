@@ -45,6 +45,7 @@
 //     accumulator layout.
 // A pool step's merge part runs the same body over a compact grid (below).
 #include "launch.h"
+#include "guard.cuh"
 #include "merge_layout.h"
 
 namespace dl {
@@ -185,8 +186,12 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
     const bool compact = units != (long long)gridDim.x;
     uint32_t *xw = reinterpret_cast<uint32_t *>(fl + RG::xw);
     if (compact) {
-        if (tid < 4) xw[tid] = 0u;
-        if (tid == 0) xw[4] = 0xffffffffu;  // batch -1: none checked yet
+        if (tid < 4) {
+            DL_GUARD(xw + tid, 4) xw[tid] = 0u;
+        }
+        if (tid == 0) {
+            DL_GUARD(xw + 4, 4) xw[4] = 0xffffffffu;  // batch -1: none checked yet
+        }
         __syncthreads();
     }
     for (;;) {
@@ -211,7 +216,9 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                 }
                 const uint32_t bal = __ballot_sync(0xffffffffu, mine);
                 __syncthreads();  // every thread has read the previous words
-                if (lane == 0) xw[warp] = bal;
+                if (lane == 0) {
+                    DL_GUARD(xw + warp, 4) xw[warp] = bal;
+                }
                 __syncthreads();
 #pragma unroll
                 for (int w = 0; w < 4; ++w) m[w] = xw[w];
@@ -222,8 +229,8 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
             unit = (long long)blockIdx.x + ((long long)batch * nthr + 32 * w + bit) * gridDim.x;
             __syncthreads();  // every thread has read the words before they change
             if (tid == 0) {
-                xw[w] = m[w] & (m[w] - 1u);
-                xw[4] = (uint32_t)batch;
+                DL_GUARD(xw + w, 4) xw[w] = m[w] & (m[w] - 1u);
+                DL_GUARD(xw + 4, 4) xw[4] = (uint32_t)batch;
             }
         }
         const long long head = unit / tiles;  // batch head (this step's inputs, o)
@@ -249,15 +256,18 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 #pragma unroll 4
                     for (int u = tid; u < ROWS * CPR; u += nthr) {
                         const int r = u / CPR, ch = u % CPR;
-                        cp_async16(raw + r * DK + ch * 16, src + (long long)r * DK + ch * 16);
+                        DL_GUARD(raw + r * DK + ch * 16, 16) cp_async16(raw + r * DK + ch * 16, src + (long long)r * DK + ch * 16);
                     }
-                    if (tid < ROWS / 4) cp_async16(scl + 4 * tid, i8_scales + shead * DV + row0 + 4 * tid);
+                    if (tid < ROWS / 4) {
+                        DL_GUARD(scl + 4 * tid, 16) cp_async16(scl + 4 * tid, i8_scales + shead * DV + row0 + 4 * tid);
+                    }
                 } else {
                     constexpr int CPR = DK / TL::CE;  // chunks per row
                     const ST *src = S + (shead * DV + row0) * DK;
 #pragma unroll 4
                     for (int u = tid; u < ROWS * CPR; u += nthr) {
                         const int r = u / CPR, ch = u % CPR;
+                        DL_GUARD(tile + TL::off(r, ch * TL::CE), 16)
                         cp_async16(tile + TL::off(r, ch * TL::CE), src + (long long)r * DK + ch * TL::CE);
                     }
                 }
@@ -331,7 +341,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                     auto put = [](float *dst, const float *x, bool real, float pad) {
 #pragma unroll
                         for (int e = 0; e < E; e += 4)
-                            *reinterpret_cast<float4 *>(dst + e) =
+                            DL_GUARD(dst + e, 16) *reinterpret_cast<float4 *>(dst + e) =
                                 real ? make_float4(x[e], x[e + 1], x[e + 2], x[e + 3])
                                      : make_float4(pad, pad, pad, pad);
                     };
@@ -349,14 +359,18 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                         if (c < NB * VC) put(sv + r * C::VS + col, vx[u], r < nb, 0.f);
                     }
                     if (tid < NB) {
-                        sb[tid] = bsc;  // 0 for padded entries
-                        if constexpr (!CHAN) fa[tid] = asc;
+                        DL_GUARD(sb + tid, 4) sb[tid] = bsc;  // 0 for padded entries
+                        if constexpr (!CHAN) {
+                            DL_GUARD(fa + tid, 4) fa[tid] = asc;
+                        }
                     }
                     if (qload) put(sq + tid * E, qx, true, 0.f);
 #pragma unroll
                     for (int u = 0; u < CN; ++u) {
                         const int idx = tid + u * nthr, ci = idx / NB, cj = idx % NB;
-                        if (idx < NB * NB && !(cur_here && ci == nl)) sx[ci * C::XS + cj] = cval[u];
+                        if (idx < NB * NB && !(cur_here && ci == nl)) {
+                            DL_GUARD(sx + ci * C::XS + cj, 4) sx[ci * C::XS + cj] = cval[u];
+                        }
                     }
                 };
                 if (bf) stage(bf16{});
@@ -378,15 +392,15 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
 #pragma unroll
                     for (int i = 0; i < NB; ++i) {
                         gm *= ac[i];
-                        kh[C::kof(i, c)] = gm * kc[i];
+                        DL_GUARD(kh + C::kof(i, c), 4) kh[C::kof(i, c)] = gm * kc[i];
                     }
-                    gn[c] = gm;
+                    DL_GUARD(gn + c, 4) gn[c] = gm;
                     __syncwarp();  // the warp's lanes have read their decays before F lands over them
                     const int fc = f_pos(c);
                     float f = 1.f;
 #pragma unroll
                     for (int j = NB - 1; j >= 0; --j) {
-                        ff[j * C::WS + fc] = kc[j] * f;
+                        DL_GUARD(ff + j * C::WS + fc, 4) ff[j * C::WS + fc] = kc[j] * f;
                         f *= ac[j];
                     }
                 }
@@ -407,7 +421,7 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                             const int u = tid + i * nthr, r = u / (DK / 4), c4 = (u % (DK / 4)) * 4;
                             const uint32_t w = wv[i];
                             const float sc = scl[r];
-                            *reinterpret_cast<float4 *>(tile + TL::off(r, c4)) =
+                            DL_GUARD(tile + TL::off(r, c4), 16) *reinterpret_cast<float4 *>(tile + TL::off(r, c4)) =
                                 make_float4((float)(int8_t)w * sc, (float)(int8_t)(w >> 8) * sc,
                                             (float)(int8_t)(w >> 16) * sc, (float)(int8_t)(w >> 24) * sc);
                         }
@@ -440,7 +454,10 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                         if (lane <= m && m < nl) acc = fmaf(cnm, sx[m * C::XS + lane], acc);
                     }
                     const float bn = sb[nl];
-                    if (lane < NB) sxw[warp * C::XS + lane] = lane < nl ? -bn * acc : (lane == nl ? bn : 0.f);
+                    if (lane < NB) {
+                        DL_GUARD(sxw + warp * C::XS + lane, 4)
+                        sxw[warp * C::XS + lane] = lane < nl ? -bn * acc : (lane == nl ? bn : 0.f);
+                    }
                     __syncwarp();
                 }
 
@@ -560,16 +577,16 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                         oacc[1] = fmaf(s1.x, qv.x, fmaf(s1.y, qv.y, fmaf(s1.z, qv.z, fmaf(s1.w, qv.w, oacc[1]))));
                     }
                     if constexpr (Q8) {
-                        st_tile4(p0, s0);
-                        st_tile4(p1, s1);
+                        DL_GUARD(p0, 4 * sizeof(TT)) st_tile4(p0, s0);
+                        DL_GUARD(p1, 4 * sizeof(TT)) st_tile4(p1, s1);
                         rmax0 = fmaxf(rmax0, fmaxf(fmaxf(fabsf(s0.x), fabsf(s0.y)), fmaxf(fabsf(s0.z), fabsf(s0.w))));
                         rmax1 = fmaxf(rmax1, fmaxf(fmaxf(fabsf(s1.x), fabsf(s1.y)), fmaxf(fabsf(s1.z), fabsf(s1.w))));
                     } else if (last) {
                         st_state4(Sw + g * DK + col, s0);
                         st_state4(Sw + (g + 8) * DK + col, s1);
                     } else {
-                        st_tile4(p0, s0);
-                        st_tile4(p1, s1);
+                        DL_GUARD(p0, 4 * sizeof(TT)) st_tile4(p0, s0);
+                        DL_GUARD(p1, 4 * sizeof(TT)) st_tile4(p1, s1);
                     }
                 }
                 if constexpr (Q8) {
@@ -580,8 +597,8 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                             rmax1 = fmaxf(rmax1, __shfl_xor_sync(0xffffffffu, rmax1, off));
                         }
                         if (t == 0) {
-                            wsc[warp * 16 + g] = i8_scale(rmax0);
-                            wsc[warp * 16 + g + 8] = i8_scale(rmax1);
+                            DL_GUARD(wsc + warp * 16 + g, 4) wsc[warp * 16 + g] = i8_scale(rmax0);
+                            DL_GUARD(wsc + warp * 16 + g + 8, 4) wsc[warp * 16 + g + 8] = i8_scale(rmax1);
                         }
                         __syncwarp();
                         constexpr int CPR = DK / 16;  // 16-code chunks per row
@@ -710,6 +727,11 @@ __global__ void pool_counts_kernel(const int *__restrict__ slot, int *__restrict
 cudaError_t launch_pool_counts(const PoolIdx &pool, int B, bool advance, cudaStream_t st) {
     pool_counts_kernel<<<(B + 127) / 128, 128, 0, st>>>(pool.slot, pool.counts, B, pool.P, pool.L, advance);
     return cudaGetLastError();
+}
+
+// The guard word of this file's kernels (index-guard build; 0 otherwise).
+cudaError_t read_guard_merge(unsigned int *flags, unsigned int *line, bool clear) {
+    return read_guard_word(flags, line, clear);
 }
 
 }  // namespace dl

@@ -49,6 +49,7 @@
 // Every wait on an mbarrier is bounded; a wait that runs out sets a bit of
 // the module's fault word and the CTA drains and returns.
 #include "launch.h"
+#include "guard.cuh"
 #include "merge_tc_layout.h"
 #include "tc.cuh"
 
@@ -324,12 +325,14 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     g *= ac[e];
                     if constexpr (DELTA) {
                         const float x = g * kc[e], hi = tc::tf32_trunc(x);
-                        *reinterpret_cast<float *>(kh + kh_off(e, c)) = hi;
-                        *reinterpret_cast<float *>(kh + kh_off(NB + e, c)) = x - hi;
+                        DL_GUARD(kh + kh_off(e, c), 4) *reinterpret_cast<float *>(kh + kh_off(e, c)) = hi;
+                        DL_GUARD(kh + kh_off(NB + e, c), 4) *reinterpret_cast<float *>(kh + kh_off(NB + e, c)) = x - hi;
                     }
                 }
-                gam[c] = g;
-                if constexpr (WITH_CUR) qf[c] = to_f(rq[raw_q_off(c, 1)]);
+                DL_GUARD(gam + c, 4) gam[c] = g;
+                if constexpr (WITH_CUR) {
+                    DL_GUARD(qf + c, 4) qf[c] = to_f(rq[raw_q_off(c, 1)]);
+                }
             }
             float fv[NB];  // F_e[c], into row c of F (this warp's quarter of F, which its last stores have read)
             {
@@ -350,7 +353,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                         const float x = fv[(4 * u + e) % NB], hi = tc::tf32_trunc(x);
                         wp[e] = u < 4 ? hi : x - hi;
                     }
-                    *reinterpret_cast<float4 *>(ff + ff_off(c, 4 * u)) = wv;
+                    DL_GUARD(ff + ff_off(c, 4 * u), 16) *reinterpret_cast<float4 *>(ff + ff_off(c, 4 * u)) = wv;
                 }
             }
             tc::fence_async_smem();       // Khat and F are read by the tensor cores
@@ -429,10 +432,11 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     p[NB + e] = fv[e] * qc;
                 }
                 multi_sum<2 * NB>(p, lane);  // lane l: this warp's sum of item l
-                red[quad * 2 * NB + lane] = p[0];
+                DL_GUARD(red + quad * 2 * NB + lane, 4) red[quad * 2 * NB + lane] = p[0];
                 tc::named_sync(bar_id, 128);
-                if (ct < 2 * NB)
-                    cn[ct] = red[ct] + red[2 * NB + ct] + red[4 * NB + ct] + red[6 * NB + ct];
+                if (ct < 2 * NB) {
+                    DL_GUARD(cn + ct, 4) cn[ct] = red[ct] + red[2 * NB + ct] + red[4 * NB + ct] + red[6 * NB + ct];
+                }
                 tc::named_sync(bar_id, 128);
                 if (DELTA && ct <= nl) {
                     // X(nl, ct) = -beta_nl sum_{m = ct..nl-1} C(nl, m) X(m, ct); X(nl, nl) = beta_nl
@@ -440,7 +444,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 #pragma unroll
                     for (int m = 0; m < NB; ++m)
                         if (m >= ct && m < nl) acc = fmaf(cn[m], scf(sc_x(m, ct)), acc);
-                    *reinterpret_cast<float *>(sc + sc_x(nl, ct)) = ct == nl ? bcur : -bcur * acc;
+                    DL_GUARD(sc + sc_x(nl, ct), 4) *reinterpret_cast<float *>(sc + sc_x(nl, ct)) = ct == nl ? bcur : -bcur * acc;
                 }
                 if constexpr (DELTA) tc::named_sync(bar_id, 128);
             }
@@ -521,7 +525,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<uint4 *>(buf + tile_off(lane, 4 * u)) =
+                    DL_GUARD(buf + tile_off(lane, 4 * u), 16) *reinterpret_cast<uint4 *>(buf + tile_off(lane, 4 * u)) =
                         make_uint4(d[4 * u + 0], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
                 tc::fence_async_smem();  // the staging tile is read by the TMA store
                 __syncwarp();
@@ -645,6 +649,11 @@ cudaError_t read_tc_faults(unsigned int *out, bool clear) {
         e = cudaMemcpyToSymbol(g_tc_faults, &zero, sizeof(unsigned int));
     }
     return e;
+}
+
+// The guard word of this file's kernels (index-guard build; 0 otherwise).
+cudaError_t read_guard_merge_tc(unsigned int *flags, unsigned int *line, bool clear) {
+    return read_guard_word(flags, line, clear);
 }
 
 }  // namespace dl

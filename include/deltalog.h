@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define DL_ABI_VERSION 8
+#define DL_ABI_VERSION 9
 #define DL_MAX_LOG 64
 
 typedef enum {
@@ -318,10 +318,21 @@ int dl_abi_version(void);
  * dl_log_merge_read) bound every such wait; a wait that runs out (about two
  * seconds; it means a bug, not a slow GPU) sets bit 0 here, abandons its work
  * (the state it was merging is then unspecified) and returns, so the device
- * stays usable. *flags receives the word; clear != 0 resets it to 0.
+ * stays usable. In the index-guard build (dl_index_guard_build() == 1), bit 1
+ * means that a kernel skipped a shared-memory write that lay outside its
+ * block's shared memory or was misaligned (a bug; that call's results are
+ * wrong); dl_last_error() then names the source file and line of the first
+ * one. *flags receives the word; clear != 0 resets it to 0.
  * Synchronous: it waits for the device's pending work (cudaMemcpyFromSymbol).
  * No counterpart on the pages: it is a health check of this library. */
 dl_status dl_device_faults(unsigned int *flags, int clear);
+
+/* 1 in the index-guard debug build (libdeltalog_guard.so, compiled with
+ * DL_INDEX_GUARD: every shared-memory write of the kernels checks its bounds
+ * and alignment first, and a write that fails is skipped and reported through
+ * dl_device_faults), else 0. The guard build computes the same results as the
+ * ordinary one, more slowly. No counterpart on the pages. */
+int dl_index_guard_build(void);
 
 #ifdef __cplusplus
 }

@@ -40,6 +40,23 @@ def test_exports_every_declared_symbol(lib):
     assert lib.dl_abi_version() == b.ABI_VERSION
 
 
+def test_index_guard_build_exports_the_same_abi(lib):
+    """The ordinary library says it is not the index-guard build; the guard
+    build (compiled here; nvcc needs no GPU) exports every declared symbol,
+    the same ABI version, and says it is."""
+    assert lib.dl_index_guard_build() == 0
+    from gated_delta_rule_104_b200 import build
+
+    path = build.build(guard=True)
+    g = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(g, name), name
+    g.dl_index_guard_build.restype = ctypes.c_int
+    g.dl_abi_version.restype = ctypes.c_int
+    assert g.dl_index_guard_build() == 1
+    assert g.dl_abi_version() == b.ABI_VERSION
+
+
 def test_status_strings(lib):
     assert b.dl_status_string(0) == "ok"
     assert "log full" in b.dl_status_string(3)
