@@ -100,7 +100,7 @@ def alg_bytes(w: W.Workload, kind: str, n: int) -> int:
     return per_head * w.heads
 
 
-KERNELS_PER_CALL = {"eager": 1, "append_read": 2, "merge_read": 1, "merge": 1, "pool": 4}
+KERNELS_PER_CALL = {"eager": 1, "append_read": 2, "merge_read": 1, "merge": 1, "pool": 4}  # see Launcher.kernels
 
 
 # ---------------------------------------------------------------- helpers
@@ -345,6 +345,15 @@ class Launcher:
         self.rwkv6 = w.decay == W.RWKV6
         self.L = log.L if log is not None else 0
 
+    def kernels(self, kind):
+        """Kernels one call of `kind` launches: the deferred read runs as one
+        kernel on an fp32 or bf16 base with L <= 16, else as two."""
+        import torch
+
+        if kind == "append_read":
+            return 1 if self.S.dtype in (torch.float32, torch.bfloat16) and self.L <= 16 else 2
+        return KERNELS_PER_CALL[kind]
+
     def plan(self):
         """(kind, n) of each launch of one decode, in order."""
         out, n = [], 0
@@ -496,7 +505,7 @@ def timed(launcher, steps, warmup, use_graph=True):
             per_kind.setdefault(kind, []).append((n, ev[i].elapsed_time(ev[i + 1])))
     del graph
     ms = reduce_max(total_ms / steps)
-    return ms, per_kind, steps * sum(KERNELS_PER_CALL[kind] for kind, _ in plan)
+    return ms, per_kind, steps * sum(launcher.kernels(kind) for kind, _ in plan)
 
 
 def roofline_for(w, per_kind, kind, peak, peak_note, traffic):

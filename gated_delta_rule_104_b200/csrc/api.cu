@@ -388,6 +388,9 @@ dl_status dl_device_faults(unsigned int *flags, int clear) {
     dl_status st = cuda_status(dl::read_tc_faults(&w, clear != 0), "fault word read");
     if (st != DL_OK) return st;
     *flags = w;
+    st = cuda_status(dl::read_read_faults(&w, clear != 0), "fault word read");
+    if (st != DL_OK) return st;
+    *flags |= w;
     struct {
         const char *file;
         cudaError_t (*read)(unsigned int *, unsigned int *, bool);

@@ -41,7 +41,9 @@
 //                 waits for the prep grid only before reading the workspace.
 #include "launch.h"
 #include "guard.cuh"
-#include "prep_layout.h"
+#include "prep.cuh"
+#include "fused_layout.h"
+#include "tc.cuh"
 
 namespace dl {
 
@@ -55,21 +57,10 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
                    float *__restrict__ log_x, int L, int n, float *__restrict__ work, long long heads,
                    PoolIdx pool) {
     pdl_launch_dependents();
-    constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
-    using P = PrepSmem<(int)sizeof(IT), DK, EMAX, CHAN>;
-    constexpr int CW = DK / 32;            // key columns per lane (contiguous)
-    constexpr int RV = DV / 32;            // value rows per lane
-    constexpr int CH = EMAX < 32 ? EMAX : 32;  // entries per butterfly
-    constexpr int E = 16 / (int)sizeof(IT);    // elements per 16-byte chunk
+    using P = PrepSmem<(int)sizeof(IT), DK, EMAX, Rule<KIND>::CHAN>;
     extern __shared__ float4 smem_raw[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5;
     unsigned char *base = reinterpret_cast<unsigned char *>(smem_raw) + (size_t)warp * P::BYTES;
-    IT *sk = reinterpret_cast<IT *>(base + P::K_OFF);
-    IT *sa = reinterpret_cast<IT *>(base + P::A_OFF);
-    float *fl = reinterpret_cast<float *>(base + P::F_OFF);
-    float *fas = fl + P::AS, *fbeta = fl + P::BETA, *fd = fl + P::D, *fcn = fl + P::CN, *fs = fl + P::S,
-          *xrow = fl + P::XROW;
-
     // A pool step launches this kernel as a programmatic dependent of its merge
     // part (which works on other slots), so the two overlap; every warp waits
     // for that grid before it exits, so that this grid's completion implies the
@@ -80,235 +71,8 @@ replay_prep_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         pdl_wait();
         return;
     }
-    const long long lrow = shead * L;
-    const int c0 = lane * CW, r0 = lane * RV;
-    // The log stays L2-resident between steps: its loads and stores carry an
-    // evict-last policy (the base streams through with evict-first); the
-    // cp.async staging copies carry none.
-    const uint64_t keep = l2_policy_keep();
-
-    // Stage keys and decays of entries 0..n-1 (log) and n (this step), raw.
-    for (int u = lane; u < (n + 1) * (DK / E); u += 32) {
-        const int e = u / (DK / E), col = (u % (DK / E)) * E;
-        if (e < n) {
-            DL_GUARD(sk + e * DK + col, 16) cp_async16(sk + e * DK + col, log_k + (lrow + e) * DK + col);
-            if constexpr (CHAN) {
-                DL_GUARD(sa + e * DK + col, 16) cp_async16(sa + e * DK + col, log_a + (lrow + e) * DK + col);
-            }
-        } else {
-            DL_GUARD(sk + e * DK + col, 16) cp_async16(sk + e * DK + col, k + head * DK + col);
-            if constexpr (CHAN) {
-                DL_GUARD(sa + e * DK + col, 16) cp_async16(sa + e * DK + col, a + head * DK + col);
-            }
-        }
-    }
-    cp_async_commit();
-    // Everything else the head needs is loaded next, all loads before the first
-    // store that consumes one (a warp issues in order: a store waiting on its
-    // load would hold back every load behind it).
-    constexpr int SB = (EMAX + 31) / 32;
-    RawCopy<1, IT> bx[SB], ax[SB];  // beta and a head-wise decay of entries lane, lane + 32 (<= n), raw
-#pragma unroll
-    for (int i = 0; i < SB; ++i) {
-        const int e = lane + 32 * i;
-        if (e <= n) {
-            if constexpr (DELTA) {
-                if (e < n) bx[i].load_hint(log_b + lrow + e, keep);
-                else bx[i].load(beta + head);
-            }
-            if constexpr (!CHAN) {
-                if (e < n) ax[i].load_hint(log_a + lrow + e, keep);
-                else ax[i].load(a + head);
-            }
-        }
-    }
-    // X rows of the logged entries (rows j < n, columns e <= j), XB per lane a batch.
-    constexpr int XB = 8;
-    float xx[XB];
-    auto x_load = [&](int base) {
-#pragma unroll
-        for (int i = 0; i < XB; ++i) {
-            const int u = base + i * 32 + lane, j = u / EMAX, e = u % EMAX;
-            xx[i] = 0.f;
-            if (DELTA && u < n * EMAX && e <= j) {
-                float t1[1];
-                load_vec_hint<1>(log_x + (lrow + j) * L + e, t1, keep);
-                xx[i] = t1[0];
-            }
-        }
-    };
-    auto x_store = [&](int base) {
-#pragma unroll
-        for (int i = 0; i < XB; ++i) {
-            const int u = base + i * 32 + lane, j = u / EMAX, e = u % EMAX;
-            if (DELTA && u < n * EMAX && e <= j) {
-                DL_GUARD(xrow + j * EMAX + e, 4) xrow[j * EMAX + e] = xx[i];
-            }
-        }
-    };
-    x_load(0);
-    // D1: the entry is appended unchanged (raw input elements).
-    RawCopy<CW, IT> ck, ca;
-    RawCopy<RV, IT> cv;
-    ck.load(k + head * DK + c0);
-    cv.load(v + head * DV + r0);
-    if constexpr (CHAN) ca.load(a + head * DK + c0);
-    float qv[CW];
-    load_vec<CW>(q + head * DK + c0, qv);
-    // the stores
-#pragma unroll
-    for (int i = 0; i < SB; ++i) {
-        const int e = lane + 32 * i;
-        if (e <= n) {
-            float t1[1];
-            if constexpr (DELTA) {
-                bx[i].widen(t1);
-                DL_GUARD(fbeta + e, 4) fbeta[e] = t1[0];
-            }
-            if constexpr (!CHAN) {
-                ax[i].widen(t1);
-                DL_GUARD(fas + e, 4) fas[e] = t1[0];
-            }
-        }
-    }
-    x_store(0);
-    for (int base = 32 * XB; DELTA && base < n * EMAX; base += 32 * XB) {  // longer logs only
-        x_load(base);
-        x_store(base);
-    }
-    ck.store(log_k + (lrow + n) * DK + c0, keep);
-    cv.store(log_v + (lrow + n) * DV + r0, keep);
-    if constexpr (CHAN) {
-        ca.store(log_a + (lrow + n) * DK + c0, keep);
-    } else if (lane == 0) {
-        copy_hint<1>(log_a + lrow + n, a + head, keep);
-    }
-    if (DELTA && lane == 0) copy_hint<1>(log_b + lrow + n, beta + head, keep);
-    cp_async_wait_all();
-    __syncwarp();
-
-    auto decay = [&](int e, float (&ae)[CW]) {
-        if constexpr (CHAN) {
-            load_vec<CW>(sa + e * DK + c0, ae);
-        } else {
-#pragma unroll
-            for (int c = 0; c < CW; ++c) ae[c] = fas[e];
-        }
-    };
-
-    // d_e = k_e . (D(n, e) o q) and C(n, e) = k_e . (D(n, e) o k_n), newest first.
-    float z[CW], y[CW];
-#pragma unroll
-    for (int c = 0; c < CW; ++c) z[c] = qv[c];
-    load_vec<CW>(sk + n * DK + c0, y);
-    for (int top = n; top >= 0; top -= CH) {
-        float pd[CH], pc[CH];
-#pragma unroll
-        for (int jj = 0; jj < CH; ++jj) {
-            pd[jj] = 0.f;
-            pc[jj] = 0.f;
-            const int e = top - jj;
-            if (e >= 0) {
-                float ke[CW], ae[CW];
-                load_vec<CW>(sk + e * DK + c0, ke);
-                decay(e, ae);
-#pragma unroll
-                for (int c = 0; c < CW; ++c) {
-                    pd[jj] = fmaf(ke[c], z[c], pd[jj]);
-                    z[c] *= ae[c];
-                    if constexpr (DELTA) {
-                        pc[jj] = fmaf(ke[c], y[c], pc[jj]);
-                        y[c] *= ae[c];
-                    }
-                }
-            }
-        }
-        multi_sum<CH>(pd, lane);
-        if constexpr (DELTA) multi_sum<CH>(pc, lane);
-        constexpr int shift = CH == 32 ? 0 : CH == 16 ? 1 : CH == 8 ? 2 : 3;
-        const int e = top - (lane >> shift);
-        if ((lane & ((1 << shift) - 1)) == 0 && e >= 0) {
-            DL_GUARD(fd + e, 4) fd[e] = pd[0];
-            DL_GUARD(fcn + e, 4) fcn[e] = pc[0];  // (C(n, n) is not used)
-        }
-    }
-    __syncwarp();
-    // X row n: X(n, n) = beta_n, X(n, j) = -beta_n sum_{m=j..n-1} C(n, m) X(m, j).
-    const float bn = DELTA ? fbeta[n] : 0.f;
-    for (int j = lane; DELTA && j <= n; j += 32) {
-        float acc = 0.f;
-#pragma unroll 4
-        for (int m = j; m < n; ++m) acc = fmaf(fcn[m], xrow[m * EMAX + j], acc);
-        const float xnj = j == n ? bn : -bn * acc;
-        DL_GUARD(xrow + n * EMAX + j, 4) xrow[n * EMAX + j] = xnj;
-        st_hint(log_x + (lrow + n) * L + j, __float_as_uint(xnj), keep);
-    }
-    __syncwarp();
-    // s_e = sum_{i=e..n} X(i, e) d_i (the back-substitution, as one dot per entry).
-    for (int e = lane; e <= n; e += 32) {
-        float acc = 0.f;
-        if constexpr (DELTA) {
-#pragma unroll 4
-            for (int i = e; i <= n; ++i) acc = fmaf(xrow[i * EMAX + e], fd[i], acc);
-        } else {
-            acc = fd[e];
-        }
-        DL_GUARD(fs + e, 4) fs[e] = acc;
-    }
-    __syncwarp();
-
-    // x_0 = gamma_n o q - sum_e s_e (gamma_e o k_e);  w = sum_e s_e v_e.
-    float g[CW], xs[CW];
-#pragma unroll
-    for (int c = 0; c < CW; ++c) {
-        g[c] = 1.f;
-        xs[c] = 0.f;
-    }
-#pragma unroll 4
-    for (int e = 0; e <= n; ++e) {
-        float ke[CW], ae[CW];
-        load_vec<CW>(sk + e * DK + c0, ke);
-        decay(e, ae);
-        const float se = fs[e];
-#pragma unroll
-        for (int c = 0; c < CW; ++c) {
-            g[c] *= ae[c];
-            if constexpr (DELTA) xs[c] = fmaf(se * g[c], ke[c], xs[c]);
-        }
-    }
-    float w[RV];
-#pragma unroll
-    for (int r = 0; r < RV; ++r) w[r] = 0.f;
-    // Entries in batches of VB: a batch's raw words are all loaded before any is
-    // widened (a widening right after its load would stall the loads behind it).
-    constexpr int VB = 8;
-    using VC = RawCopy<RV, IT>;
-    for (int e0 = 0; e0 <= n; e0 += VB) {
-        VC raw[VB];
-#pragma unroll
-        for (int i = 0; i < VB; ++i) {
-            const int e = e0 + i;
-            if (e < n) raw[i].load_hint(log_v + (lrow + e) * DV + r0, keep);
-            else if (e == n) raw[i].load(v + head * DV + r0);
-        }
-#pragma unroll
-        for (int i = 0; i < VB; ++i) {
-            const int e = e0 + i;
-            if (e <= n) {
-                const float se = fs[e];
-                float ve[RV];
-                raw[i].widen(ve);
-#pragma unroll
-                for (int r = 0; r < RV; ++r) w[r] = fmaf(se, ve[r], w[r]);
-            }
-        }
-    }
-
-    float *wk = work + head * (DK + DV);
-#pragma unroll
-    for (int c = 0; c < CW; ++c) wk[c0 + c] = fmaf(g[c], qv[c], -xs[c]);
-#pragma unroll
-    for (int r = 0; r < RV; ++r) wk[DK + r0 + r] = w[r];
+    prep_head<IT, DK, DV, KIND, EMAX, false>(q, k, v, beta, a, log_k, log_v, log_b, log_a, log_x, L, n, head, shead,
+                                             base, work + head * (DK + DV));
     pdl_wait();
 }
 
@@ -376,6 +140,206 @@ append_decode_kernel(const ST *__restrict__ Sbar, const float *__restrict__ work
     }
 }
 
+// ------------------------------------------------------------------ fused append-read
+//
+// The same step in one persistent kernel (one block per SM; layout and roles
+// in fused_layout.h), so that ReplayPrep runs under the base stream instead
+// of ahead of it: prep warps work through the block's heads a few heads ahead
+// of the decode warps and hand each head's (x_0, w) over in shared memory;
+// decode warps keep NBUF bulk copies of the base in flight per warp and form
+// o exactly as append_decode does (the same products and sums in the same
+// order, so the two paths agree bit for bit). Used for logs of up to 16
+// entries on an fp32 or bf16 base without a slot pool; no workspace.
+// Every mbarrier wait is bounded (about two seconds); a wait that runs out
+// sets bit 0 of g_read_faults and the block leaves its loops, waits for the
+// copies it has in flight, and returns.
+
+__device__ unsigned int g_read_faults = 0;
+
+namespace {
+
+__device__ __forceinline__ uint64_t read_globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for the phase of `bar` with parity `par`; false once about two seconds
+// have passed (setting *abort and the fault bit) or another warp gave up.
+__device__ __forceinline__ bool fused_wait(uint64_t *bar, uint32_t par, volatile int *abort) {
+    if (tc::mbar_try_wait(bar, par)) return true;
+    const uint64_t t0 = read_globaltimer();
+    for (uint32_t i = 0;; ++i) {
+        if (tc::mbar_try_wait(bar, par)) return true;
+        if ((i & 63u) == 63u) {
+            if (*abort) return false;
+            if (read_globaltimer() - t0 > 2000000000ull) {
+                *abort = 1;
+                atomicOr(&g_read_faults, 1u);
+                return false;
+            }
+        }
+    }
+}
+// The same without the abort check: for draining a warp's own copies.
+__device__ __forceinline__ void fused_drain(uint64_t *bar, uint32_t par) {
+    const uint64_t t0 = read_globaltimer();
+    while (!tc::mbar_try_wait(bar, par)) {
+        if (read_globaltimer() - t0 > 2000000000ull) {
+            atomicOr(&g_read_faults, 1u);
+            return;
+        }
+    }
+}
+
+}  // namespace
+
+template <class IT, class ST, int DK, int DV, int KIND>
+__global__ void __launch_bounds__(fused::Layout<(int)sizeof(IT), (int)sizeof(ST), DK, DV, Rule<KIND>::CHAN>::WARPS * 32, 1)
+append_read_fused_kernel(const ST *__restrict__ Sbar, const IT *__restrict__ q, const IT *__restrict__ k,
+                         const IT *__restrict__ v, const IT *__restrict__ beta, const IT *__restrict__ a,
+                         IT *__restrict__ log_k, IT *__restrict__ log_v, IT *__restrict__ log_b,
+                         IT *__restrict__ log_a, float *__restrict__ log_x, int L, int n, float *__restrict__ o,
+                         long long heads) {
+    using LY = fused::Layout<(int)sizeof(IT), (int)sizeof(ST), DK, DV, Rule<KIND>::CHAN>;
+    using C = DecodeShape<ST, DK>;
+    constexpr int VEC = C::VEC, NP = LY::NP, ND = fused::ND, NBUF = fused::NBUF, NSLOT = LY::NSLOT,
+                  UPH = LY::UPH;
+    static_assert(C::UNIT == LY::UNIT_ROWS, "a bulk copy holds one decode unit");
+    static_assert(DV % LY::UNIT_ROWS == 0, "units tile a head");
+    extern __shared__ float4 smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + LY::BAR_FULL);
+    uint64_t *freeb = reinterpret_cast<uint64_t *>(sm + LY::BAR_FREE);
+    uint64_t *ringb = reinterpret_cast<uint64_t *>(sm + LY::BAR_RING);
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + LY::ABORT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nh = heads > (long long)blockIdx.x ? (int)((heads - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+
+    // Launched as a programmatic dependent of the kernel before it: the block
+    // sets up its barriers while that kernel drains, and touches no global
+    // memory before the wait (the base, the log and the inputs may all be
+    // that kernel's output). The kernel after it may likewise start early.
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSLOT; ++s) {
+            tc::mbar_init(&full[s], 32);     // the prep warp's 32 lanes
+            tc::mbar_init(&freeb[s], UPH);   // one arrival per decode unit of the head
+        }
+        for (int u = 0; u < ND * NBUF; ++u) tc::mbar_init(&ringb[u], 1);
+        *abort = 0;
+        tc::mbar_init_fence();
+    }
+    __syncthreads();
+    pdl_wait();
+
+    if (warp < NP) {
+        // ------------------------------------------------ ReplayPrep, heads warp, warp + NP, ...
+        unsigned char *base = sm + LY::prep(warp);
+        for (int i = warp; i < nh; i += NP) {
+            const int s = i % NSLOT;
+            if (i >= NSLOT && !fused_wait(&freeb[s], (uint32_t)((i / NSLOT - 1) & 1), abort)) break;
+            const long long head = (long long)blockIdx.x + (long long)i * gridDim.x;
+            prep_head<IT, DK, DV, KIND, fused::EMAX, true>(q, k, v, beta, a, log_k, log_v, log_b, log_a, log_x, L,
+                                                             n, head, head, base,
+                                                             reinterpret_cast<float *>(sm + LY::slot(s)));
+            tc::mbar_arrive(&full[s]);  // each lane after its own stores of x_0 and w
+        }
+    } else {
+        // ------------------------------------------------ AppendDecode, units d, d + ND, ... of the block's heads
+        const int d = warp - NP;
+        const int nf = nh * UPH;
+        const int sub = lane / C::G, col = (lane % C::G) * VEC;
+        // (a buffer is refilled only after every lane's reads of it have
+        // returned their values, which the unit's sums consumed)
+        auto issue = [&](int f, int b) {
+            if (lane == 0) {
+                const long long head = (long long)blockIdx.x + (long long)(f / UPH) * gridDim.x;
+                uint64_t *bar = &ringb[d * NBUF + b];
+                tc::mbar_arrive_expect_tx(bar, fused::UNIT_BYTES);
+                tc::bulk_load(sm + LY::ring(d, b), Sbar + (head * DV + (long long)(f % UPH) * LY::UNIT_ROWS) * DK,
+                              fused::UNIT_BYTES, bar);
+            }
+        };
+        int issued = 0;
+        for (int b = 0; b < NBUF && d + b * ND < nf; ++b, ++issued) issue(d + b * ND, b);
+        int t = 0;
+        for (;; ++t) {
+            const int f = d + t * ND;
+            if (f >= nf) break;
+            const int b = t % NBUF, i = f / UPH, j = f % UPH, s = i % NSLOT;
+            if (!fused_wait(&ringb[d * NBUF + b], (uint32_t)((t / NBUF) & 1), abort)) break;
+            if (!fused_wait(&full[s], (uint32_t)((i / NSLOT) & 1), abort)) break;
+            const long long head = (long long)blockIdx.x + (long long)i * gridDim.x;
+            const ST *tile = reinterpret_cast<const ST *>(sm + LY::ring(d, b));
+            const float *sl = reinterpret_cast<const float *>(sm + LY::slot(s));
+            float xv[VEC], res[C::R];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) xv[e] = sl[col + e];
+            const bool writer = (lane % C::G) == 0;
+#pragma unroll
+            for (int r = 0; r < C::R; ++r) {
+                const int ru = r * C::RPW + sub;  // row within the unit
+                float sv[VEC];
+                StateVec<ST>::unpack(*reinterpret_cast<const uint4 *>(tile + ru * DK + col), sv);
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc = fmaf(sv[e], xv[e], acc);
+                acc = group_sum<C::G>(acc);
+                res[r] = writer ? acc + sl[DK + j * LY::UNIT_ROWS + ru] : 0.f;
+            }
+            // the unit reads nothing more of slot s or of buffer b: hand the
+            // slot back and refill the buffer before the unit's stores, so that
+            // neither waits behind them
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&freeb[s]);
+            if (f + NBUF * ND < nf) {
+                issue(f + NBUF * ND, b);
+                ++issued;
+            }
+#pragma unroll
+            for (int r = 0; r < C::R; ++r)
+                if (writer) o[head * DV + j * LY::UNIT_ROWS + r * C::RPW + sub] = res[r];
+        }
+        // after a wait gave up: the copies this warp still has in flight land
+        // before the block exits
+        if (lane == 0)
+            for (int u = t; u < issued; ++u) fused_drain(&ringb[d * NBUF + u % NBUF], (uint32_t)((u / NBUF) & 1));
+        __syncwarp();
+    }
+}
+
+template <class IT, class ST, int DK, int DV, int KD>
+static cudaError_t launch_fused(const StepParams &p, const LogParams &lg, int n, cudaStream_t st) {
+    using LY = fused::Layout<(int)sizeof(IT), (int)sizeof(ST), DK, DV, Rule<KD>::CHAN>;
+    static_assert(LY::REQUEST <= fused::SMEM_LIMIT, "layout fits the shared memory a block may request");
+    static_assert(LY::NP >= 1, "at least one prep warp");
+    auto kern = append_read_fused_kernel<IT, ST, DK, DV, KD>;
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), LY::REQUEST);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long heads = (long long)p.B * p.H;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<long long>(heads, sms));
+    cfg.blockDim = dim3(LY::WARPS * 32);
+    cfg.dynamicSmemBytes = LY::REQUEST;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const ST *>(p.S), static_cast<const IT *>(p.q),
+                           static_cast<const IT *>(p.k), static_cast<const IT *>(p.v),
+                           static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), static_cast<IT *>(lg.k),
+                           static_cast<IT *>(lg.v), static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.x, lg.L,
+                           n, p.o, heads);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 size_t read_work_bytes(int B, int H, int dk, int dv) { return (size_t)B * H * (dk + dv) * sizeof(float); }
 
 template <class ST, int DK, int DV>
@@ -429,8 +393,9 @@ static cudaError_t launch_prep(const StepParams &p, const LogParams &lg, int n, 
                               static_cast<IT *>(lg.beta), static_cast<IT *>(lg.a), lg.x, lg.L, n, work, heads, pool);
 }
 
-cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
-                               const PoolIdx &pool) {
+// The two-kernel form (replay_prep, then append_decode with the workspace).
+static cudaError_t launch_append_read_split(const StepParams &p, const LogParams &lg, int n, float *work,
+                                           cudaStream_t st, const PoolIdx &pool) {
     return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
         using ST = decltype(st_t);
         using IT = decltype(it_t);
@@ -450,9 +415,25 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
     });
 }
 
+bool fused_read_supported(const StepParams &p, int L, const PoolIdx &pool) {
+    return pool.slot == nullptr && (p.s_dt == DL_F32 || p.s_dt == DL_BF16) && prep_emax(L) == fused::EMAX;
+}
+
+cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
+                               const PoolIdx &pool) {
+    if (!fused_read_supported(p, lg.L, pool)) return launch_append_read_split(p, lg, n, work, st, pool);
+    return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
+        using ST = decltype(st_t);
+        using IT = decltype(it_t);
+        return launch_fused<IT, ST, decltype(dk_c)::value, decltype(dv_c)::value, decltype(ch_c)::value>(p, lg, n,
+                                                                                                         st);
+    });
+}
+
 // ------------------------------------------------------------------ no-allocation variant
 //
-// dl_log_append_read_noalloc runs the same two kernels with their scratch in
+// dl_log_append_read_noalloc runs the two-kernel form of the step
+// (replay_prep, then append_decode) for every shape, with its scratch in
 // this fixed module-level array instead of a caller-provided workspace, for
 // callers that cannot allocate device memory. The array belongs to the CUDA
 // module of this file, so every device that loads the library holds it until
@@ -483,7 +464,16 @@ cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg,
     float *work = nullptr;
     cudaError_t e = noalloc_work_address(&work);
     if (e != cudaSuccess) return e;
-    return launch_append_read(p, lg, n, work, st);
+    return launch_append_read_split(p, lg, n, work, st, PoolIdx{});
+}
+
+cudaError_t read_read_faults(unsigned int *out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_read_faults, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_read_faults, &zero, sizeof(unsigned int));
+    }
+    return e;
 }
 
 // The guard word of this file's kernels (index-guard build; 0 otherwise).

@@ -89,7 +89,10 @@ inline cudaError_t allow_smem(const void *kern, size_t bytes) {
 }
 
 cudaError_t launch_eager(const StepParams &p, cudaStream_t st);
-// Deferred read: needs read_work_bytes() of fp32 workspace (x_0 and w per head).
+// Deferred read. The fused one-kernel form (fused_read_supported: an fp32 or
+// bf16 base, logs of up to 16 entries, no slot pool) needs no workspace; the
+// two-kernel form takes read_work_bytes() of fp32 workspace (x_0 and w per head).
+bool fused_read_supported(const StepParams &p, int L, const PoolIdx &pool);
 cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
                                const PoolIdx &pool = PoolIdx{});
 size_t read_work_bytes(int B, int H, int dk, int dv);
@@ -107,6 +110,8 @@ cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log,
 // The tensor-core kernels' fault word (bit 0: a bounded wait ran out), read
 // synchronously; cleared afterwards when `clear`.
 cudaError_t read_tc_faults(unsigned int *out, bool clear);
+// The same for the fused append-read kernel (deferred_read.cu).
+cudaError_t read_read_faults(unsigned int *out, bool clear);
 // index-guard words of the kernels' files (bit 1: a shared-memory write out of
 // bounds was skipped; line: the source line of the first); 0 in the ordinary build
 cudaError_t read_guard_merge(unsigned int *flags, unsigned int *line, bool clear);

@@ -177,7 +177,12 @@ size_t dl_log_work_bytes(int B, int H, int d_k, int d_v);
  *          (missing or smaller than dl_log_work_bytes -> DL_ERR_INVALID_ARG)
  *   n      entries already in the log, 0 <= n < L; n >= L -> DL_ERR_LOG_FULL
  *   q, k, v, beta, a, o: as the eager step of the same kind (DL_RWKV6: beta
- *          is not used and may be null). */
+ *          is not used and may be null).
+ * With an fp32 or bf16 base and L <= 16 the step runs as one persistent
+ * kernel (the key-side work of each head done in shared memory a few heads
+ * ahead of the base stream) and log->work is checked but not used; otherwise
+ * (an int8 base, L > 16) as two kernels that hand the key-side results over
+ * in log->work. Both forms give the same results, bit for bit. */
 dl_status dl_log_append_read(const void *S_base, dl_dtype s_dtype, dl_decay kind,
                              const dl_log *log, int n,
                              const void *q, const void *k, const void *v,
@@ -213,7 +218,8 @@ dl_status dl_log_merge_read(void *S_base, dl_dtype s_dtype, dl_decay kind,
  * plugin host that hands a kernel only its input and output buffers, or a
  * latency-critical decode loop where a cudaMalloc would synchronise the
  * device. It computes exactly what dl_log_append_read computes, with the same
- * arguments and checks, except that log->work is ignored (it may be null):
+ * arguments and checks, always in the two-kernel form of that step, except
+ * that log->work is ignored (it may be null):
  * the per-head scratch lives in a fixed array of DL_NOALLOC_WORK_BYTES inside
  * the library, which every device that loads the library keeps until the
  * process exits.
@@ -315,7 +321,8 @@ int dl_abi_version(void);
 
 /* Fault word of the library's kernels on the current device. The kernels that
  * wait on on-chip barriers (the tcgen05 merge of dl_log_merge and
- * dl_log_merge_read) bound every such wait; a wait that runs out (about two
+ * dl_log_merge_read, and the one-kernel form of dl_log_append_read) bound
+ * every such wait; a wait that runs out (about two
  * seconds; it means a bug, not a slow GPU) sets bit 0 here, abandons its work
  * (the state it was merging is then unspecified) and returns, so the device
  * stays usable. In the index-guard build (dl_index_guard_build() == 1), bit 1

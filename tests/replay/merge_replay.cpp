@@ -1,16 +1,17 @@
 // Host replay of the shared-memory addresses (and the log's global rows)
 // that the warp-MMA merge kernel (gated_delta_rule_104_b200/csrc/merge.cu,
-// its compact pool walk included) and the replay-prep kernel
-// (gated_delta_rule_104_b200/csrc/deferred_read.cu) form, for every
-// instantiation and every log fill they accept. The region offsets and the
-// swizzles come from the kernels' own layout headers (merge_layout.h,
-// prep_layout.h); the loops are the kernels' loops with their bounds. Each
+// its compact pool walk included), the replay-prep kernel and the fused
+// append-read kernel (gated_delta_rule_104_b200/csrc/deferred_read.cu, the
+// latter's ReplayPrep from prep.cuh) form, for every instantiation and every
+// log fill they accept. The region offsets and the swizzles come from the
+// kernels' own layout headers (merge_layout.h, prep_layout.h,
+// fused_layout.h); the loops are the kernels' loops with their bounds. Each
 // access is checked to lie inside its region and to be aligned for its
 // width; the regions must not overlap and must fit the dynamic shared memory
 // the launch requests.
 //
-// Usage: merge_replay [merge | prep] [shrink <region> <bytes>]...
-//   merge, prep: replay only that kernel.
+// Usage: merge_replay [merge | prep | fused] [shrink <region> <bytes>]...
+//   merge, prep, fused: replay only that kernel.
 //   shrink: the bounds table believes <region> is <bytes> shorter than the
 //   layout says (a planted overrun: the replay must then fail; it stops at
 //   the first failure).
@@ -25,6 +26,7 @@
 
 #include "merge_layout.h"
 #include "prep_layout.h"
+#include "fused_layout.h"
 
 using namespace dl;
 
@@ -322,14 +324,14 @@ int merge_cases() {
 template <int IB, int DK, int DV, int EMAX, bool CHAN>
 struct PrepReplay {
     using P = PrepSmem<IB, DK, EMAX, CHAN>;
-    static constexpr int WARPS = prep_warps(EMAX), CW = DK / 32, E = 16 / IB, CH = EMAX < 32 ? EMAX : 32,
-                         SBN = (EMAX + 31) / 32, XB = 8;
+    static constexpr int CW = DK / 32, E = 16 / IB, CH = EMAX < 32 ? EMAX : 32, SBN = (EMAX + 31) / 32, XB = 8;
     bool delta;
+    int WARPS;  // staging areas laid out from offset 0: the prep kernel's warps, or the fused kernel's prep warps
     Table t;
-    PrepReplay(bool de) : delta(de) {
+    PrepReplay(bool de, int warps = prep_warps(EMAX), const char *kernel = "prep") : delta(de), WARPS(warps) {
         char b[96];
-        std::snprintf(b, sizeof b, "prep in%d dk%d dv%d emax%d %s %s", IB, DK, DV, EMAX, CHAN ? "chan" : "head",
-                      de ? "delta" : "rwkv6");
+        std::snprintf(b, sizeof b, "%s in%d dk%d dv%d emax%d %s %s", kernel, IB, DK, DV, EMAX,
+                      CHAN ? "chan" : "head", de ? "delta" : "rwkv6");
         t.tag = b;
         for (int w = 0; w < WARPS; ++w) {
             const std::string p = "w" + std::to_string(w) + ".";
@@ -453,18 +455,124 @@ int prep_all() {
            prep_cases<IB, DK, DV, 64, false>() + prep_cases<IB, DK, DV, 64, true>();
 }
 
+// ---------------------------------------------------------------- fused append-read (deferred_read.cu)
+
+template <int IB, int SB, int DK, int DV, bool CHAN>
+struct FusedReplay {
+    using LY = fused::Layout<IB, SB, DK, DV, CHAN>;
+    static constexpr int VEC = 16 / SB, G = DK / VEC, RPW = 32 / G, R = 8, CW = DK / 32, RV = DV / 32;
+    PrepReplay<IB, DK, DV, fused::EMAX, CHAN> rp;
+    FusedReplay(bool de) : rp(de, LY::NP, "fused") {
+        Table &t = rp.t;
+        for (int s = 0; s < LY::NSLOT; ++s) t.add("slot" + std::to_string(s), LY::slot(s), LY::SLOT_BYTES);
+        for (int d = 0; d < fused::ND; ++d)
+            for (int b = 0; b < fused::NBUF; ++b)
+                t.add("ring" + std::to_string(d) + "." + std::to_string(b), LY::ring(d, b), fused::UNIT_BYTES);
+        t.add("full", LY::BAR_FULL, 8 * LY::NSLOT);
+        t.add("free", LY::BAR_FREE, 8 * LY::NSLOT);
+        t.add("ringbar", LY::BAR_RING, 8 * fused::ND * fused::NBUF);
+        t.add("abort", LY::ABORT_OFF, 4);
+    }
+    void layout() {
+        Table &t = rp.t;
+        if (LY::UNIT_ROWS != R * RPW) fail("a bulk copy is not one decode unit", t.tag);
+        if (DV % LY::UNIT_ROWS) fail("units do not tile a head", t.tag);
+        if (LY::NP < 1 || LY::NSLOT % LY::NP) fail("each slot must belong to one prep warp", t.tag);
+        if ((size_t)LY::REQUEST > SMEM_LIMIT) fail("fused request above 227 KiB", t.tag);
+        if (LY::BYTES + 127 > LY::REQUEST) fail("no room to align the base to 128 bytes", t.tag);
+        if (LY::RING_OFF % 16 || fused::UNIT_BYTES % 16) fail("bulk-copy buffers not 16-byte aligned", t.tag);
+        if (LY::BAR_OFF % 8) fail("mbarriers not 8-byte aligned", t.tag);
+        t.no_overlap(LY::BYTES);
+    }
+    // the decode side, the same at every fill: (x_0, w) stored into each slot
+    // and read back by a decode unit, and every buffer read as a unit's tile
+    void decode() {
+        Table &t = rp.t;
+        for (int s = 0; s < LY::NSLOT; ++s) {
+            const std::string sl = "slot" + std::to_string(s);
+            for (int lane = 0; lane < 32; ++lane) {
+                for (int c = 0; c < CW; ++c) t.acc(sl, (long)(lane * CW + c) * 4, 4, 4, "x_0 store");
+                for (int r = 0; r < RV; ++r) t.acc(sl, (long)(DK + lane * RV + r) * 4, 4, 4, "w store");
+                const int sub = lane / G, col = (lane % G) * VEC;
+                for (int e = 0; e < VEC; ++e) t.acc(sl, (long)(col + e) * 4, 4, 4, "x_0 read");
+                for (int j = 0; j < LY::UPH; ++j)
+                    for (int r = 0; r < R; ++r)
+                        t.acc(sl, (long)(DK + j * LY::UNIT_ROWS + r * RPW + sub) * 4, 4, 4, "w read");
+            }
+        }
+        for (int d = 0; d < fused::ND; ++d)
+            for (int b = 0; b < fused::NBUF; ++b) {
+                const std::string rg = "ring" + std::to_string(d) + "." + std::to_string(b);
+                for (int lane = 0; lane < 32; ++lane) {
+                    const int sub = lane / G, col = (lane % G) * VEC;
+                    for (int r = 0; r < R; ++r) t.acc(rg, ((long)(r * RPW + sub) * DK + col) * SB, 16, 16, "base slice");
+                }
+            }
+    }
+    // one fill n: ReplayPrep of every prep warp, and the base copies of
+    // `heads` heads checked against the base's extent
+    void run(int n, int L, long long heads) {
+        Table &t = rp.t;
+        rp.run(n, L);
+        // bulk-copy sources: every unit of every head inside the base, 16-byte aligned
+        const unsigned long long total = (unsigned long long)heads * DV * DK * SB;
+        for (long long h = 0; h < heads; ++h)
+            for (int j = 0; j < LY::UPH; ++j) {
+                const unsigned long long off = ((unsigned long long)h * DV + (unsigned long long)j * LY::UNIT_ROWS) * DK * SB;
+                if (off + fused::UNIT_BYTES > total || off % 16) fail("base copy outside the base", t.tag);
+            }
+        if (shrink.count("unit")) {  // a base believed one row shorter per head
+            const unsigned long long short_total = total - (unsigned long long)heads * DK * SB;
+            const unsigned long long last = ((unsigned long long)(heads - 1) * DV + (DV - LY::UNIT_ROWS)) * DK * SB;
+            if (last + fused::UNIT_BYTES > short_total) fail("out of region", t.tag + " base copy");
+        }
+    }
+};
+
+template <int IB, int SB, int DK, int DV, bool CHAN>
+int fused_cases() {
+    int cases = 0;
+    for (int delta = 0; delta < 2; ++delta) {
+        if (!delta && !CHAN) continue;
+        FusedReplay<IB, SB, DK, DV, CHAN> fr(delta);
+        fr.layout();
+        fr.decode();
+        for (int L : {1, 2, 5, 15, 16}) {
+            for (int n = 0; n < L; ++n) {
+                fr.run(n, L, 3 + 7 * n);
+                ++cases;
+            }
+        }
+    }
+    return cases;
+}
+
+template <int IB, int SB>
+int fused_all() {
+    int c = 0;
+    c += fused_cases<IB, SB, 64, 64, false>() + fused_cases<IB, SB, 64, 64, true>();
+    c += fused_cases<IB, SB, 64, 128, false>() + fused_cases<IB, SB, 64, 128, true>();
+    c += fused_cases<IB, SB, 64, 256, false>() + fused_cases<IB, SB, 64, 256, true>();
+    c += fused_cases<IB, SB, 128, 64, false>() + fused_cases<IB, SB, 128, 64, true>();
+    c += fused_cases<IB, SB, 128, 128, false>() + fused_cases<IB, SB, 128, 128, true>();
+    c += fused_cases<IB, SB, 128, 256, false>() + fused_cases<IB, SB, 128, 256, true>();
+    return c;
+}
+
 }  // namespace
 
 int main(int argc, char **argv) {
-    bool do_merge = true, do_prep = true;
+    bool do_merge = true, do_prep = true, do_fused = true;
     for (int i = 1; i < argc; ++i) {
         if (std::strcmp(argv[i], "shrink") == 0 && i + 2 < argc) {
             shrink[argv[i + 1]] = std::atol(argv[i + 2]);
             i += 2;
         } else if (std::strcmp(argv[i], "merge") == 0) {
-            do_prep = false;
+            do_prep = do_fused = false;
         } else if (std::strcmp(argv[i], "prep") == 0) {
-            do_merge = false;
+            do_merge = do_fused = false;
+        } else if (std::strcmp(argv[i], "fused") == 0) {
+            do_merge = do_prep = false;
         }
     }
     int cases = 0;
@@ -482,6 +590,8 @@ int main(int argc, char **argv) {
         cases += prep_all<2, 64, 64>() + prep_all<2, 128, 128>() + prep_all<2, 128, 256>();
         cases += prep_all<4, 64, 64>() + prep_all<4, 128, 128>() + prep_all<4, 128, 256>();
     }
+    // fused append-read: bf16 and fp32 inputs, fp32 and bf16 bases, every d_k x d_v
+    if (do_fused) cases += fused_all<2, 4>() + fused_all<2, 2>() + fused_all<4, 4>() + fused_all<4, 2>();
     std::printf("%d cases, %d failures\n", cases, failures);
     return failures ? 1 : 0;
 }

@@ -1,8 +1,10 @@
-"""CPU replay of the warp-MMA merge's and the replay-prep kernel's addresses (no GPU).
+"""CPU replay of the addresses of the warp-MMA merge, the replay-prep kernel
+and the fused append-read kernel (no GPU).
 
 tests/replay/merge_replay.cpp walks the loops of merge.cu (the compact pool
-walk included) and of replay_prep in deferred_read.cu with the layout
-functions the kernels themselves use (merge_layout.h, prep_layout.h), for
+walk included), of replay_prep and of append_read_fused in deferred_read.cu
+(ReplayPrep from prep.cuh) with the layout functions the kernels themselves
+use (merge_layout.h, prep_layout.h, fused_layout.h), for
 every instantiation and a grid of log fills, and checks every shared-memory
 access for bounds and alignment, that the regions do not overlap and fit the
 shared memory the launch requests, and that the swizzles are one-to-one. A
@@ -54,5 +56,17 @@ PLANTS = [("xw", 16), ("tile", 4), ("kh", 4), ("ff", 36), ("fa", 4), ("gn", 4), 
 @pytest.mark.parametrize("region,nbytes", PLANTS)
 def test_a_planted_overrun_is_caught(replay, region, nbytes):
     r = run(replay, "prep" if "." in region else "merge", "shrink", region, str(nbytes))
+    assert r.returncode == 1, r.stdout[-2000:]
+    assert "out of region" in r.stdout
+
+
+# the fused kernel: the last float of a slot (w's last row), the last 16 bytes
+# of a base buffer, a prep warp's X rows, and a base one row short per head
+FUSED_PLANTS = [("slot3", 4), ("ring7.2", 4), ("w5.xrow", 4), ("w0.sk", 4), ("unit", 0)]
+
+
+@pytest.mark.parametrize("region,nbytes", FUSED_PLANTS)
+def test_a_planted_overrun_in_the_fused_read_is_caught(replay, region, nbytes):
+    r = run(replay, "fused", "shrink", region, str(nbytes))
     assert r.returncode == 1, r.stdout[-2000:]
     assert "out of region" in r.stdout
