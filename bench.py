@@ -347,11 +347,15 @@ class Launcher:
 
     def kernels(self, kind):
         """Kernels one call of `kind` launches: the deferred read runs as one
-        kernel on an fp32 or bf16 base with L <= 16, else as two."""
+        kernel on an fp32 or bf16 base with L <= 16, d_v <= 128 and at least
+        32 heads per SM, else as two."""
         import torch
 
         if kind == "append_read":
-            return 1 if self.S.dtype in (torch.float32, torch.bfloat16) and self.L <= 16 else 2
+            sms = torch.cuda.get_device_properties(self.S.device).multi_processor_count
+            one = (self.S.dtype in (torch.float32, torch.bfloat16) and self.L <= 16 and self.w.d_v <= 128
+                   and self.w.heads >= 32 * sms)
+            return 1 if one else 2
         return KERNELS_PER_CALL[kind]
 
     def plan(self):

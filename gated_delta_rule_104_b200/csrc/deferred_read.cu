@@ -415,8 +415,19 @@ static cudaError_t launch_append_read_split(const StepParams &p, const LogParams
     });
 }
 
+// The one-kernel form pays where each block has many heads to pipeline: its
+// first head's ReplayPrep is exposed once per launch, and with a few heads per
+// SM (or 256-row heads, whose ReplayPrep is twice as long) the two-kernel form,
+// whose prep grid covers every head at once, measured faster.
 bool fused_read_supported(const StepParams &p, int L, const PoolIdx &pool) {
-    return pool.slot == nullptr && (p.s_dt == DL_F32 || p.s_dt == DL_BF16) && prep_emax(L) == fused::EMAX;
+    if (pool.slot != nullptr || !(p.s_dt == DL_F32 || p.s_dt == DL_BF16) || prep_emax(L) != fused::EMAX ||
+        p.dv > 128)
+        return false;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return false;
+    return (long long)p.B * p.H >= (long long)fused::MIN_HEADS_PER_SM * sms;
 }
 
 cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, float *work, cudaStream_t st,
@@ -425,8 +436,11 @@ cudaError_t launch_append_read(const StepParams &p, const LogParams &lg, int n, 
     return dispatch(p, [&](auto st_t, auto it_t, auto dk_c, auto dv_c, auto ch_c) -> cudaError_t {
         using ST = decltype(st_t);
         using IT = decltype(it_t);
-        return launch_fused<IT, ST, decltype(dk_c)::value, decltype(dv_c)::value, decltype(ch_c)::value>(p, lg, n,
-                                                                                                         st);
+        constexpr int DV = decltype(dv_c)::value;
+        if constexpr (DV <= 128)
+            return launch_fused<IT, ST, decltype(dk_c)::value, DV, decltype(ch_c)::value>(p, lg, n, st);
+        else
+            return launch_append_read_split(p, lg, n, work, st, pool);
     });
 }
 

@@ -1,7 +1,8 @@
 // Shared-memory layout of the fused append-read kernel (deferred_read.cu,
 // append_read_fused_kernel), in host- and device-callable form, so that a
 // host program can replay the addresses the kernel forms and check them
-// against the regions below.
+// against the regions below. The kernel serves d_v <= 128 (d_v = 256 layouts
+// are laid out and replayed too, but the read takes its two-kernel form there).
 //
 // One persistent block per SM, in two roles that work on the block's heads
 // (batch heads blockIdx.x, blockIdx.x + gridDim.x, ...) in order:
@@ -40,9 +41,10 @@ constexpr int EMAX = 16;                  // log entries the fused kernel stages
 constexpr int ND = 8;                     // decode warps
 constexpr int NBUF = 3;                   // base buffers in flight per decode warp
 constexpr int UNIT_BYTES = 4096;          // one bulk copy: 32 lanes x 8 rows' 16-byte slices
+constexpr int MIN_HEADS_PER_SM = 32;      // the one-kernel read is used from this many heads per SM
 // prep warps at most: 12, or 8 where ReplayPrep holds more per lane (fp32
-// inputs, or d_v = 256), so that the block's registers (65536 over its
-// threads) leave no prep warp spilling
+// inputs), so that the block's registers (65536 over its threads) leave no
+// prep warp spilling
 DL_HD constexpr int np_max(int IB, int DV) { return (IB == 4 || DV > 128) ? 8 : 12; }
 constexpr int SMEM_LIMIT = 227 * 1024;    // dynamic shared memory a block may request
 constexpr int ALIGN_SLACK = 128;          // the kernel aligns its base up to 128 bytes

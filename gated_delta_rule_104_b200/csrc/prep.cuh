@@ -67,20 +67,6 @@ __device__ __forceinline__ void prep_head(const IT *__restrict__ q, const IT *__
         }
     }
     cp_async_commit();
-    // With at most 16 entries of 2-byte values (d_v <= 128: 2 registers per
-    // entry), every entry's values for w are loaded now, with the keys, and
-    // consumed at the end: the head then needs one round trip to memory
-    // instead of one more per batch of 8 entries.
-    constexpr bool EARLY_V = EMAX == 16 && sizeof(IT) == 2 && DV <= 128;
-    using VC = RawCopy<RV, IT>;
-    VC vraw[EARLY_V ? EMAX : 1];
-    if constexpr (EARLY_V) {
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e < n) vraw[e].load_hint(log_v + (lrow + e) * DV + r0, keep);
-            else if (e == n) vraw[e].load(v + head * DV + r0);
-        }
-    }
     // Everything else the head needs is loaded next, all loads before the first
     // store that consumes one (a warp issues in order: a store waiting on its
     // load would hold back every load behind it).
@@ -257,23 +243,11 @@ __device__ __forceinline__ void prep_head(const IT *__restrict__ q, const IT *__
     float w[RV];
 #pragma unroll
     for (int r = 0; r < RV; ++r) w[r] = 0.f;
-    if constexpr (EARLY_V) {
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e <= n) {
-                const float se = fs[e];
-                float ve[RV];
-                vraw[e].widen(ve);
-#pragma unroll
-                for (int r = 0; r < RV; ++r) w[r] = fmaf(se, ve[r], w[r]);
-            }
-        }
-    }
-    // Otherwise entries in batches of VB: a batch's raw words are all loaded
-    // before any is widened (a widening right after its load would stall the
-    // loads behind it).
+    // Entries in batches of VB: a batch's raw words are all loaded before any is
+    // widened (a widening right after its load would stall the loads behind it).
     constexpr int VB = 8;
-    for (int e0 = 0; !EARLY_V && e0 <= n; e0 += VB) {
+    using VC = RawCopy<RV, IT>;
+    for (int e0 = 0; e0 <= n; e0 += VB) {
         VC raw[VB];
 #pragma unroll
         for (int i = 0; i < VB; ++i) {
