@@ -103,8 +103,8 @@ cudaError_t launch_append_read_noalloc(const StepParams &p, const LogParams &lg,
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur,
                          cudaStream_t st, const PoolIdx &pool = PoolIdx{}, int part = POOL_MERGE_FULL);
 // The same merge on the tcgen05 tensor cores (merge_tc.cu), for the cases
-// merge_tc_supported() accepts: an fp32 base, d_k = 128, d_v a multiple of
-// 128, 1..16 entries in all, no slot pool.
+// merge_tc_supported() accepts: an fp32 or int8 base, d_k = 128, d_v a
+// multiple of 128, 1..16 entries in all, no slot pool.
 bool merge_tc_supported(const StepParams &p, int n_log, bool with_cur, const PoolIdx &pool);
 cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st);
 // The tensor-core kernels' fault word (bit 0: a bounded wait ran out), read

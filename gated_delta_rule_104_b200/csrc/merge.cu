@@ -683,8 +683,8 @@ static cudaError_t launch_merge_nb(const StepParams &p, const LogParams &lg, int
 
 cudaError_t launch_merge(const StepParams &p, const LogParams &lg, int n_log, bool with_cur, cudaStream_t st,
                          const PoolIdx &pool, int part) {
-    // An fp32 base with d_k = 128 and at most 16 entries to merge goes to the
-    // tcgen05 kernel (merge_tc.cu); every other case runs here.
+    // An fp32 or int8 base with d_k = 128 and at most 16 entries to merge goes
+    // to the tcgen05 kernel (merge_tc.cu); every other case runs here.
     if (merge_tc_supported(p, n_log, with_cur, pool)) return launch_merge_tc(p, lg, n_log, with_cur, st);
     // The input dtype and d_v are run-time arguments of the merge kernel (they
     // only change staging and the grid), which keeps instantiations few.

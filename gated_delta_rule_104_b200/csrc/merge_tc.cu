@@ -1,7 +1,16 @@
-// Merge of the bounded log into an fp32 base on the 5th-generation tensor
-// cores (DeltaLog page, "Core Mechanism: Base + Log", the merge phase: the
-// base absorbs every update the log holds and the log starts empty again),
-// alone or fused with one step's read.
+// Merge of the bounded log into an fp32 or int8 base on the 5th-generation
+// tensor cores (DeltaLog page, "Core Mechanism: Base + Log", the merge phase:
+// the base absorbs every update the log holds and the log starts empty
+// again), alone or fused with one step's read.
+//
+// An int8 base (codes with one fp32 scale per row; the low-precision base of
+// the DAMP abstract) takes the same path: the loader brings the unit's codes
+// by one TMA box into the tile's last column chunk and its row scales by a
+// bulk copy; each thread widens its row (code * scale, fp32) into the fp32
+// tile as it makes its pass over the row, the tensor cores reading each half
+// of the tile once the group has written it; the merged row is rounded back
+// (scale = max|row| / 127, codes to nearest, ties to even) and stored from
+// registers.
 //
 // The arithmetic is the log-decay form of merge.cu (same symbols): for a
 // block of n <= 16 entries with decays a_i, keys k_i, values v_i, strengths
@@ -111,16 +120,16 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) 
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
 
-template <class IT, int KIND, bool WITH_CUR, int NWG>
+template <class IT, int KIND, bool WITH_CUR, int NWG, bool Q8>
 __global__ void __launch_bounds__(threads_for(NWG), 1)
 merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_st,
                 const IT *__restrict__ log_k, const IT *__restrict__ log_v, const IT *__restrict__ log_b,
                 const IT *__restrict__ log_a, const float *__restrict__ log_x, int L, int n_log,
                 const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                 const IT *__restrict__ beta, const IT *__restrict__ a, float *__restrict__ o, int DV,
-                long long units) {
+                long long units, int8_t *__restrict__ codes, float *__restrict__ i8_scales) {
     constexpr bool CHAN = Rule<KIND>::CHAN, DELTA = Rule<KIND>::DELTA;
-    constexpr Layout LY{sizeof(IT), CHAN, NWG};
+    constexpr Layout LY{sizeof(IT), CHAN, NWG, Q8};
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + LY.off_bar());
@@ -165,7 +174,9 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
             tc::tma_prefetch_desc(&map_st);
         }
         constexpr uint32_t KB = DK * sizeof(IT), VB = ROWS * sizeof(IT);  // one entry's key / value-tile bytes
-        const uint32_t tx = (uint32_t)LY.tile() + (uint32_t)nb * (KB * (CHAN ? 2 : 1) + VB) + (WITH_CUR ? KB : 0);
+        // the unit's base: the fp32 tile, or the int8 codes (ROWS x DK bytes) and row scales
+        constexpr uint32_t BASE_TX = Q8 ? (uint32_t)(ROWS * DK + ROWS * 4) : (uint32_t)LY.tile();
+        const uint32_t tx = BASE_TX + (uint32_t)nb * (KB * (CHAN ? 2 : 1) + VB) + (WITH_CUR ? KB : 0);
         for (int i = 0; i < n_mine; ++i) {
             const int s = i % NS;
             if (i >= NS && !wait_bar(B_FREE(s), (uint32_t)((i / NS - 1) & 1), abort)) break;
@@ -179,9 +190,13 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
             if (lane == 0) tc::mbar_arrive_expect_tx(full, tx);
             __syncwarp();
             uint8_t *rk = st + LY.off_raw_k(), *ra = st + LY.off_raw_a(), *rv = st + LY.off_raw_v();
-            if (lane < NCHUNK)
+            if constexpr (Q8) {
+                if (lane == 0) tc::tma_load_2d(st + LY.off_codes(), &map_s, 0, (int)(un.head * DV + un.row0), full);
+                if (lane == 1) tc::bulk_load(st + LY.off_scl(), i8_scales + un.head * DV + un.row0, ROWS * 4, full);
+            } else if (lane < NCHUNK) {
                 tc::tma_load_2d(st + LY.off_tile() + lane * (ROWS * 128), &map_s, lane * CHUNK,
                                 (int)(un.head * DV + un.row0), full);
+            }
             if (lane == NCHUNK && n_log > 0) tc::bulk_load(rk, log_k + lrow * DK, (uint32_t)n_log * KB, full);
             if (CHAN && lane == NCHUNK + 1 && n_log > 0)
                 tc::bulk_load(ra, log_a + lrow * DK, (uint32_t)n_log * KB, full);
@@ -223,11 +238,13 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     if (!wait_bar(B_KH(w), par, abort)) break;
                     tc::tc_fence_after();
                     const uint32_t tile = tc::smem_u32(sm + LY.stage(s) + LY.off_tile());
+                    if constexpr (!Q8) {  // the TMA tile is in place already
 #pragma unroll
-                    for (int kk = 0; kk < DK / 8; ++kk) {
-                        const uint64_t ad = tc::smem_desc(tile + g_a_start(kk), 16, 1024, tc::SWZ_128);
-                        const uint64_t bd = tc::smem_desc(kh + g_b_start(kk), 16, 1024, tc::SWZ_128);
-                        tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
+                        for (int kk = 0; kk < DK / 8; ++kk) {
+                            const uint64_t ad = tc::smem_desc(tile + g_a_start(kk), 16, 1024, tc::SWZ_128);
+                            const uint64_t bd = tc::smem_desc(kh + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                            tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
+                        }
                     }
                     bool ok = true;
 #pragma unroll
@@ -237,6 +254,15 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                             break;
                         }
                         tc::tc_fence_after();
+                        if constexpr (Q8) {  // the half of the fp32 tile the group has just written
+#pragma unroll
+                            for (int kq = 0; kq < DK / 16; ++kq) {
+                                const int kk = h * (DK / 16) + kq;
+                                const uint64_t ad = tc::smem_desc(tile + g_a_start(kk), 16, 1024, tc::SWZ_128);
+                                const uint64_t bd = tc::smem_desc(kh + g_b_start(kk), 16, 1024, tc::SWZ_128);
+                                tc::mma_ss_tf32(tw + COL_G, ad, bd, ID_G, kk > 0);
+                            }
+                        }
 #pragma unroll
                         for (int kq = 0; kq < DK / 16; ++kq) {
                             const int kk = h * (DK / 16) + kq;
@@ -365,12 +391,32 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
             //    time (the second half once G has read the first); for the fused
             //    read also (S o gamma) . q
             float oacc = 0.f;
+            // an int8 base: this row's scale; chunk ch's 32 codes are pieces 2ch and
+            // 2ch + 1 of the row in the code box, read before the chunk's fp32
+            // columns are written (chunk 3's columns overwrite the row's codes)
+            const float rs = Q8 ? *reinterpret_cast<const float *>(st + LY.off_scl() + 4 * r) : 0.f;
             auto row_chunk = [&](int ch, uint32_t (&lo)[32]) {
                 uint32_t y[32];
+                uint4 cw[2];
+                if constexpr (Q8) {
+                    cw[0] = *reinterpret_cast<const uint4 *>(st + LY.off_codes() + code_off(r, 2 * ch));
+                    cw[1] = *reinterpret_cast<const uint4 *>(st + LY.off_codes() + code_off(r, 2 * ch + 1));
+                }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int col = ch * CHUNK + 4 * u;
-                    const float4 x = *reinterpret_cast<const float4 *>(tile + tile_off(r, col));
+                    float4 x;
+                    if constexpr (Q8) {  // codes 4u .. 4u + 3 of the chunk, widened and scaled
+                        const uint4 &c4 = cw[u / 4];
+                        const uint32_t wd = (u % 4) == 0 ? c4.x : (u % 4) == 1 ? c4.y : (u % 4) == 2 ? c4.z : c4.w;
+                        x = make_float4((float)(int8_t)(wd & 0xff) * rs, (float)(int8_t)((wd >> 8) & 0xff) * rs,
+                                        (float)(int8_t)((wd >> 16) & 0xff) * rs, (float)(int8_t)(wd >> 24) * rs);
+                        if constexpr (DELTA) {  // the fp32 tile is the A operand of G's tile part
+                            DL_GUARD(tile + tile_off(r, col), 16) *reinterpret_cast<float4 *>(tile + tile_off(r, col)) = x;
+                        }
+                    } else {
+                        x = *reinterpret_cast<const float4 *>(tile + tile_off(r, col));
+                    }
                     const float4 gv = *reinterpret_cast<const float4 *>(gam + col);
                     const float4 sg = make_float4(x.x * gv.x, x.y * gv.y, x.z * gv.z, x.w * gv.w);
                     y[4 * u + 0] = __float_as_uint(sg.x);
@@ -399,6 +445,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     tc::tmem_st32(trow + COL_LO + CHUNK, lo);
                     tc::tmem_wait_st();
                     tc::tc_fence_before();
+                    if constexpr (Q8) tc::fence_async_smem();  // the tile's first half is read by the tensor cores
                     tc::named_sync(bar_id, 128);
                     if (ct == 0) tc::mbar_arrive(B_LO(w));  // first half
                 }
@@ -413,6 +460,7 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
                     tc::tmem_st32(trow + COL_LO + CHUNK, lo);
                     tc::tmem_wait_st();
                     tc::tc_fence_before();
+                    if constexpr (Q8) tc::fence_async_smem();  // and its second half
                     tc::named_sync(bar_id, 128);
                     if (ct == 0) tc::mbar_arrive(B_LO(w));  // second half
                 }
@@ -515,30 +563,62 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
             //    still reading suffices, at the next chunk and at the unit's end.
             if (!wait_bar(B_D(w), par, abort)) break;
             tc::tc_fence_after();
+            if constexpr (Q8) {
+                // an int8 base: the row's max over two reads of its 128 columns, then
+                // its codes (16-byte stores of the row's own 128 bytes) and its scale
+                float mx = 0.f;
 #pragma unroll 1
-            for (int ch = 0; ch < NCHUNK; ++ch) {
-                uint32_t d[32];
-                tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
-                uint8_t *buf = sm + LY.group(w) + LY.out_buf(quad, ch & 1);
-                if (ch >= 1 && lane == 0) tc::bulk_wait_read<1>();
-                __syncwarp();
-                tc::tmem_wait_ld();
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    uint32_t d[32];
+                    tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    DL_GUARD(buf + tile_off(lane, 4 * u), 16) *reinterpret_cast<uint4 *>(buf + tile_off(lane, 4 * u)) =
-                        make_uint4(d[4 * u + 0], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
-                tc::fence_async_smem();  // the staging tile is read by the TMA store
-                __syncwarp();
-                if (lane == 0) {
-                    tc::tma_store_2d(&map_st, ch * CHUNK, (int)(un.head * DV + un.row0 + 32 * quad), buf);
-                    tc::bulk_commit();
+                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(__uint_as_float(d[i])));
                 }
+                const float sc = i8_scale(mx);
+                int8_t *crow = codes + (un.head * DV + un.row0 + r) * (long long)DK;
+#pragma unroll 1
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    uint32_t d[32];
+                    tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
+                    tc::tmem_wait_ld();
+                    uint32_t wd[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        wd[i] = (uint32_t)(i8_code(__uint_as_float(d[4 * i + 0]), sc) & 0xff) |
+                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 1]), sc) & 0xff) << 8) |
+                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 2]), sc) & 0xff) << 16) |
+                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 3]), sc) & 0xff) << 24);
+                    st_stream(crow + ch * CHUNK, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+                    st_stream(crow + ch * CHUNK + 16, make_uint4(wd[4], wd[5], wd[6], wd[7]));
+                }
+                i8_scales[un.head * DV + un.row0 + r] = sc;
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    uint32_t d[32];
+                    tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
+                    uint8_t *buf = sm + LY.group(w) + LY.out_buf(quad, ch & 1);
+                    if (ch >= 1 && lane == 0) tc::bulk_wait_read<1>();
+                    __syncwarp();
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        DL_GUARD(buf + tile_off(lane, 4 * u), 16) *reinterpret_cast<uint4 *>(buf + tile_off(lane, 4 * u)) =
+                            make_uint4(d[4 * u + 0], d[4 * u + 1], d[4 * u + 2], d[4 * u + 3]);
+                    tc::fence_async_smem();  // the staging tile is read by the TMA store
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_store_2d(&map_st, ch * CHUNK, (int)(un.head * DV + un.row0 + 32 * quad), buf);
+                        tc::bulk_commit();
+                    }
+                }
+                // the warp's quarter of Khat, rewritten by the next unit's key side,
+                // is free once the third store has read it; the fourth may still be
+                // reading the warp's quarter of F, which the next F write waits for
+                if (lane == 0) tc::bulk_wait_read<1>();
+                __syncwarp();
             }
-            // the warp's quarter of Khat, rewritten by the next unit's key side,
-            // is free once the third store has read it; the fourth may still be
-            // reading the warp's quarter of F, which the next F write waits for
-            if (lane == 0) tc::bulk_wait_read<1>();
-            __syncwarp();
             tc::tc_fence_before();  // [COL_SG, +128) is rewritten by the group's next unit
         }
         if (lane == 0) tc::bulk_wait_all();  // the warp's last stores have landed
@@ -590,12 +670,27 @@ cudaError_t state_map(CUtensorMap *m, void *S, unsigned long long rows, unsigned
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <class IT, int KD, bool WC>
+// The int8 codes [rows, 128] as a tensor map of 128 x 128 boxes (one unit's
+// codes; 128-byte rows under 128-byte swizzle).
+cudaError_t code_map(CUtensorMap *m, void *codes, unsigned long long rows) {
+    EncodeTiledFn fn = encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)DK, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)DK};
+    const cuuint32_t box[2] = {(cuuint32_t)DK, (cuuint32_t)ROWS};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <class IT, int KD, bool WC, bool Q8>
 cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cudaStream_t st) {
-    constexpr int NWG = groups_for(sizeof(IT), Rule<KD>::CHAN);
-    constexpr Layout LY{sizeof(IT), Rule<KD>::CHAN, NWG};
+    constexpr int NWG = groups_for(sizeof(IT), Rule<KD>::CHAN, Q8);
+    constexpr Layout LY{sizeof(IT), Rule<KD>::CHAN, NWG, Q8};
     static_assert(LY.request() <= SMEM_LIMIT, "layout fits the shared memory a block may request");
-    auto kern = merge_tc_kernel<IT, KD, WC, NWG>;
+    auto kern = merge_tc_kernel<IT, KD, WC, NWG, Q8>;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(kern), LY.request());
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -604,8 +699,17 @@ cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cud
     if (e != cudaSuccess) return e;
     const long long heads = (long long)p.B * p.H;
     CUtensorMap map, map_st;  // loads: 32 x 128 boxes; each warp's stores: 32 x 32 boxes
-    e = state_map(&map, p.S, (unsigned long long)heads * p.dv, CHUNK, ROWS);
-    if (e == cudaSuccess) e = state_map(&map_st, p.S, (unsigned long long)heads * p.dv, CHUNK, 32);
+    int8_t *codes = nullptr;
+    float *scales = nullptr;
+    if constexpr (Q8) {  // codes [heads * d_v, 128], then one fp32 scale per row
+        codes = static_cast<int8_t *>(p.S);
+        scales = reinterpret_cast<float *>(codes + heads * p.dv * DK);
+        e = code_map(&map, p.S, (unsigned long long)heads * p.dv);
+        map_st = map;  // not used: the rows are stored from registers
+    } else {
+        e = state_map(&map, p.S, (unsigned long long)heads * p.dv, CHUNK, ROWS);
+        if (e == cudaSuccess) e = state_map(&map_st, p.S, (unsigned long long)heads * p.dv, CHUNK, 32);
+    }
     if (e != cudaSuccess) return e;
     const long long units = heads * (p.dv / ROWS);
     const unsigned grid = (unsigned)std::min<long long>(units, sms);
@@ -613,7 +717,7 @@ cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cud
         map, map_st, static_cast<const IT *>(lg.k), static_cast<const IT *>(lg.v), static_cast<const IT *>(lg.beta),
         static_cast<const IT *>(lg.a), lg.x, lg.L, n_log, static_cast<const IT *>(p.q), static_cast<const IT *>(p.k),
         static_cast<const IT *>(p.v), static_cast<const IT *>(p.beta), static_cast<const IT *>(p.a), p.o, p.dv,
-        units);
+        units, codes, scales);
     return cudaGetLastError();
 }
 
@@ -621,7 +725,7 @@ cudaError_t launch_tc_t(const StepParams &p, const LogParams &lg, int n_log, cud
 
 bool merge_tc_supported(const StepParams &p, int n_log, bool with_cur, const PoolIdx &pool) {
     const long long rows = (long long)p.B * p.H * p.dv;
-    return pool.slot == nullptr && p.s_dt == DL_F32 && p.dk == DK && p.dv % ROWS == 0 &&
+    return pool.slot == nullptr && (p.s_dt == DL_F32 || p.s_dt == DL_I8) && p.dk == DK && p.dv % ROWS == 0 &&
            n_log + (with_cur ? 1 : 0) <= NB && n_log + (with_cur ? 1 : 0) >= 1 && rows < (1LL << 31) &&
            encoder() != nullptr;
 }
@@ -630,8 +734,12 @@ cudaError_t launch_merge_tc(const StepParams &p, const LogParams &lg, int n_log,
     auto with_kind = [&](auto it_t, auto kd_c) -> cudaError_t {
         using IT = decltype(it_t);
         constexpr int KD = decltype(kd_c)::value;
-        if (with_cur) return launch_tc_t<IT, KD, true>(p, lg, n_log, st);
-        return launch_tc_t<IT, KD, false>(p, lg, n_log, st);
+        if (p.s_dt == DL_I8) {
+            if (with_cur) return launch_tc_t<IT, KD, true, true>(p, lg, n_log, st);
+            return launch_tc_t<IT, KD, false, true>(p, lg, n_log, st);
+        }
+        if (with_cur) return launch_tc_t<IT, KD, true, false>(p, lg, n_log, st);
+        return launch_tc_t<IT, KD, false, false>(p, lg, n_log, st);
     };
     auto with_it = [&](auto it_t) -> cudaError_t {
         if (p.kind == DL_RWKV6) return with_kind(it_t, std::integral_constant<int, DL_RWKV6>{});

@@ -57,6 +57,9 @@ struct Layout {
     size_t in_size;  // bytes of one input element (2: bf16, 4: fp32)
     bool chan;       // one decay per key channel (else per entry)
     int nwg;         // compute groups
+    bool q8 = false; // an int8 base: the unit's codes land in the tile's last column chunk (box 3,
+                     // rows of 128 codes under the same 128-byte swizzle) and its row scales in
+                     // the stage's scale region; the compute group writes the widened fp32 tile
 
     // ---- one stage
     DL_HD constexpr size_t tile() const { return (size_t)ROWS * DK * 4; }  // 64 KiB, 4 column chunks of 16 KiB
@@ -71,7 +74,10 @@ struct Layout {
     DL_HD constexpr size_t off_raw_v() const { return off_raw_a() + raw_a(); }
     DL_HD constexpr size_t off_raw_q() const { return off_raw_v() + raw_v(); }
     DL_HD constexpr size_t off_sc() const { return off_raw_q() + raw_q(); }
-    DL_HD constexpr size_t stage_bytes() const { return round_up(off_sc() + sc_floats() * 4, 1024); }
+    DL_HD constexpr size_t off_scl() const { return off_sc() + sc_floats() * 4; }  // int8 row scales [128]
+    DL_HD constexpr size_t scl_bytes() const { return q8 ? (size_t)ROWS * 4 : 0; }
+    DL_HD constexpr size_t off_codes() const { return off_tile() + (size_t)(NCHUNK - 1) * ROWS * 128; }
+    DL_HD constexpr size_t stage_bytes() const { return round_up(off_scl() + scl_bytes(), 1024); }
     DL_HD constexpr size_t stage(int s) const { return (size_t)s * stage_bytes(); }
 
     // ---- one compute group's regions (from the group's base)
@@ -150,9 +156,14 @@ DL_HD constexpr uint32_t kh_off(int n, int c) {
 DL_HD constexpr uint32_t ff_off(int c, int j) { return swz128((uint32_t)(c * 128 + j * 4)); }
 // Groups the launch can afford: two when their regions fit beside the
 // two stages, else one.
-DL_HD constexpr int groups_for(size_t in_size, bool chan) {
-    return Layout{in_size, chan, 2}.request() <= SMEM_LIMIT ? 2 : 1;
+DL_HD constexpr int groups_for(size_t in_size, bool chan, bool q8 = false) {
+    return Layout{in_size, chan, 2, q8}.request() <= SMEM_LIMIT ? 2 : 1;
 }
+// Byte offset inside the int8 code box (box 3 of the tile) of the 16-code
+// piece j (codes 16j..16j+15) of row r: rows 128 bytes apart, pieces permuted
+// by the same 128-byte swizzle, so row r's codes stay inside row r's 128 bytes
+// of the box (which its own fp32 columns 96..127 overwrite last).
+DL_HD constexpr uint32_t code_off(int r, int j) { return swz128((uint32_t)(r * 128 + j * 16)); }
 
 }  // namespace mtc
 }  // namespace dl

@@ -1,7 +1,10 @@
 // Host replay of every shared-memory, tensor-memory and global address the
 // tensor-core merge kernel (gated_delta_rule_104_b200/csrc/merge_tc.cu)
 // forms, for every instantiation (input element size, channel or head decay,
-// delta rule or RWKV6, fused read or not) and every entry count it accepts.
+// delta rule or RWKV6, fused read or not, fp32 or int8 base) and every entry
+// count it accepts. With an int8 base it also checks that each thread reads
+// its row's codes before its own fp32 columns overwrite them, and that no
+// thread writes over another row's codes.
 // It uses the same layout functions as the kernel (merge_tc_layout.h) and
 // walks the kernel's loops with their bounds, checking that each access lies
 // inside its region, is aligned for its width, that regions do not overlap,
@@ -42,15 +45,16 @@ struct Region {
 
 struct Replay {
     size_t in_size;
-    bool chan, delta, with_cur;
+    bool chan, delta, with_cur, q8;
     Layout ly;
     std::vector<Region> regions;
 
-    Replay(size_t in, bool ch, bool de, bool wc)
-        : in_size(in), chan(ch), delta(de), with_cur(wc), ly{in, ch, groups_for(in, ch)} {
+    Replay(size_t in, bool ch, bool de, bool wc, bool q)
+        : in_size(in), chan(ch), delta(de), with_cur(wc), q8(q), ly{in, ch, groups_for(in, ch, q), q} {
         for (int s = 0; s < NS; ++s) {
             const std::string p = "stage" + std::to_string(s) + ".";
             add(p + "tile", ly.stage(s) + ly.off_tile(), ly.tile());
+            if (q8) add(p + "scl", ly.stage(s) + ly.off_scl(), ly.scl_bytes());
             add(p + "raw_k", ly.stage(s) + ly.off_raw_k(), ly.raw_k());
             if (chan) add(p + "raw_a", ly.stage(s) + ly.off_raw_a(), ly.raw_a());
             add(p + "raw_v", ly.stage(s) + ly.off_raw_v(), ly.raw_v());
@@ -72,8 +76,8 @@ struct Replay {
     }
     std::string tag() const {
         char b[96];
-        std::snprintf(b, sizeof b, "in%zu %s %s %s", in_size, chan ? "chan" : "head", delta ? "delta" : "rwkv6",
-                      with_cur ? "fused" : "merge");
+        std::snprintf(b, sizeof b, "in%zu %s %s %s %s", in_size, chan ? "chan" : "head", delta ? "delta" : "rwkv6",
+                      with_cur ? "fused" : "merge", q8 ? "int8 base" : "fp32 base");
         return b;
     }
     void add(const std::string &name, size_t off, size_t bytes) {
@@ -128,9 +132,17 @@ struct Replay {
         for (int s = 0; s < NS; ++s) {
             const std::string p = "stage" + std::to_string(s) + ".";
             size_t tx = 0;
-            for (int ch = 0; ch < NCHUNK; ++ch) {
-                acc(p + "tile", ch * ROWS * 128, ROWS * 128, 1024, "TMA box");
-                tx += ROWS * 128;
+            if (q8) {  // the codes' one TMA box into the tile's last column chunk, the scales by a bulk copy
+                if (ly.off_codes() - ly.off_tile() != (size_t)(NCHUNK - 1) * ROWS * 128) fail("code box offset", tag());
+                acc(p + "tile", ly.off_codes() - ly.off_tile(), ROWS * DK, 1024, "code TMA box");
+                tx += ROWS * DK;
+                acc(p + "scl", 0, ROWS * 4, 16, "row scales");
+                tx += ROWS * 4;
+            } else {
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    acc(p + "tile", ch * ROWS * 128, ROWS * 128, 1024, "TMA box");
+                    tx += ROWS * 128;
+                }
             }
             // (lanes 16 + e copy entry e's value tile: every entry has a lane)
             if (nb > 16) fail("more entries than value-copy lanes", tag());
@@ -151,7 +163,8 @@ struct Replay {
                 bulk(p + "raw_q", raw_q_off(0, in_size), KB, "step query");
             }
             // the byte count the loader expects (merge_tc.cu: tx)
-            const size_t expect = ly.tile() + (size_t)nb * (KB * (chan ? 2 : 1) + VB) + (with_cur ? KB : 0);
+            const size_t base_tx = q8 ? (size_t)ROWS * DK + ROWS * 4 : ly.tile();
+            const size_t expect = base_tx + (size_t)nb * (KB * (chan ? 2 : 1) + VB) + (with_cur ? KB : 0);
             if (tx != expect) fail("expected bytes differ from the bytes copied", tag());
             if (tx >= (1u << 20)) fail("transaction count beyond the mbarrier's range", tag());
             for (int lane = 0; lane < 32; ++lane)
@@ -225,6 +238,31 @@ struct Replay {
                     acc(p + "sc", sc_x(nl, ct), 4, 4, "fused X row write");
                 }
                 for (int e = 0; e < NB; ++e) acc(gp + "cn", (NB + e) * 4, 4, 4, "F q read");
+            }
+            if (q8) {
+                acc(p + "scl", r * 4, 4, 4, "row scale");
+                // chunk ch reads pieces 2ch, 2ch + 1 of the row's codes, then writes its
+                // fp32 columns; no chunk may write a code byte that a later chunk reads
+                std::set<uint32_t> written;
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    for (int j = 2 * ch; j < 2 * ch + 2; ++j) {
+                        const uint32_t co = (uint32_t)(ly.off_codes() - ly.off_tile()) + code_off(r, j);
+                        acc(p + "tile", co, 16, 16, "code piece");
+                        for (uint32_t b = co; b < co + 16; ++b)
+                            if (written.count(b)) fail("a code piece read after its bytes were overwritten", tag());
+                        if (co < (uint32_t)(ly.off_codes() - ly.off_tile()) + r * 128u ||
+                            co + 16 > (uint32_t)(ly.off_codes() - ly.off_tile()) + (r + 1) * 128u)
+                            fail("a code piece outside its row's 128 bytes", tag());
+                    }
+                    if (delta)
+                        for (int col = ch * CHUNK; col < (ch + 1) * CHUNK; col += 4)
+                            for (uint32_t b = tile_off(r, col); b < tile_off(r, col) + 16; ++b) written.insert(b);
+                }
+                // what the tile's writes overwrite of other rows' codes: nothing
+                for (uint32_t b : written) {
+                    const uint32_t cb = (uint32_t)(ly.off_codes() - ly.off_tile());
+                    if (b >= cb && (b - cb) / 128 != (uint32_t)r) fail("a tile write over another row's codes", tag());
+                }
             }
             for (int col = 0; col < DK; col += 4) {
                 acc(p + "tile", tile_off(r, col), 16, 16, "tile piece");
@@ -319,12 +357,13 @@ int main(int argc, char **argv) {
         }
     }
     int cases = 0;
+    for (int q8 = 0; q8 < 2; ++q8)
     for (size_t in : {2, 4})
         for (int chan = 0; chan < 2; ++chan)
             for (int delta = 0; delta < 2; ++delta)
                 for (int wc = 0; wc < 2; ++wc) {
                     if (!delta && !chan) continue;  // RWKV6 has channel decay
-                    Replay rp(in, chan, delta, wc);
+                    Replay rp(in, chan, delta, wc, q8);
                     rp.layout_checks();
                     rp.descriptors();
                     for (int n_log = wc ? 0 : 1; n_log + wc <= NB; ++n_log) {

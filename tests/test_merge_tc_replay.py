@@ -38,10 +38,10 @@ def run(exe, *args):
 def test_every_access_in_bounds_and_aligned(replay):
     r = run(replay)
     assert r.returncode == 0, r.stdout[-3000:]
-    assert "192 cases, 0 failures" in r.stdout
+    assert "384 cases, 0 failures" in r.stdout
 
 
-@pytest.mark.parametrize("region", ["sc", "kh", "ff", "raw_k", "raw_v", "raw_q", "red", "qf", "gam", "tile"])
+@pytest.mark.parametrize("region", ["sc", "kh", "ff", "raw_k", "raw_v", "raw_q", "red", "qf", "gam", "tile", "scl"])
 def test_a_planted_four_byte_overrun_is_caught(replay, region):
     r = run(replay, "shrink", region, "4")
     assert r.returncode == 1, r.stdout[-2000:]
