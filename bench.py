@@ -352,9 +352,10 @@ class Launcher:
         import torch
 
         if kind == "append_read":
+            if not isinstance(self.S, torch.Tensor) or self.S.dtype not in (torch.float32, torch.bfloat16):
+                return 2  # an int8 base
             sms = torch.cuda.get_device_properties(self.S.device).multi_processor_count
-            one = (self.S.dtype in (torch.float32, torch.bfloat16) and self.L <= 16 and self.w.d_v <= 128
-                   and self.w.heads >= 32 * sms)
+            one = self.L <= 16 and self.w.d_v <= 128 and self.w.heads >= 32 * sms
             return 1 if one else 2
         return KERNELS_PER_CALL[kind]
 

@@ -15,8 +15,11 @@ to_i8_kernel(const ST *__restrict__ S, int8_t *__restrict__ codes, float *__rest
     const ST *row = S + r * dk;
     float m = 0.f;
     for (int c = lane; c < dk; c += 32) m = fmaxf(m, fabsf(to_f(row[c])));
-    const float sc = i8_scale(warp_max(m));
-    for (int c = lane; c < dk; c += 32) codes[r * dk + c] = (int8_t)i8_code(to_f(row[c]), sc);
+    const float sc = i8_scale(warp_max(m)), inv = i8_inv(sc);
+    if (i8_fast(sc))
+        for (int c = lane; c < dk; c += 32) codes[r * dk + c] = (int8_t)i8_code(to_f(row[c]), sc, inv);
+    else
+        for (int c = lane; c < dk; c += 32) codes[r * dk + c] = (int8_t)i8_code_div(to_f(row[c]), sc);
     if (lane == 0) scales[r] = sc;
 }
 

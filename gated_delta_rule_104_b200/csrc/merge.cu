@@ -604,16 +604,15 @@ merge_kernel(ST *__restrict__ S, const void *__restrict__ log_k, const void *__r
                         constexpr int CPR = DK / 16;  // 16-code chunks per row
                         for (int i = lane; i < 16 * CPR; i += 32) {
                             const int rl = i / CPR, c0 = (i % CPR) * 16;
-                            const float sc = wsc[warp * 16 + rl];
+                            const float sc = wsc[warp * 16 + rl], inv = i8_inv(sc);
+                            const bool fast = i8_fast(sc);
                             uint32_t wd[4];
 #pragma unroll
                             for (int qd = 0; qd < 4; ++qd) {
                                 const float4 x =
                                     *reinterpret_cast<const float4 *>(tile + TL::off(tr + rl, c0 + 4 * qd));
-                                wd[qd] = (uint32_t)(i8_code(x.x, sc) & 0xff) |
-                                         ((uint32_t)(i8_code(x.y, sc) & 0xff) << 8) |
-                                         ((uint32_t)(i8_code(x.z, sc) & 0xff) << 16) |
-                                         ((uint32_t)(i8_code(x.w, sc) & 0xff) << 24);
+                                wd[qd] = fast ? i8_pack4<true>(x.x, x.y, x.z, x.w, sc, inv)
+                                              : i8_pack4<false>(x.x, x.y, x.z, x.w, sc, inv);
                             }
                             st_stream(Sw + rl * DK + c0, make_uint4(wd[0], wd[1], wd[2], wd[3]));
                         }

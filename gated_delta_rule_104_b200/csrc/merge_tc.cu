@@ -575,23 +575,29 @@ merge_tc_kernel(const __grid_constant__ CUtensorMap map_s, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(__uint_as_float(d[i])));
                 }
-                const float sc = i8_scale(mx);
+                const float sc = i8_scale(mx), inv = i8_inv(sc);
                 int8_t *crow = codes + (un.head * DV + un.row0 + r) * (long long)DK;
+                auto store_codes = [&](auto fast_c) {
+                    constexpr bool FAST = decltype(fast_c)::value;
 #pragma unroll 1
-                for (int ch = 0; ch < NCHUNK; ++ch) {
-                    uint32_t d[32];
-                    tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
-                    tc::tmem_wait_ld();
-                    uint32_t wd[8];
+                    for (int ch = 0; ch < NCHUNK; ++ch) {
+                        uint32_t d[32];
+                        tc::tmem_ld32(trow + COL_SG + ch * CHUNK, d);
+                        tc::tmem_wait_ld();
+                        uint32_t wd[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        wd[i] = (uint32_t)(i8_code(__uint_as_float(d[4 * i + 0]), sc) & 0xff) |
-                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 1]), sc) & 0xff) << 8) |
-                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 2]), sc) & 0xff) << 16) |
-                                ((uint32_t)(i8_code(__uint_as_float(d[4 * i + 3]), sc) & 0xff) << 24);
-                    st_stream(crow + ch * CHUNK, make_uint4(wd[0], wd[1], wd[2], wd[3]));
-                    st_stream(crow + ch * CHUNK + 16, make_uint4(wd[4], wd[5], wd[6], wd[7]));
-                }
+                        for (int i = 0; i < 8; ++i)
+                            wd[i] = i8_pack4<FAST>(__uint_as_float(d[4 * i + 0]), __uint_as_float(d[4 * i + 1]),
+                                                   __uint_as_float(d[4 * i + 2]), __uint_as_float(d[4 * i + 3]), sc,
+                                                   inv);
+                        st_stream(crow + ch * CHUNK, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+                        st_stream(crow + ch * CHUNK + 16, make_uint4(wd[4], wd[5], wd[6], wd[7]));
+                    }
+                };
+                if (i8_fast(sc))
+                    store_codes(std::true_type{});
+                else
+                    store_codes(std::false_type{});
                 i8_scales[un.head * DV + un.row0 + r] = sc;
             } else {
 #pragma unroll 1
