@@ -325,8 +325,10 @@ def config_block(w, L, args):
                          "unfused": "DeltaLog deferred, separate merge every L steps",
                          "pool": "slot pool, staggered log fills (each step 1/L of the rows merge)"}[args.schedule],
             "global_batch": w.B * max(1, dist_env()[2]), "seq_len": w.T,
+            # (the reference arm prints the same block as this arm; its own timing,
+            # host wall time of the oracle, is stated in its cpu_baseline)
             "timing": ("launches issued directly, CUDA events around the decode"
-                       if getattr(args, "no_graph", False) or getattr(args, "impl", "ours") == "reference"
+                       if getattr(args, "no_graph", False)
                        else "one decode captured as a CUDA graph, replayed once per step between CUDA events; "
                             "per-kernel split from one more decode with events around each launch"),
             "l2": "inputs larger than L2 (state %d MiB per GPU), no flush" % (w.state_bytes() >> 20)}
