@@ -5,7 +5,7 @@ shared-memory write of the kernels (stores and cp.async destinations) checks
 that it lies inside the block's shared memory and is aligned, and a write
 that fails is skipped and reported in bit 1 of the fault word. This test
 runs the parity suites of the merge kernels (warp-MMA and tcgen05), the
-read, the pool step and the int8 base in a child process with that library
+read (both forms), the pool step and the int8 base in a child process with that library
 loaded; every case must still match the fp64 oracle, and after each one the
 guard must report nothing.
 """
@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SUITES = ["test_parity_gpu.py", "test_merge_tc_gpu.py", "test_pool_gpu.py", "test_i8_gpu.py"]
+SUITES = ["test_parity_gpu.py", "test_merge_tc_gpu.py", "test_pool_gpu.py", "test_i8_gpu.py", "test_fused_read_gpu.py"]
 
 
 def test_parity_suites_pass_under_the_index_guard():
